@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Benchmark of the WKV hot path on B200: prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole operator over one batch of synthetic inputs
+already resident in HBM.  The default workload is the RWKV-4 1.5B-shaped layer
+(B=8, T=1024, C=2048, float32 k/v/r/y, sigmoid gate, random initial state):
+one wkv_forward call per step.  Other workloads (layer_14b, stream_1m: one
+1024-token chunk with the state carried, decode: one wkv_step over 24 layers)
+are available with --workload.
+
+Timing: W warm-up steps, then exactly K steps between a barrier +
+synchronize on both sides, timed with CUDA events on the launching stream;
+the inputs rotate over two sets whose size exceeds the 126 MB L2, so no step
+finds its inputs in L2.  With N GPUs (torchrun) every rank runs the same
+per-GPU workload on its own seeds (independent sequences: no collective on the
+data path), the time is the max over ranks and the value is the total.
+
+`--impl reference` times the fp64 CPU oracle on the host cores on a bounded
+lane sample per step (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "WKV elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
+UNIT = "elements/s"
+SPEC_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["rwkv_wkv_recurrence_02_b200/csrc/wkv_chunk.cuh", "rwkv_wkv_recurrence_02_b200/csrc/wkv_common.cuh",
+                  "rwkv_wkv_recurrence_02_b200/csrc/wkv_seq.cuh", "rwkv_wkv_recurrence_02_b200/csrc/wkv_step.cuh",
+                  "rwkv_wkv_recurrence_02_b200/csrc/wkv_api.cu"]
+
+
+# ---------------------------------------------------------------------------
+# helpers that need no GPU (unit-tested on CPU)
+# ---------------------------------------------------------------------------
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def algorithmic_bytes(wl, B, T, C, layers=0) -> int:
+    """Bytes one call must move at minimum: every input element read once,
+    every output written once, the state read and written once, w and u once."""
+    eb = wl.elem_bytes
+    if layers:  # decode step over `layers` layers
+        n = layers * B * C
+        io = n * eb * (3 if wl.gate else 2) + n * eb          # k, v, (r) in; y out
+        return io + n * 12 * 2 + layers * C * 8               # state in + out; w, u
+    n = B * T * C
+    io = n * eb * (3 if wl.gate else 2) + n * eb
+    state = B * C * 12 * (2 if wl.random_state or wl.chunk else 1)
+    return io + state + C * 8
+
+
+def max_over_ranks(value: float, dist=None) -> float:
+    """Largest value across ranks (the slowest rank's time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    backend = dist.get_backend()
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Per-rank seed: each rank processes its own independent sequences."""
+    return base + 7919 * rank
+
+
+def whole_job_rate(units_per_rank_step: int, world: int, steps: int, seconds: float) -> float:
+    return units_per_rank_step * world * steps / seconds
+
+
+def load_traffic(workload: str):
+    """ncu DRAM bytes per launch recorded for this workload, if the kernel
+    sources are unchanged since they were taken."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            rec = json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("traffic_bytes_per_launch")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.period = period_s
+        self.stop_evt = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self.stop_evt.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                util = self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((time.time(), mhz, reasons, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.thread.start()
+        return self
+
+    def stop(self):
+        self.stop_evt.set()
+        if self.ok:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        src = inside if inside else [s for s in self.samples if s[0] >= t0 - 1.0]
+        if not src:
+            src = self.samples[-3:]
+        mhz = [s[1] for s in src]
+        reasons = sorted({name for s in src for name, bit in self.REASONS.items() if s[2] & bit})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(src), "in_window": bool(inside)}
+
+
+# ---------------------------------------------------------------------------
+# workloads on the GPU
+# ---------------------------------------------------------------------------
+class ForwardCase:
+    """Two resident input sets of one wkv_forward workload (rotated per step)."""
+
+    def __init__(self, wl, device, seed_base, T=None):
+        import torch
+        from rwkv_wkv_recurrence_02_b200 import inputs as I
+        self.wl = wl
+        T = (wl.chunk or wl.T) if T is None else T
+        self.B, self.T, self.C = wl.B, T, wl.C
+        self.sets = []
+        nsets = 2
+        one = algorithmic_bytes(wl, self.B, self.T, self.C)
+        while nsets * one < 2 * L2_BYTES:
+            nsets += 1
+        for i in range(nsets):
+            d = I.make_forward_inputs(wl, T=T, device=device, seed_offset=seed_base + i)
+            if wl.chunk and d["state"] is None:
+                d["state"] = I.fresh_state(self.B, self.C, device=device)
+            self.sets.append(d)
+        self.y = [torch.empty((self.B, T, self.C), dtype=wl.torch_dtype, device=device) for _ in range(nsets)]
+        self.s_out = [torch.empty((3, self.B, self.C), dtype=torch.float32, device=device) for _ in range(nsets)]
+        self.elements = self.B * self.T * self.C
+        self.bytes = algorithmic_bytes(wl, self.B, self.T, self.C)
+        self.launches_per_step = 1
+
+    def step(self, i, wkv, ws):
+        d = self.sets[i % len(self.sets)]
+        if self.wl.chunk:   # streaming: the state is carried in place
+            wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"], y=self.y[i % len(self.y)],
+                            state_out=d["state"], workspace=ws)
+        else:
+            wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"], y=self.y[i % len(self.y)],
+                            state_out=self.s_out[i % len(self.s_out)], workspace=ws)
+
+
+class DecodeCase:
+    """Decode: one wkv_step over all layers per step, inputs from the ring."""
+
+    def __init__(self, wl, device, seed_base):
+        import torch
+        from rwkv_wkv_recurrence_02_b200 import inputs as I
+        self.wl, self.I = wl, I
+        self.w, self.u = I.make_params(wl, layers=wl.layers, device=device, seed=wl.seed + seed_base)
+        self.k, self.v, self.r = I.make_decode_ring(wl, device=device)
+        self.state = I.fresh_state(wl.B, wl.C, layers=wl.layers, device=device)
+        self.y = torch.empty((wl.layers, wl.B, wl.C), dtype=wl.torch_dtype, device=device)
+        self.elements = wl.layers * wl.B * wl.C
+        self.bytes = algorithmic_bytes(wl, wl.B, 1, wl.C, layers=wl.layers)
+        self.launches_per_step = 1
+
+    def step(self, i, wkv, ws):
+        a = self.I.decode_ring_start(self.wl, i)
+        L = self.wl.layers
+        wkv.wkv_step(self.w, self.u, self.k[a:a + L], self.v[a:a + L], self.state,
+                     None if self.r is None else self.r[a:a + L], y=self.y)
+
+
+def make_case(name, device, seed_base):
+    from rwkv_wkv_recurrence_02_b200 import inputs as I
+    wl = I.WORKLOADS[name]
+    if wl.layers:
+        return DecodeCase(wl, device, seed_base)
+    return ForwardCase(wl, device, seed_base)
+
+
+def e2e_measure(case, wkv, ws, steps, warmup, stream):
+    """Same metric through the public API with host buffers: each step copies
+    its inputs from pinned host memory and reads the result back."""
+    import torch
+    if not isinstance(case, ForwardCase):
+        return None
+    d = case.sets[0]
+    host = {k: (None if v is None else v.to("cpu").pin_memory()) for k, v in d.items()}
+    y_host = torch.empty(case.y[0].shape, dtype=case.y[0].dtype).pin_memory()
+    s_host = torch.empty((3, case.B, case.C), dtype=torch.float32).pin_memory()
+    dev = {k: (None if v is None else torch.empty_like(v, device=d["k"].device)) for k, v in host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = y_host.numel() * y_host.element_size() + s_host.numel() * 4
+
+    def one():
+        for k, v in host.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        y, s = wkv.wkv_forward(dev["w"], dev["u"], dev["k"], dev["v"], dev["r"], dev["state"], y=case.y[0],
+                               state_out=case.s_out[0], workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+        s_host.copy_(s, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3
+    return {"seconds": sec, "steps": steps, "h2d": h2d, "d2h": d2h}
+
+
+def cpu_baseline_sample(workload: str, budget_s: float, max_reps: int = 1000):
+    """Time the oracle as it stands on this host's cores: whole steps of the
+    workload (or a lane sample of one) repeated for about `budget_s`."""
+    import numpy as np
+    import oracle
+    from rwkv_wkv_recurrence_02_b200 import inputs as I
+    wl = I.WORKLOADS[workload]
+    if wl.layers:
+        B, C = wl.B, wl.C
+        w, u = I.make_params(wl, layers=wl.layers)
+        k, v, r = I.make_decode_ring(wl)
+        L = wl.layers
+        st = np.zeros((L, 3, B, C))
+        st[:, 2] = -1e38
+        f = lambda x: x.float().numpy()
+        args = (f(w), f(u), f(k[:L]), f(v[:L]), st, f(r[:L]))
+        run = lambda: oracle.wkv_step(args[0], args[1], args[2], args[3], args[4], args[5])
+        elems, sample = L * B * C, f"one decode step of all {L} layers (B={B}, C={C})"
+    else:
+        T = wl.chunk or wl.T
+        B, C = wl.B, wl.C
+        # lanes so that one repetition takes a bounded time
+        lanes_total = B * C
+        cap = max(1, int(2e7 // T))
+        csub = C if lanes_total <= cap else max(1, cap // B)
+        d = I.make_forward_inputs(wl, T=T, C=csub)
+        f = lambda x: None if x is None else x.float().numpy()
+        st = None if d["state"] is None else d["state"].double().numpy()
+        run = lambda: oracle.wkv_forward(f(d["w"]), f(d["u"]), f(d["k"]), f(d["v"]), f(d["r"]), st)
+        elems = B * T * csub
+        sample = (f"full step B={B}, T={T}, C={C}" if csub == C else
+                  f"lane sample B={B}, T={T}, C={csub} of {C}")
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        run()
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= max_reps:
+            break
+    sec = time.perf_counter() - t0
+    return {"value": elems * reps / sec, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{sample}, repeated {reps}x over {sec:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+def config_of(case, workload, world):
+    wl = case.wl
+    cfg = {"workload": workload, "B": wl.B, "T": (wl.chunk or wl.T), "C": wl.C, "io_dtype": wl.dtype,
+           "gate": wl.gate, "parallelism": f"dp{world}" if world > 1 else "single",
+           "l2": "inputs rotate over sets totalling >2x the 126 MB L2"}
+    if wl.layers:
+        cfg.update({"layers": wl.layers, "T": 1, "steps_per_sequence": wl.steps})
+    if wl.chunk:
+        cfg["stream"] = f"one chunk of {wl.chunk} tokens per step, state carried in place"
+    return cfg
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import rwkv_wkv_recurrence_02_b200 as wkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    wkv.lib()
+    case = make_case(args.workload, device, rank_seed(0, rank))
+    ws = wkv.Workspace(device)
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        case.step(i, wkv, ws)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local).start()
+    time.sleep(0.05)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = time.time()
+    e0.record(stream)
+    for i in range(args.steps):
+        case.step(args.warmup + i, wkv, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None)
+    if ws.buf is not None and ws.status() != 0:
+        raise SystemExit("the GPU reported a cross-block wait timeout during the benchmark")
+    value = whole_job_rate(case.elements, world, args.steps, sec)
+    per_launch = sec / args.steps / case.launches_per_step
+    peak, peak_kind = load_peaks()
+    achieved = case.bytes / per_launch / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "io_dtype": case.wl.dtype,
+        "data": "synthetic (seeded; distributions of the workload definition)",
+        "config": config_of(case, args.workload, world),
+        "hbm_gbs": achieved, "hbm_pct_of_spec_8tbs": 100.0 * achieved / SPEC_HBM_GBS,
+        "hbm_pct_of_measured": 100.0 * achieved / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": case.bytes,
+                     "traffic": load_traffic(args.workload)},
+        "gpu_launches": args.steps * case.launches_per_step,
+        "clocks": clocks.summary(t0, t1),
+    }
+    if not args.no_e2e:
+        e = e2e_measure(case, wkv, ws, min(args.steps, args.e2e_steps), 2, stream)
+        if e is not None:
+            out["e2e"] = {"value": whole_job_rate(case.elements, world, e["steps"],
+                                                  max_over_ranks(e["seconds"], dist if world > 1 else None)),
+                          "unit": UNIT, "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                          "steps": e["steps"], "path": "pinned host -> wkv_forward (C ABI) -> pinned host"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_sample(args.workload, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle on the host cores, as it stands, on a bounded lane sample
+    per step, so that the whole run stays within a few minutes."""
+    import numpy as np
+    import oracle
+    from rwkv_wkv_recurrence_02_b200 import inputs as I
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = I.WORKLOADS[args.workload]
+    budget = args.ref_budget_s
+    f = lambda x: None if x is None else x.float().numpy()
+    if wl.layers:
+        raise SystemExit("--impl reference times the forward workloads")
+    T, B, C = (wl.chunk or wl.T), wl.B, wl.C
+    # calibrate: seconds per lane (all T tokens) with all cores busy
+    cal = I.make_forward_inputs(wl, B=1, T=T, C=min(C, 256))
+    t0 = time.perf_counter()
+    oracle.wkv_forward(f(cal["w"]), f(cal["u"]), f(cal["k"]), f(cal["v"]), f(cal["r"]),
+                       None if cal["state"] is None else cal["state"].double().numpy())
+    per_lane = (time.perf_counter() - t0) / min(C, 256)
+    lanes = int(max(1, min(B * C, budget / max(1, args.steps + args.warmup) / per_lane)))
+    csub = max(1, min(C, lanes))
+    d = I.make_forward_inputs(wl, B=1, T=T, C=csub)
+    st = None if d["state"] is None else d["state"].double().numpy()
+    args_np = (f(d["w"]), f(d["u"]), f(d["k"]), f(d["v"]), f(d["r"]), st)
+    for _ in range(args.warmup):
+        oracle.wkv_forward(*args_np)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.wkv_forward(*args_np)
+    sec = time.perf_counter() - t0
+    elems = T * csub
+    value = elems * args.steps / sec
+    sample = f"lane sample B=1, T={T}, C={csub} of the workload's B={B}, C={C} per step"
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "B": B, "T": T, "C": C, "io_dtype": wl.dtype, "gate": wl.gate},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="layer_1b5",
+                   choices=["tiny", "layer_1b5", "layer_14b", "stream_1m", "decode"])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--ref-budget-s", type=float, default=90.0)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,151 @@
+/*
+ * wkv.h -- C ABI of libwkv.so, the sm_100a (B200) implementation of the RWKV-4
+ * WKV time-mixing operator.
+ *
+ * The operator.  The article "RWKVアーキテクチャ徹底解説：Transformerに匹敵する
+ * 線形アテンションRNN" (youngju.dev) defines, per channel c of a sequence
+ * (section "コア計算", the explicit sum):
+ *
+ *   wkv_t = ( sum_{i<t} e^{-(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *         / ( sum_{i<t} e^{-(t-1-i) w + k_i}     + e^{u + k_t}     )
+ *
+ * with a per-channel decay w = exp(decay) > 0 and bonus u.  Its block diagram
+ * ("高レベル構造") gates the result, out_t = sigmoid(r_t) * wkv_t.  The same
+ * article evaluates the sum as a recurrence over a (numerator, denominator,
+ * running max) state ("リカレント定式化", "対数空間計算による数値安定性") in
+ * two modes that give the same result: a parallel pass over a chunk and one
+ * token at a time ("二重性：Transformerモード vs RNNモード").  The skill page
+ * "rwkv-architecture" (agnxi.com) streams a long document through chunks while
+ * carrying that state ("Process million-token sequences").
+ *
+ * Layouts (row-major, channel fastest, no padding):
+ *   k, v, r, y : (B, T, C) in the dtype `dtype` (all four the same)
+ *   w, u       : (C,) float32
+ *   state      : (3, B, C) float32 = {a, b, p}: numerator N = a*e^p and
+ *                denominator D = b*e^p of all tokens seen so far, before the
+ *                decay of the next step.  p is a natural-log exponent.  The
+ *                empty state is (0, 0, -1e38).  After a call, p follows the
+ *                running-max convention p <- max(p - w, k_t).
+ *
+ * Ownership and execution.  The caller allocates every buffer, in device
+ * memory of the current CUDA device.  The library allocates nothing and keeps
+ * no state except a per-device SM-count cache and a thread-local message for
+ * the last CUDA error.  Every call is asynchronous on `stream` (a cudaStream_t;
+ * NULL is the legacy default stream) and returns before the GPU finishes.
+ *
+ * Errors.  Every entry point returns a wkv_status.  Argument errors are found
+ * on the host before anything is launched; nothing is written then.
+ * WKV_ERR_CUDA reports a launch failure (wkv_last_cuda_error() has the text).
+ * Errors that only the GPU can see (a cross-block wait that ran out of time)
+ * are recorded in the workspace and read with wkv_workspace_status().
+ */
+#ifndef WKV_H_
+#define WKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+/* dtype of k, v, r and y.  w, u and the state are always float32. */
+typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;
+
+typedef enum {
+    WKV_OK = 0,
+    WKV_ERR_NULLPTR = -1,    /* a required pointer is NULL */
+    WKV_ERR_SHAPE = -2,      /* negative size, or B*T*C / L*B*C beyond 2^62 */
+    WKV_ERR_DTYPE = -3,      /* dtype is not a wkv_dtype */
+    WKV_ERR_ALIGN = -4,      /* pointer not aligned to its element (workspace: 256 B) */
+    WKV_ERR_ALIAS = -5,      /* an output overlaps an input or another output */
+    WKV_ERR_CUDA = -6,       /* CUDA launch error; see wkv_last_cuda_error() */
+    WKV_ERR_TIMEOUT = -7,    /* a cross-block wait on the GPU gave up (from wkv_workspace_status) */
+    WKV_ERR_WORKSPACE = -8   /* workspace NULL or smaller than wkv_forward_workspace_bytes() */
+} wkv_status;
+
+/*
+ * wkv_forward -- parallel ("GPT") mode over one chunk of T tokens.
+ *
+ * For every lane (b, c) it computes y[b,t,c] = sigmoid(r[b,t,c]) * wkv_t (no
+ * sigmoid factor when r is NULL) for t = 0..T-1, where the state `state_in`
+ * enters the sums as the tokens before the chunk: it contributes
+ * e^{-t w} * N_in to the numerator (and D_in to the denominator) of output t.
+ * state_out receives the state after token T-1, so feeding it back as the
+ * next chunk's state_in reproduces one unchunked pass.
+ *
+ *   B, T, C      sizes, each >= 0.  B == 0 or C == 0: nothing to do.  T == 0:
+ *                y untouched, state_out = state_in (or the empty state).
+ *   dtype        wkv_dtype of k, v, r, y.
+ *   w, u         (C,) float32 device arrays; w > 0 (not checked on the device).
+ *   k, v         (B,T,C) device arrays, required.
+ *   r            (B,T,C) device array, or NULL for no gate.
+ *   state_in     (3,B,C) float32 device array, or NULL for the empty state.
+ *   y            (B,T,C) device array, written.  Must not overlap any input.
+ *   state_out    (3,B,C) float32 device array, or NULL.  May be the same
+ *                pointer as state_in (in-place update); any other overlap
+ *                with an input or with y is WKV_ERR_ALIAS.
+ *   workspace    device scratch of at least wkv_forward_workspace_bytes(B,T,C,
+ *                dtype) bytes, 256-byte aligned, zeroed once by
+ *                wkv_workspace_init() before its first use and reusable by any
+ *                later call with any shape.  May be NULL when the required
+ *                size is 0.  Calls sharing a workspace must be ordered on the
+ *                GPU (same stream, or synchronised); they race otherwise.
+ *   stream       CUDA stream of the launch.
+ */
+int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype,
+                const float* w, const float* u,
+                const void* k, const void* v, const void* r,
+                const float* state_in, void* y, float* state_out,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of workspace wkv_forward needs for these sizes (0: none).  Returns 0
+ * for invalid sizes too; wkv_forward then reports the argument error. */
+size_t wkv_forward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype);
+
+/* Zero `bytes` bytes of a workspace on `stream` (cudaMemsetAsync).  Needed
+ * once after allocation, and again after wkv_workspace_status() reported an
+ * error. */
+int wkv_workspace_init(void* workspace, size_t bytes, cudaStream_t stream);
+
+/* Synchronise `stream`, then read the error word the kernels keep in the
+ * workspace: WKV_OK, or WKV_ERR_TIMEOUT if a wait for another block's partial
+ * result gave up (those outputs were written as NaN). */
+int wkv_workspace_status(const void* workspace, cudaStream_t stream);
+
+/*
+ * wkv_step -- RNN ("decode") mode: one token for L independent layers, each
+ * with B sequences, updating the state in place.  Equal to wkv_forward with
+ * T = 1 on each layer (the article's dual-mode section and the skill page's
+ * "RNN mode (sequential processing, same result)").
+ *
+ *   L, B, C      sizes, each >= 0 (any 0: nothing to do).
+ *   dtype        wkv_dtype of k, v, r, y.
+ *   w, u         (L, C) float32 device arrays, one row per layer.
+ *   k, v         (L, B, C) device arrays, required.
+ *   r            (L, B, C) device array, or NULL for no gate.
+ *   state        (L, 3, B, C) float32 device array, read and overwritten.
+ *   y            (L, B, C) device array, written.  No overlaps allowed.
+ *   stream       CUDA stream of the launch.
+ */
+int wkv_step(int64_t L, int64_t B, int64_t C, int dtype,
+             const float* w, const float* u,
+             const void* k, const void* v, const void* r,
+             float* state, void* y, cudaStream_t stream);
+
+/* Static English text for a wkv_status value. */
+const char* wkv_strerror(int status);
+
+/* Text of the last CUDA error seen by a call on this host thread ("" if none). */
+const char* wkv_last_cuda_error(void);
+
+/* ABI version of this header: 1. */
+int wkv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_H_ */

@@ -1,0 +1,233 @@
+"""B200 (sm_100a) RWKV-4 WKV operator: Python binding of libwkv.so.
+
+The binding only marshals arguments: every step of the operator runs in the
+CUDA kernels behind the C ABI declared in ``include/wkv.h``.  There is no CPU
+fallback; if ``libwkv.so`` is missing the import fails with instructions.
+
+Two layers:
+
+* ``lib()`` returns the ctypes handle; its functions carry the C names
+  (``wkv_forward``, ``wkv_step``, ``wkv_forward_workspace_bytes``, ...) and take
+  plain integers / pointers.
+* ``wkv_forward(...)`` and ``wkv_step(...)`` below take torch CUDA tensors,
+  allocate outputs and the workspace with torch when not given, pass
+  ``data_ptr()`` values and the current stream, and raise ``WkvError`` on a
+  non-zero status.
+"""
+import ctypes
+import os
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwkv.so")
+
+WKV_F32 = 0
+WKV_BF16 = 1
+STATUS = {
+    0: "WKV_OK", -1: "WKV_ERR_NULLPTR", -2: "WKV_ERR_SHAPE", -3: "WKV_ERR_DTYPE",
+    -4: "WKV_ERR_ALIGN", -5: "WKV_ERR_ALIAS", -6: "WKV_ERR_CUDA", -7: "WKV_ERR_TIMEOUT",
+    -8: "WKV_ERR_WORKSPACE",
+}
+# the functions include/wkv.h declares
+EXPORTS = ("wkv_forward", "wkv_forward_workspace_bytes", "wkv_workspace_init", "wkv_workspace_status",
+           "wkv_step", "wkv_strerror", "wkv_last_cuda_error", "wkv_abi_version")
+
+_lib = None
+_lock = threading.Lock()
+
+
+class WkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().wkv_strerror(status).decode()
+        if status == -6:
+            msg += ": " + lib().wkv_last_cuda_error().decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+def lib():
+    """ctypes handle of libwkv.so with argument types set."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run "
+                              "`python -c 'import __graft_entry__ as g; g.build()'` from the repository root "
+                              "(or rwkv_wkv_recurrence_02_b200/build_ext.py)")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, vp, i32, sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.wkv_forward.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.wkv_forward.restype = i32
+        L.wkv_forward_workspace_bytes.argtypes = [i64, i64, i64, i32]
+        L.wkv_forward_workspace_bytes.restype = sz
+        L.wkv_workspace_init.argtypes = [vp, sz, vp]
+        L.wkv_workspace_init.restype = i32
+        L.wkv_workspace_status.argtypes = [vp, vp]
+        L.wkv_workspace_status.restype = i32
+        L.wkv_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.wkv_step.restype = i32
+        L.wkv_strerror.argtypes = [i32]
+        L.wkv_strerror.restype = ctypes.c_char_p
+        L.wkv_last_cuda_error.argtypes = []
+        L.wkv_last_cuda_error.restype = ctypes.c_char_p
+        L.wkv_abi_version.argtypes = []
+        L.wkv_abi_version.restype = i32
+        _lib = L
+        return L
+
+
+# ---------------------------------------------------------------------------
+# torch front end (plumbing only)
+# ---------------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return WKV_F32
+    if t.dtype == torch.bfloat16:
+        return WKV_BF16
+    raise TypeError(f"k/v/r/y must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check(status, where):
+    if status != 0:
+        raise WkvError(status, where)
+
+
+def _need(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+class Workspace:
+    """Device scratch for wkv_forward's cross-block exchange, grown on demand.
+
+    Zeroed once per allocation (wkv_workspace_init); afterwards calls reuse it
+    without clearing.  Calls that share one Workspace must be ordered on the
+    GPU (the default: the current stream)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int, stream=None):
+        torch = _torch()
+        if nbytes == 0:
+            return None, 0
+        if self.buf is None or self.buf.numel() < nbytes:
+            dev = self.device if self.device is not None else torch.device("cuda", torch.cuda.current_device())
+            self.buf = torch.empty(int(nbytes) + 256, dtype=torch.uint8, device=dev)
+            _check(lib().wkv_workspace_init(self._aligned_ptr(), self.buf.numel() - 256, _stream_ptr(stream)),
+                   "wkv_workspace_init")
+        return self._aligned_ptr(), self.buf.numel() - 256
+
+    def _aligned_ptr(self):
+        p = self.buf.data_ptr()
+        return (p + 255) & ~255
+
+    def status(self, stream=None) -> int:
+        if self.buf is None:
+            return 0
+        return lib().wkv_workspace_status(self._aligned_ptr(), _stream_ptr(stream))
+
+    def reset(self, stream=None):
+        if self.buf is not None:
+            _check(lib().wkv_workspace_init(self._aligned_ptr(), self.buf.numel() - 256, _stream_ptr(stream)),
+                   "wkv_workspace_init")
+
+
+_workspaces = {}
+
+
+def default_workspace(device) -> Workspace:
+    key = (device.type, device.index)
+    ws = _workspaces.get(key)
+    if ws is None:
+        ws = _workspaces[key] = Workspace(device)
+    return ws
+
+
+def workspace_bytes(B: int, T: int, C: int, dtype_code: int) -> int:
+    return int(lib().wkv_forward_workspace_bytes(B, T, C, dtype_code))
+
+
+def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, want_state=True,
+                workspace: Workspace = None, stream=None):
+    """Parallel mode over one chunk.  k, v, r: (B, T, C) CUDA tensors (float32
+    or bfloat16); w, u: (C,) float32; state_in: (3, B, C) float32 or None.
+    Returns (y, state_out) (state_out None if want_state is False and none
+    was given).  state_out may be state_in for an in-place update."""
+    torch = _torch()
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    dev = k.device
+    if dev.type != "cuda":
+        raise ValueError("wkv_forward runs on CUDA tensors only")
+    code = _dtype_code(k)
+    _need(v, "v", (B, T, C), k.dtype, dev)
+    _need(r, "r", (B, T, C), k.dtype, dev)
+    _need(w, "w", (C,), torch.float32, dev)
+    _need(u, "u", (C,), torch.float32, dev)
+    _need(k, "k", (B, T, C), k.dtype, dev)
+    _need(state_in, "state_in", (3, B, C), torch.float32, dev)
+    if y is None:
+        y = torch.empty((B, T, C), dtype=k.dtype, device=dev)
+    _need(y, "y", (B, T, C), k.dtype, dev)
+    if state_out is None and want_state:
+        state_out = torch.empty((3, B, C), dtype=torch.float32, device=dev)
+    _need(state_out, "state_out", (3, B, C), torch.float32, dev)
+    ws = workspace if workspace is not None else default_workspace(dev)
+    ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
+    _check(lib().wkv_forward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
+                             _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, _stream_ptr(stream)), "wkv_forward")
+    return y, state_out
+
+
+def wkv_step(w, u, k, v, state, r=None, *, y=None, stream=None):
+    """RNN mode: one token for L layers.  w, u: (L, C) float32; k, v, r:
+    (L, B, C); state: (L, 3, B, C) float32, updated in place.  Returns y."""
+    torch = _torch()
+    if k.dim() != 3:
+        raise ValueError("k must be (L, B, C)")
+    Lr, B, C = k.shape
+    dev = k.device
+    if dev.type != "cuda":
+        raise ValueError("wkv_step runs on CUDA tensors only")
+    code = _dtype_code(k)
+    _need(v, "v", (Lr, B, C), k.dtype, dev)
+    _need(r, "r", (Lr, B, C), k.dtype, dev)
+    _need(w, "w", (Lr, C), torch.float32, dev)
+    _need(u, "u", (Lr, C), torch.float32, dev)
+    _need(state, "state", (Lr, 3, B, C), torch.float32, dev)
+    if y is None:
+        y = torch.empty((Lr, B, C), dtype=k.dtype, device=dev)
+    _need(y, "y", (Lr, B, C), k.dtype, dev)
+    _check(lib().wkv_step(Lr, B, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state), _ptr(y),
+                          _stream_ptr(stream)), "wkv_step")
+    return y

@@ -1,0 +1,328 @@
+// wkv_api.cu -- the C ABI of libwkv.so (declared in include/wkv.h).
+//
+// Host side only: argument validation, kernel selection and launches.  Every
+// step of the operator runs in the kernels of wkv_seq.cuh, wkv_chunk.cuh and
+// wkv_step.cuh; there is no host fallback.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+
+#include "../../include/wkv.h"
+#include "wkv_chunk.cuh"
+#include "wkv_seq.cuh"
+#include "wkv_step.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+constexpr int64_t kMaxElems = int64_t(1) << 62;
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {0};
+
+// Chunked-kernel geometry: W warps per CTA, LS tokens per warp segment.
+constexpr int kW = 8;
+constexpr int kLS = 8;
+constexpr int kTT = kW * kLS;
+// Sequences at most this long take the sequential kernel.
+constexpr int64_t kSeqMaxT = 16;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per cross-CTA wait
+
+int record_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return WKV_OK;
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return WKV_ERR_CUDA;
+}
+
+int check_launch() { return record_cuda(cudaPeekAtLastError()); }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// [p, p+bytes) intersects [q, q+qbytes)?
+bool overlaps(const void* p, size_t bytes, const void* q, size_t qbytes) {
+    if (p == nullptr || q == nullptr || bytes == 0 || qbytes == 0) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + qbytes && b < a + bytes;
+}
+
+bool mul_ok(int64_t a, int64_t b, int64_t c, int64_t* out) {
+    if (a < 0 || b < 0 || c < 0) return false;
+    __int128 p = static_cast<__int128>(a) * b * c;
+    if (p >= kMaxElems) return false;
+    *out = static_cast<int64_t>(p);
+    return true;
+}
+
+size_t elem_bytes(int dtype) { return dtype == WKV_BF16 ? 2 : 4; }
+
+struct ChunkGeom {
+    int64_t nCB, nLB, nchunks, units;
+    size_t status_off, agg_off, inc_off, bytes;
+};
+
+ChunkGeom chunk_geom(int64_t B, int64_t T, int64_t C, int V) {
+    ChunkGeom g{};
+    const int64_t CB = 32 * V;
+    g.nCB = (C + CB - 1) / CB;
+    g.nLB = B * g.nCB;
+    g.nchunks = (T + kTT - 1) / kTT;
+    g.units = g.nLB * g.nchunks;
+    if (g.nchunks <= 1) return g;  // no cross-CTA exchange, no workspace
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    g.status_off = 256;
+    g.agg_off = g.status_off + up(size_t(g.units) * 8);
+    g.inc_off = g.agg_off + up(size_t(g.units) * 3 * CB * 4);
+    g.bytes = g.inc_off + up(size_t(g.units) * 3 * CB * 4);
+    return g;
+}
+
+bool use_sequential(int64_t T) { return T <= kSeqMaxT; }
+
+[[maybe_unused]] int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (g_sm_count[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        g_sm_count[dev] = n;
+    }
+    return g_sm_count[dev];
+}
+
+// Vector width 2 needs an even C and every row base aligned to 2 elements.
+int pick_vec(int64_t C, int dtype, const void* const* io, int nio, const float* const* f32, int nf) {
+    if (C % 2 != 0) return 1;
+    const size_t eb = elem_bytes(dtype);
+    for (int i = 0; i < nio; ++i)
+        if (io[i] && !aligned(io[i], 2 * eb)) return 1;
+    for (int i = 0; i < nf; ++i)
+        if (f32[i] && !aligned(f32[i], 8)) return 1;
+    return 2;
+}
+
+template <typename IO, int V, bool GATE>
+void launch_seq(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const void* k,
+                const void* v, const void* r, const float* s_in, void* y, float* s_out,
+                cudaStream_t st) {
+    const int64_t groups = B * (C / V);
+    const int threads = 256;
+    const int64_t blocks = (groups + threads - 1) / threads;
+    wkv::seq_forward_kernel<IO, V, GATE><<<static_cast<unsigned>(blocks), threads, 0, st>>>(
+        B, T, C, w, u, static_cast<const IO*>(k), static_cast<const IO*>(v),
+        static_cast<const IO*>(r), s_in, static_cast<IO*>(y), s_out);
+}
+
+template <typename IO, int V, bool GATE>
+void launch_chunk(const wkv::ChunkArgs& a, int64_t grid, cudaStream_t st) {
+    wkv::chunk_forward_kernel<IO, V, GATE, kW, kLS><<<static_cast<unsigned>(grid), kW * 32, 0, st>>>(a);
+}
+
+template <typename IO, int V>
+void dispatch_forward(bool gate, bool seq, const wkv::ChunkArgs& a, int64_t grid, cudaStream_t st) {
+    if (seq) {
+        if (gate)
+            launch_seq<IO, V, true>(a.B, a.T, a.C, a.w, a.u, a.k, a.v, a.r, a.s_in, a.y, a.s_out, st);
+        else
+            launch_seq<IO, V, false>(a.B, a.T, a.C, a.w, a.u, a.k, a.v, a.r, a.s_in, a.y, a.s_out, st);
+    } else {
+        if (gate)
+            launch_chunk<IO, V, true>(a, grid, st);
+        else
+            launch_chunk<IO, V, false>(a, grid, st);
+    }
+}
+
+template <typename IO, int V, bool GATE>
+void launch_step(int64_t L, int64_t B, int64_t C, const float* w, const float* u, const void* k,
+                 const void* v, const void* r, float* state, void* y, cudaStream_t st) {
+    const int64_t total = L * B * (C / V);
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    wkv::step_kernel<IO, V, GATE><<<static_cast<unsigned>(blocks), threads, 0, st>>>(
+        L, B, C, w, u, static_cast<const IO*>(k), static_cast<const IO*>(v),
+        static_cast<const IO*>(r), state, static_cast<IO*>(y));
+}
+
+}  // namespace
+
+extern "C" {
+
+int wkv_abi_version(void) { return 1; }
+
+const char* wkv_strerror(int status) {
+    switch (status) {
+        case WKV_OK: return "success";
+        case WKV_ERR_NULLPTR: return "a required pointer is NULL";
+        case WKV_ERR_SHAPE: return "invalid size (negative, or element count beyond 2^62)";
+        case WKV_ERR_DTYPE: return "unknown dtype (expected WKV_F32 or WKV_BF16)";
+        case WKV_ERR_ALIGN: return "pointer not aligned to its element type (workspace: 256 bytes)";
+        case WKV_ERR_ALIAS: return "an output buffer overlaps an input or another output";
+        case WKV_ERR_CUDA: return "CUDA error (see wkv_last_cuda_error)";
+        case WKV_ERR_TIMEOUT: return "a cross-block wait on the GPU gave up; affected outputs are NaN";
+        case WKV_ERR_WORKSPACE: return "workspace missing or smaller than wkv_forward_workspace_bytes()";
+        default: return "unknown wkv status";
+    }
+}
+
+const char* wkv_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t wkv_forward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype) {
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n) || (dtype != WKV_F32 && dtype != WKV_BF16)) return 0;
+    if (n == 0 || use_sequential(T)) return 0;
+    // the larger of the two vector widths' layouts, so the size does not
+    // depend on pointer alignment
+    const size_t a = chunk_geom(B, T, C, 1).bytes, b = chunk_geom(B, T, C, 2).bytes;
+    return a > b ? a : b;
+}
+
+int wkv_workspace_init(void* workspace, size_t bytes, cudaStream_t stream) {
+    if (bytes == 0) return WKV_OK;
+    if (workspace == nullptr) return WKV_ERR_NULLPTR;
+    if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
+    return record_cuda(cudaMemsetAsync(workspace, 0, bytes, stream));
+}
+
+int wkv_workspace_status(const void* workspace, cudaStream_t stream) {
+    if (workspace == nullptr) return WKV_ERR_NULLPTR;
+    if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
+    int rc = record_cuda(cudaStreamSynchronize(stream));
+    if (rc != WKV_OK) return rc;
+    wkv::WsHeader h{};
+    rc = record_cuda(cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost));
+    if (rc != WKV_OK) return rc;
+    return (h.error & wkv::kErrTimeout) ? WKV_ERR_TIMEOUT : WKV_OK;
+}
+
+int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                const void* k, const void* v, const void* r, const float* state_in, void* y,
+                float* state_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
+    if (B == 0 || C == 0) return WKV_OK;
+    const int64_t lanes = B * C;
+    const size_t eb = elem_bytes(dtype);
+    const size_t io_bytes = size_t(n) * eb, st_bytes = size_t(lanes) * 3 * 4, p_bytes = size_t(C) * 4;
+    if (T == 0) {
+        if (state_out == nullptr) return WKV_OK;
+        if (!aligned(state_out, 4) || (state_in && !aligned(state_in, 4))) return WKV_ERR_ALIGN;
+        if (state_in && state_in != state_out && overlaps(state_in, st_bytes, state_out, st_bytes))
+            return WKV_ERR_ALIAS;
+        if (state_in == state_out) return WKV_OK;
+        wkv::copy_state_kernel<<<static_cast<unsigned>((lanes + 255) / 256), 256, 0, stream>>>(
+            lanes, state_in, state_out);
+        return check_launch();
+    }
+    if (!w || !u || !k || !v || !y) return WKV_ERR_NULLPTR;
+    if (!aligned(w, 4) || !aligned(u, 4) || !aligned(k, eb) || !aligned(v, eb) || !aligned(y, eb) ||
+        (r && !aligned(r, eb)) || (state_in && !aligned(state_in, 4)) || (state_out && !aligned(state_out, 4)))
+        return WKV_ERR_ALIGN;
+    // y must be disjoint from every input and from state_out
+    const void* ins[] = {k, v, r};
+    for (const void* p : ins)
+        if (overlaps(y, io_bytes, p, io_bytes)) return WKV_ERR_ALIAS;
+    if (overlaps(y, io_bytes, w, p_bytes) || overlaps(y, io_bytes, u, p_bytes) ||
+        overlaps(y, io_bytes, state_in, st_bytes) || overlaps(y, io_bytes, state_out, st_bytes))
+        return WKV_ERR_ALIAS;
+    if (state_out) {
+        for (const void* p : ins)
+            if (overlaps(state_out, st_bytes, p, io_bytes)) return WKV_ERR_ALIAS;
+        if (overlaps(state_out, st_bytes, w, p_bytes) || overlaps(state_out, st_bytes, u, p_bytes))
+            return WKV_ERR_ALIAS;
+        if (state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes))
+            return WKV_ERR_ALIAS;
+    }
+
+    const void* io[] = {k, v, r, y};
+    const float* f32[] = {w, u, state_in, state_out};
+    const int V = pick_vec(C, dtype, io, 4, f32, 4);
+    const bool seq = use_sequential(T);
+
+    wkv::ChunkArgs a{};
+    a.w = w;
+    a.u = u;
+    a.k = k;
+    a.v = v;
+    a.r = r;
+    a.s_in = state_in;
+    a.y = y;
+    a.s_out = state_out;
+    a.B = B;
+    a.T = T;
+    a.C = C;
+    a.wait_limit_ns = kWaitLimitNs;
+    int64_t grid = 0;
+    if (!seq) {
+        const ChunkGeom g = chunk_geom(B, T, C, V);
+        a.nCB = g.nCB;
+        a.nLB = g.nLB;
+        a.nchunks = g.nchunks;
+        a.units = g.units;
+        grid = g.units;
+        if (grid > 0x7fffffffLL) return WKV_ERR_SHAPE;
+        if (g.bytes > 0) {
+            if (workspace == nullptr) return WKV_ERR_WORKSPACE;
+            if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
+            if (workspace_bytes < wkv_forward_workspace_bytes(B, T, C, dtype)) return WKV_ERR_WORKSPACE;
+            char* ws = static_cast<char*>(workspace);
+            a.hdr = reinterpret_cast<wkv::WsHeader*>(ws);
+            a.status = reinterpret_cast<unsigned long long*>(ws + g.status_off);
+            a.agg = reinterpret_cast<float*>(ws + g.agg_off);
+            a.inc = reinterpret_cast<float*>(ws + g.inc_off);
+        }
+    }
+    if (seq && B * (C / V) > int64_t(0x7fffffff) * 256) return WKV_ERR_SHAPE;
+    if (dtype == WKV_F32) {
+        if (V == 2) dispatch_forward<float, 2>(r != nullptr, seq, a, grid, stream);
+        else dispatch_forward<float, 1>(r != nullptr, seq, a, grid, stream);
+    } else {
+        if (V == 2) dispatch_forward<__nv_bfloat16, 2>(r != nullptr, seq, a, grid, stream);
+        else dispatch_forward<__nv_bfloat16, 1>(r != nullptr, seq, a, grid, stream);
+    }
+    return check_launch();
+}
+
+int wkv_step(int64_t L, int64_t B, int64_t C, int dtype, const float* w, const float* u,
+             const void* k, const void* v, const void* r, float* state, void* y, cudaStream_t stream) {
+    if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    int64_t n = 0;
+    if (!mul_ok(L, B, C, &n)) return WKV_ERR_SHAPE;
+    if (n == 0) return WKV_OK;
+    if (!w || !u || !k || !v || !state || !y) return WKV_ERR_NULLPTR;
+    const size_t eb = elem_bytes(dtype);
+    if (!aligned(w, 4) || !aligned(u, 4) || !aligned(state, 4) || !aligned(k, eb) || !aligned(v, eb) ||
+        !aligned(y, eb) || (r && !aligned(r, eb)))
+        return WKV_ERR_ALIGN;
+    const size_t io_bytes = size_t(n) * eb, st_bytes = size_t(n) * 3 * 4, p_bytes = size_t(L) * C * 4;
+    const void* ins[] = {k, v, r};
+    for (const void* p : ins)
+        if (overlaps(y, io_bytes, p, io_bytes) || overlaps(state, st_bytes, p, io_bytes)) return WKV_ERR_ALIAS;
+    if (overlaps(y, io_bytes, state, st_bytes) || overlaps(y, io_bytes, w, p_bytes) ||
+        overlaps(y, io_bytes, u, p_bytes) || overlaps(state, st_bytes, w, p_bytes) ||
+        overlaps(state, st_bytes, u, p_bytes))
+        return WKV_ERR_ALIAS;
+    const void* io[] = {k, v, r, y};
+    const float* f32[] = {w, u, state};
+    const int V = pick_vec(C, dtype, io, 4, f32, 3);
+    if (L * B * (C / V) > int64_t(0x7fffffff) * 256) return WKV_ERR_SHAPE;
+    const bool g = r != nullptr;
+#define WKV_STEP(IO_, V_)                                                                  \
+    (g ? launch_step<IO_, V_, true>(L, B, C, w, u, k, v, r, state, y, stream)              \
+       : launch_step<IO_, V_, false>(L, B, C, w, u, k, v, r, state, y, stream))
+    if (dtype == WKV_F32) {
+        if (V == 2) WKV_STEP(float, 2);
+        else WKV_STEP(float, 1);
+    } else {
+        if (V == 2) WKV_STEP(__nv_bfloat16, 2);
+        else WKV_STEP(__nv_bfloat16, 1);
+    }
+#undef WKV_STEP
+    return check_launch();
+}
+
+}  // extern "C"

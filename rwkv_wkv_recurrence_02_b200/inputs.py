@@ -136,12 +136,27 @@ def make_chunk(wl: Workload, index: int, B=None, C=None, device="cpu"):
     return make_sequence(wl, B, wl.chunk, C, device=device, seed=wl.seed * 1000003 + index)
 
 
-def make_decode_set(wl: Workload, index: int, B=None, C=None, device="cpu"):
-    """k, v, r of shape (layers, B, C) for ring slot `index` of the decode workload."""
+def make_decode_ring(wl: Workload, B=None, C=None, device="cpu"):
+    """k, v, r of the decode ring: shape (ring + layers - 1, B, C).  Rows
+    0..ring-1 are the ring's input sets (one (B, C) set per layer-step); the
+    last layers-1 rows repeat the first ones, so the sets of step s,
+    (s*layers + l) mod ring for l = 0..layers-1, are the contiguous slice
+    starting at row (s*layers) mod ring."""
     B = wl.B if B is None else B
     C = wl.C if C is None else C
-    k, v, r = make_sequence(wl, wl.layers, B, C, device=device, seed=wl.seed * 1000003 + index)
-    return k, v, r
+    g = _gen(device, wl.seed * 1000003)
+    k = torch.randn((wl.ring, B, C), dtype=torch.float32, device=device, generator=g) * wl.k_std
+    v = torch.randn((wl.ring, B, C), dtype=torch.float32, device=device, generator=g)
+    r = torch.randn((wl.ring, B, C), dtype=torch.float32, device=device, generator=g) if wl.gate else None
+    dt = wl.torch_dtype
+    k, v, r = k.to(dt), v.to(dt), (None if r is None else r.to(dt))
+    ext = lambda x: None if x is None else torch.cat([x, x[: wl.layers - 1]]).contiguous()
+    return ext(k), ext(v), ext(r)
+
+
+def decode_ring_start(wl: Workload, step: int) -> int:
+    """First ring row of decode step `step` (see make_decode_ring)."""
+    return (step * wl.layers) % wl.ring
 
 
 def fresh_state(B: int, C: int, layers: int = 0, device="cpu"):

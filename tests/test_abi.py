@@ -1,0 +1,147 @@
+"""The C ABI on the host: the library loads without a GPU, exports every
+function include/wkv.h declares, and rejects bad arguments before launching
+anything (these calls return before any CUDA runtime call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rwkv_wkv_recurrence_02_b200 as wkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wkv.h")
+
+OK, NULLPTR, SHAPE, DTYPE, ALIGN, ALIAS, CUDA, TIMEOUT, WORKSPACE = 0, -1, -2, -3, -4, -5, -6, -7, -8
+F32, BF16 = 0, 1
+# fake, well-aligned device addresses: every call below must fail validation
+# (or be a no-op) before it could dereference them
+BASE = 1 << 40
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s*(wkv_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    return wkv.lib()
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(wkv.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    # and through dlsym of the raw handle, not just the ctypes cache
+    raw = ctypes.CDLL(wkv.LIB_PATH)
+    for name in declared_functions():
+        assert ctypes.cast(getattr(raw, name), ctypes.c_void_p).value
+
+
+def test_abi_version_and_strerror(L):
+    assert L.wkv_abi_version() == 1
+    msgs = {L.wkv_strerror(s).decode() for s in (OK, NULLPTR, SHAPE, DTYPE, ALIGN, ALIAS, CUDA, TIMEOUT, WORKSPACE)}
+    assert len(msgs) == 9
+    assert L.wkv_strerror(12345).decode() == "unknown wkv status"
+
+
+def fwd(L, B=2, T=100, C=64, dt=F32, w=BASE, u=BASE + 4096, k=BASE + (1 << 30), v=BASE + (2 << 30),
+        r=None, s_in=None, y=BASE + (3 << 30), s_out=None, ws=None, ws_bytes=0):
+    return L.wkv_forward(B, T, C, dt, w, u, k, v, r, s_in, y, s_out, ws, ws_bytes, None)
+
+
+def test_forward_rejects_bad_dtype_and_shapes(L):
+    assert fwd(L, dt=7) == DTYPE
+    assert fwd(L, B=-1) == SHAPE
+    assert fwd(L, T=-5) == SHAPE
+    assert fwd(L, B=1 << 21, T=1 << 21, C=1 << 21) == SHAPE
+
+
+def test_forward_empty_is_a_noop(L):
+    assert fwd(L, B=0) == OK
+    assert fwd(L, C=0) == OK
+    assert fwd(L, T=0) == OK            # no state_out: nothing to write
+    s = BASE + (5 << 30)
+    assert fwd(L, T=0, s_in=s, s_out=s) == OK   # in place: nothing to copy
+
+
+def test_forward_null_pointers(L):
+    assert fwd(L, w=None) == NULLPTR
+    assert fwd(L, k=None) == NULLPTR
+    assert fwd(L, y=None) == NULLPTR
+
+
+def test_forward_alignment(L):
+    assert fwd(L, k=BASE + (1 << 30) + 2) == ALIGN
+    assert fwd(L, dt=BF16, k=BASE + (1 << 30) + 1) == ALIGN
+    assert fwd(L, s_out=BASE + (6 << 30) + 1) == ALIGN
+    ws = BASE + (7 << 30)
+    n = L.wkv_forward_workspace_bytes(2, 100, 64, F32)
+    assert fwd(L, ws=ws + 16, ws_bytes=n) == ALIGN
+
+
+def test_forward_aliasing(L):
+    k = BASE + (1 << 30)
+    assert fwd(L, y=k) == ALIAS
+    assert fwd(L, y=k + 64) == ALIAS                    # partial overlap
+    s = BASE + (5 << 30)
+    assert fwd(L, s_in=s, s_out=s + 8) == ALIAS         # partial state overlap
+    assert fwd(L, s_out=k) == ALIAS
+    assert fwd(L, s_out=BASE + (3 << 30)) == ALIAS      # state_out inside y
+
+
+def test_forward_workspace_checks(L):
+    n = L.wkv_forward_workspace_bytes(2, 100, 64, F32)
+    assert n > 0
+    assert fwd(L, ws=None, ws_bytes=0) == WORKSPACE
+    assert fwd(L, ws=BASE + (7 << 30), ws_bytes=n - 1) == WORKSPACE
+
+
+def test_workspace_size_rules(L):
+    # short sequences take the sequential kernel and need no workspace
+    assert L.wkv_forward_workspace_bytes(4, 16, 128, F32) == 0
+    assert L.wkv_forward_workspace_bytes(4, 64, 128, F32) == 0     # a single chunk
+    assert L.wkv_forward_workspace_bytes(-1, 64, 128, F32) == 0
+    small = L.wkv_forward_workspace_bytes(8, 1024, 2048, F32)
+    big = L.wkv_forward_workspace_bytes(8, 4096, 2048, F32)
+    assert 0 < small < big
+    # bounded by a few bytes per element: 2 states of 12 B per lane per chunk
+    assert small < 8 * 1024 * 2048
+
+
+def test_workspace_init_and_status_validation(L):
+    assert L.wkv_workspace_init(None, 0, None) == OK
+    assert L.wkv_workspace_init(None, 100, None) == NULLPTR
+    assert L.wkv_workspace_init(BASE + 8, 100, None) == ALIGN
+    assert L.wkv_workspace_status(None, None) == NULLPTR
+    assert L.wkv_workspace_status(BASE + 8, None) == ALIGN
+
+
+def step(L, Lr=2, B=3, C=64, dt=BF16, w=BASE, u=BASE + 4096, k=BASE + (1 << 30), v=BASE + (2 << 30), r=None,
+         state=BASE + (4 << 30), y=BASE + (3 << 30)):
+    return L.wkv_step(Lr, B, C, dt, w, u, k, v, r, state, y, None)
+
+
+def test_step_validation(L):
+    assert step(L, dt=3) == DTYPE
+    assert step(L, Lr=-1) == SHAPE
+    assert step(L, Lr=0) == OK
+    assert step(L, state=None) == NULLPTR
+    assert step(L, y=None) == NULLPTR
+    assert step(L, state=BASE + (4 << 30) + 2) == ALIGN
+    assert step(L, y=BASE + (4 << 30)) == ALIAS      # y inside the state
+    assert step(L, state=BASE + (1 << 30)) == ALIAS  # state over k
+
+
+def test_python_front_end_refuses_cpu_tensors():
+    import torch
+    k = torch.zeros(1, 4, 8)
+    with pytest.raises(ValueError):
+        wkv.wkv_forward(torch.ones(8), torch.zeros(8), k, k)
+    with pytest.raises(ValueError):
+        wkv.wkv_step(torch.ones(1, 8), torch.zeros(1, 8), k, k, torch.zeros(1, 3, 4, 8))

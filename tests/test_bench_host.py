@@ -1,0 +1,99 @@
+"""bench.py's host-side logic: byte accounting, rank helpers and the
+max-over-ranks reduction (two gloo ranks on CPU)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+from rwkv_wkv_recurrence_02_b200 import inputs as I
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_bytes_layer_1b5():
+    wl = I.WORKLOADS["layer_1b5"]
+    n = 8 * 1024 * 2048
+    # k, v, r read + y written (4 B each), state in and out, w and u
+    assert bench.algorithmic_bytes(wl, 8, 1024, 2048) == n * 16 + 8 * 2048 * 24 + 2048 * 8
+
+
+def test_algorithmic_bytes_bf16_and_decode():
+    wl = I.WORKLOADS["layer_14b"]
+    n = 4 * 8192 * 5120
+    assert bench.algorithmic_bytes(wl, 4, 8192, 5120) == n * 8 + 4 * 5120 * 12 + 5120 * 8
+    st = I.WORKLOADS["stream_1m"]
+    assert bench.algorithmic_bytes(st, 1, 1024, 4096) == 1024 * 4096 * 6 + 4096 * 24 + 4096 * 8
+    dec = I.WORKLOADS["decode"]
+    lanes = 24 * 256 * 4096
+    assert bench.algorithmic_bytes(dec, 256, 1, 4096, layers=24) == lanes * 8 + lanes * 24 + 24 * 4096 * 8
+
+
+def test_rates_and_seeds():
+    assert bench.whole_job_rate(100, 4, 10, 2.0) == 2000.0
+    assert len({bench.rank_seed(0, r) for r in range(8)}) == 8
+
+
+def test_traffic_record_invalidated_by_source_change(tmp_path, monkeypatch):
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps({"layer_1b5": {"traffic_bytes_per_launch": 123, "source_hash": "stale"}}))
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(p))
+    assert bench.load_traffic("layer_1b5") is None
+    p.write_text(json.dumps({"layer_1b5": {"traffic_bytes_per_launch": 123,
+                                           "source_hash": bench.kernel_source_hash()}}))
+    assert bench.load_traffic("layer_1b5") == 123
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    t = bench.max_over_ranks(1.0 + rank * 0.5, dist)
+    q.put((rank, t))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def test_max_over_ranks_gloo_world_2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    assert got == [(0, 1.5), (1, 1.5)]
+
+
+def test_reference_arm_nonzero_rank_exits_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "3",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_prints_one_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "3",
+                        "--warmup", "3", "--ref-budget-s", "3"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["unit"] == "elements/s" and out["value"] > 0
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["e2e"]["h2d_bytes_per_step"] == 0
+    assert out["config"]["workload"] == "layer_1b5"

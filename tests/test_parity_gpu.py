@@ -1,0 +1,302 @@
+"""CUDA path vs the fp64 oracle, element by element, on identical seeded inputs.
+
+Calls go through the C ABI (the ctypes binding).  Small shapes cover every
+tile edge and ragged tail of the kernels; the five workloads run at full size
+on the GPU with the oracle on sampled lanes (lanes are independent, so a
+sampled lane is checked exactly).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rwkv_wkv_recurrence_02_b200 as wkv
+from rwkv_wkv_recurrence_02_b200 import inputs as I
+from tests.parity import (TOL, argmax_index, gpu_argmax_index, oracle_forward, output_error, sample_channels,
+                          state_error, to_np32, to_np64)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def gen_case(B, T, C, dtype, gate, state, seed=0, k_std=1.0, device=DEV):
+    wl = I.Workload("case", B, T, C, "f32" if dtype == torch.float32 else "bf16", gate, -3.0, 1.0, 1.0, k_std,
+                    state, seed=seed + 77)
+    d = I.make_forward_inputs(wl, device="cpu")
+    return {k: (None if v is None else v.to(device)) for k, v in d.items()}
+
+
+def run_forward(d, **kw):
+    y, s = wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"], **kw)
+    torch.cuda.synchronize()
+    return y, s
+
+
+def check_forward(d, y, s, tol=None, state_tol=None):
+    tol = TOL[d["k"].dtype] if tol is None else tol
+    y_ref, s_ref, scale = oracle_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"])
+    err = output_error(y, y_ref, scale)
+    assert err <= tol, f"output error {err:.3e} > {tol:.1e}"
+    if s is not None:
+        ratio, logd, pe = state_error(s, s_ref)
+        st = tol if state_tol is None else state_tol
+        assert ratio <= st and logd <= st and pe <= st, (ratio, logd, pe)
+    return err
+
+
+SMALL = [
+    # B, T, C, dtype, gate, state
+    (1, 1, 1, torch.float32, False, False),
+    (1, 2, 7, torch.float32, True, True),
+    (3, 3, 8, torch.bfloat16, True, False),
+    (2, 16, 33, torch.float32, False, True),
+    (2, 17, 64, torch.float32, True, True),
+    (1, 63, 65, torch.bfloat16, False, True),
+    (2, 64, 64, torch.float32, True, False),
+    (1, 65, 130, torch.float32, True, True),
+    (3, 127, 66, torch.bfloat16, True, True),
+    (2, 128, 32, torch.float32, False, False),
+    (1, 129, 1, torch.float32, True, True),
+    (2, 200, 7, torch.bfloat16, False, False),
+    (1, 1000, 96, torch.float32, True, True),
+    (2, 1000, 130, torch.bfloat16, True, True),
+    (1, 4099, 64, torch.float32, False, True),
+    (1, 4099, 62, torch.bfloat16, True, False),
+]
+
+
+@pytest.mark.parametrize("B,T,C,dtype,gate,state", SMALL)
+def test_small_shapes(B, T, C, dtype, gate, state):
+    d = gen_case(B, T, C, dtype, gate, state, seed=B * 1000 + T + C)
+    y, s = run_forward(d)
+    check_forward(d, y, s)
+
+
+def test_tiny_workload_against_brute_force():
+    d = I.make_forward_inputs("tiny", device=DEV)
+    y, s = run_forward(d)
+    yb, sb = oracle.wkv_brute(to_np32(d["w"]), to_np32(d["u"]), to_np32(d["k"]), to_np32(d["v"]),
+                              want_scale=True)
+    err = output_error(y, yb, sb)
+    assert err <= TOL[torch.float32], err
+    check_forward(d, y, s)
+
+
+@pytest.mark.parametrize("kval", ["alt60", "const+60", "const-60", "outliers"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_extreme_keys(kval, dtype):
+    """+-60 keys (no overflow) and sparse +-50 outliers: mixes the fixed-scale
+    fast path with the exact running-max path inside one launch."""
+    B, T, C = 2, 700, 96
+    d = gen_case(B, T, C, dtype, True, True, seed=5)
+    t = torch.arange(T, device=DEV)[None, :, None]
+    if kval == "alt60":
+        k = torch.where(t % 2 == 0, 60.0, -60.0).expand(B, T, C)
+    elif kval == "const+60":
+        k = torch.full((B, T, C), 60.0, device=DEV)
+    elif kval == "const-60":
+        k = torch.full((B, T, C), -60.0, device=DEV)
+    else:
+        g = torch.Generator(device="cpu").manual_seed(3)
+        k = torch.randn(B, T, C, generator=g)
+        hit = torch.rand(B, T, C, generator=g) < 0.01
+        k = torch.where(hit, torch.where(torch.rand(B, T, C, generator=g) < 0.5, -50.0, 50.0), k).to(DEV)
+    d["k"] = k.to(dtype).contiguous()
+    y, s = run_forward(d)
+    check_forward(d, y, s)
+
+
+def test_state_in_place_and_chaining():
+    """state_out == state_in is allowed; chaining calls reproduces one pass."""
+    d = gen_case(2, 300, 130, torch.float32, True, True, seed=11)
+    y_full, s_full = run_forward(d)
+    st = d["state"].clone()
+    parts = []
+    for a, b in [(0, 1), (1, 70), (70, 71), (71, 200), (200, 300)]:
+        sl = lambda x: None if x is None else x[:, a:b].contiguous()
+        y, _ = wkv.wkv_forward(d["w"], d["u"], sl(d["k"]), sl(d["v"]), sl(d["r"]), st, state_out=st)
+        parts.append(y)
+    torch.cuda.synchronize()
+    y_chain = torch.cat(parts, dim=1)
+    scale = oracle_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"])[2]
+    assert output_error(y_chain, to_np64(y_full), scale) <= 2e-5
+    ratio, logd, pe = state_error(st, to_np64(s_full))
+    assert max(ratio, logd, pe) <= 2e-5
+
+
+def test_rnn_mode_equals_parallel_mode():
+    B, T, C = 3, 40, 66
+    d = gen_case(B, T, C, torch.bfloat16, True, True, seed=13)
+    y_par, s_par = run_forward(d)
+    state = d["state"].clone()[None].contiguous()
+    ys = []
+    for t in range(T):
+        ys.append(wkv.wkv_step(d["w"][None], d["u"][None], d["k"][None, :, t].contiguous(),
+                               d["v"][None, :, t].contiguous(), state, d["r"][None, :, t].contiguous())[0])
+    torch.cuda.synchronize()
+    y_rnn = torch.stack(ys, dim=1)
+    scale = oracle_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"])[2]
+    # both are bf16-rounded outputs of float32 arithmetic on identical inputs
+    assert output_error(y_rnn, to_np64(y_par).astype(np.float64), scale) <= 1e-2
+    ratio, logd, pe = state_error(state[0], to_np64(s_par))
+    assert max(ratio, logd, pe) <= 1e-4
+
+
+def test_forward_t1_equals_step():
+    d = gen_case(4, 1, 130, torch.float32, True, True, seed=17)
+    y, s = run_forward(d)
+    st = d["state"].clone()[None].contiguous()
+    y2 = wkv.wkv_step(d["w"][None], d["u"][None], d["k"].transpose(0, 1).contiguous(),
+                      d["v"].transpose(0, 1).contiguous(), st, d["r"].transpose(0, 1).contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(y2[0], y[:, 0])
+    assert torch.equal(st[0], s)
+
+
+def test_empty_and_degenerate_sizes():
+    d = gen_case(2, 5, 8, torch.float32, False, True, seed=19)
+    st = torch.empty_like(d["state"])
+    y = torch.empty((2, 0, 8), device=DEV)
+    wkv.lib()
+    rc = wkv.lib().wkv_forward(2, 0, 8, 0, d["w"].data_ptr(), d["u"].data_ptr(), d["k"].data_ptr(),
+                               d["v"].data_ptr(), None, d["state"].data_ptr(), y.data_ptr(), st.data_ptr(),
+                               None, 0, None)
+    torch.cuda.synchronize()
+    assert rc == 0 and torch.equal(st, d["state"])
+    rc = wkv.lib().wkv_forward(2, 0, 8, 0, None, None, None, None, None, None, None, st.data_ptr(), None, 0, None)
+    torch.cuda.synchronize()
+    assert rc == 0
+    assert torch.all(st[0] == 0) and torch.all(st[1] == 0) and torch.all(st[2] == -1e38)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_guard_bands_untouched(dtype):
+    """Outputs land exactly in their buffers: sentinel padding around y and
+    the state survives (bounds check without a sanitizer)."""
+    B, T, C, pad = 2, 333, 70, 4096
+    d = gen_case(B, T, C, dtype, True, True, seed=23)
+    n = B * T * C
+    ybuf = torch.full((n + 2 * pad,), 12345.0, dtype=dtype, device=DEV)
+    sbuf = torch.full((3 * B * C + 2 * pad,), 777.0, dtype=torch.float32, device=DEV)
+    y = ybuf[pad:pad + n].view(B, T, C)
+    s = sbuf[pad:pad + 3 * B * C].view(3, B, C)
+    run_forward(d, y=y, state_out=s)
+    assert torch.all(ybuf[:pad] == 12345.0) and torch.all(ybuf[pad + n:] == 12345.0)
+    assert torch.all(sbuf[:pad] == 777.0) and torch.all(sbuf[pad + 3 * B * C:] == 777.0)
+    check_forward(d, y, s)
+
+
+def test_workspace_reuse_across_shapes():
+    """One workspace serves calls of different shapes back to back (the
+    launch epoch in the status words keeps them apart)."""
+    ws = wkv.Workspace()
+    for i, (B, T, C) in enumerate([(2, 500, 64), (1, 1000, 130), (2, 500, 64), (3, 257, 32)]):
+        d = gen_case(B, T, C, torch.float32, True, True, seed=31 + i)
+        y, s = run_forward(d, workspace=ws)
+        check_forward(d, y, s)
+    assert ws.status() == 0
+
+
+# ---------------------------------------------------------------------------
+# the five workloads at full size
+# ---------------------------------------------------------------------------
+def sampled(d, idx):
+    f = lambda x: None if x is None else x[..., idx].contiguous().cpu()
+    return dict(w=d["w"][idx].cpu(), u=d["u"][idx].cpu(), k=f(d["k"]), v=f(d["v"]), r=f(d["r"]),
+                state=f(d["state"]))
+
+
+def test_layer_1b5_full():
+    d = I.make_forward_inputs("layer_1b5", device=DEV)
+    y, s = run_forward(d)
+    idx = sample_channels(d["k"].shape[2], n=512)
+    ds = sampled(d, idx)
+    check_forward(ds, y[..., idx.to(DEV)], s[..., idx.to(DEV)])
+    # the index of the term that sets the final running max
+    T = d["k"].shape[1]
+    j_ref, gap, cand = argmax_index(to_np32(ds["k"]), to_np32(ds["w"]), T, p0=to_np64(ds["state"][2]))
+    j_gpu = gpu_argmax_index(to_np64(s[2][..., idx.to(DEV)]), cand, 1)
+    clear = gap > 1e-3
+    assert clear.mean() > 0.9
+    assert np.array_equal(j_gpu[clear], j_ref[clear])
+
+
+def test_layer_14b_full():
+    d = I.make_forward_inputs("layer_14b", device=DEV)
+    y, s = run_forward(d)
+    idx = sample_channels(d["k"].shape[2], n=64)
+    ds = sampled(d, idx)
+    check_forward(ds, y[..., idx.to(DEV)], s[..., idx.to(DEV)])
+    T = d["k"].shape[1]
+    j_ref, gap, cand = argmax_index(to_np32(ds["k"]), to_np32(ds["w"]), T)
+    j_gpu = gpu_argmax_index(to_np64(s[2][..., idx.to(DEV)]), cand, 0)
+    clear = gap > 1e-2
+    assert np.array_equal(j_gpu[clear], j_ref[clear])
+
+
+def test_stream_1m_chunked_equals_single_pass():
+    wl = I.WORKLOADS["stream_1m"]
+    C, n = wl.C, wl.T // wl.chunk
+    w, u = I.make_params(wl, device=DEV)
+    chunks = [I.make_chunk(wl, i, device=DEV) for i in range(n)]
+    k = torch.cat([c[0] for c in chunks], dim=1)
+    v = torch.cat([c[1] for c in chunks], dim=1)
+    del chunks
+    y_single, s_single = wkv.wkv_forward(w, u, k, v)
+    state = I.fresh_state(1, C, device=DEV)
+    y_chain = torch.empty_like(y_single)
+    for i in range(n):
+        sl = slice(i * wl.chunk, (i + 1) * wl.chunk)
+        wkv.wkv_forward(w, u, k[:, sl], v[:, sl], None, state, y=y_chain[:, sl], state_out=state)
+    torch.cuda.synchronize()
+    idx = sample_channels(C, n=24)
+    ds = dict(w=w[idx].cpu(), u=u[idx].cpu(), k=k[..., idx].cpu(), v=v[..., idx].cpu(), r=None, state=None)
+    y_ref, s_ref, scale = oracle_forward(**ds)
+    dv = idx.to(DEV)
+    assert output_error(y_single[..., dv], y_ref, scale) <= 1e-2
+    assert output_error(y_chain[..., dv], y_ref, scale) <= 1e-2
+    for s in (s_single, state):
+        ratio, logd, pe = state_error(s[..., dv], s_ref)
+        assert max(ratio, logd, pe) <= 1e-3, (ratio, logd, pe)
+    # chained and single pass agree everywhere, not only on sampled lanes
+    diff = (y_single.float() - y_chain.float()).abs().max().item()
+    assert diff <= 2e-2 * max(1.0, y_single.float().abs().max().item())
+
+
+def test_decode_full():
+    wl = I.WORKLOADS["decode"]
+    L, B, C = wl.layers, wl.B, wl.C
+    w, u = I.make_params(wl, layers=L, device=DEV)
+    kr, vr, rr = I.make_decode_ring(wl, device=DEV)
+    state = I.fresh_state(B, C, layers=L, device=DEV)
+    y = torch.empty((L, B, C), dtype=torch.bfloat16, device=DEV)
+    g = np.random.default_rng(5)
+    bsel = torch.tensor(sorted(g.choice(B, 8, replace=False)), device=DEV)
+    csel = sample_channels(C, n=16).to(DEV)
+    steps = 200
+    ys = []
+    for s in range(steps):
+        a = I.decode_ring_start(wl, s)
+        wkv.wkv_step(w, u, kr[a:a + L], vr[a:a + L], state, rr[a:a + L], y=y)
+        ys.append(y[:, bsel][:, :, csel].clone())
+    torch.cuda.synchronize()
+    # oracle on the sampled lanes, step by step: a one-token forward per
+    # layer is the decode step (same arithmetic) and also gives the scale
+    sub = lambda x: x[:, bsel][:, :, csel].cpu()
+    ost = [oracle.fresh_state(len(bsel), len(csel)) for _ in range(L)]
+    wn, un = to_np32(w[:, csel]), to_np32(u[:, csel])
+    worst = 0.0
+    for s in range(steps):
+        a = I.decode_ring_start(wl, s)
+        kk, vv, rrr = (to_np32(sub(x[a:a + L])) for x in (kr, vr, rr))
+        yg = to_np64(ys[s])
+        for l in range(L):
+            yref, ost[l], scale = oracle.wkv_forward(wn[l], un[l], kk[l][:, None], vv[l][:, None],
+                                                     rrr[l][:, None], ost[l], want_scale=True)
+            worst = max(worst, float(np.max(np.abs(yg[l] - yref[:, 0]) / scale[:, 0])))
+    assert worst <= 1e-2, worst
+    sg = to_np64(state[:, :, bsel][:, :, :, csel])          # (L, 3, nb, nc)
+    so = np.stack(ost)                                       # (L, 3, nb, nc)
+    ratio, logd, pe = state_error(torch.from_numpy(sg.transpose(1, 0, 2, 3).copy()), so.transpose(1, 0, 2, 3))
+    assert max(ratio, logd, pe) <= 1e-3, (ratio, logd, pe)
