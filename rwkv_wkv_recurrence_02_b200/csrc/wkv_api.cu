@@ -3,6 +3,7 @@
 // Host side only: argument validation, kernel selection and launches.  Every
 // step of the operator runs in the kernels of wkv_seq.cuh, wkv_chunk.cuh and
 // wkv_step.cuh; there is no host fallback.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -12,6 +13,7 @@
 
 #include "../../include/wkv.h"
 #include "wkv_chunk.cuh"
+#include "wkv_chunk_ws.cuh"
 #include "wkv_seq.cuh"
 #include "wkv_step.cuh"
 
@@ -23,10 +25,15 @@ constexpr int64_t kMaxElems = int64_t(1) << 62;
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
 
-// Chunked-kernel geometry: W warps per CTA, LS tokens per warp segment.
+// Chunked-kernel geometry: W compute warps per CTA, LS tokens per warp
+// segment, TT = W * LS tokens per chunk.  The register-load kernel uses
+// kW warps; the warp-specialised TMA kernel kWsW compute warps and a ring of
+// kWsStages stages.  The workspace is sized for the smaller chunk.
 constexpr int kW = 8;
 constexpr int kLS = 8;
-constexpr int kTT = kW * kLS;
+constexpr int kWsW = 4;
+constexpr int kWsStages = 4;
+constexpr int kMinTT = (kW < kWsW ? kW : kWsW) * kLS;
 // Sequences at most this long take the sequential kernel.
 constexpr int64_t kSeqMaxT = 16;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per cross-CTA wait
@@ -61,28 +68,31 @@ size_t elem_bytes(int dtype) { return dtype == WKV_BF16 ? 2 : 4; }
 
 struct ChunkGeom {
     int64_t nCB, nLB, nchunks, units;
-    size_t status_off, agg_off, inc_off, bytes;
+    size_t aggw_off, incw_off, bytes;
 };
 
-ChunkGeom chunk_geom(int64_t B, int64_t T, int64_t C, int V) {
+ChunkGeom chunk_geom(int64_t B, int64_t T, int64_t C, int V, int TT) {
     ChunkGeom g{};
     const int64_t CB = 32 * V;
     g.nCB = (C + CB - 1) / CB;
     g.nLB = B * g.nCB;
-    g.nchunks = (T + kTT - 1) / kTT;
+    g.nchunks = (T + TT - 1) / TT;
     g.units = g.nLB * g.nchunks;
     if (g.nchunks <= 1) return g;  // no cross-CTA exchange, no workspace
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-    g.status_off = 256;
-    g.agg_off = g.status_off + up(size_t(g.units) * 8);
-    g.inc_off = g.agg_off + up(size_t(g.units) * 3 * CB * 4);
-    g.bytes = g.inc_off + up(size_t(g.units) * 3 * CB * 4);
+    // header, then one 16-byte word per channel per chunk for the chunk
+    // summaries and for the inclusive states
+    g.aggw_off = 256;
+    g.incw_off = g.aggw_off + up(size_t(g.units) * CB * sizeof(wkv::Word));
+    g.bytes = g.incw_off + up(size_t(g.units) * CB * sizeof(wkv::Word));
     return g;
 }
 
 bool use_sequential(int64_t T) { return T <= kSeqMaxT; }
 
-[[maybe_unused]] int sm_count() {
+int forced_kernel();
+
+int sm_count() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
     if (g_sm_count[dev] == 0) {
@@ -119,6 +129,105 @@ void launch_seq(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
 template <typename IO, int V, bool GATE>
 void launch_chunk(const wkv::ChunkArgs& a, int64_t grid, cudaStream_t st) {
     wkv::chunk_forward_kernel<IO, V, GATE, kW, kLS><<<static_cast<unsigned>(grid), kW * 32, 0, st>>>(a);
+}
+
+// ---- TMA path ----------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 3-D map over a (B, T, C) array: box = CB channels x TT tokens x 1 sequence.
+// Coordinates past T or C read as zeros.
+bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t T, int64_t C, int CB, int TT) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t eb = elem_bytes(dtype);
+    const cuuint64_t dims[3] = {cuuint64_t(C), cuuint64_t(T), cuuint64_t(B)};
+    const cuuint64_t strides[2] = {cuuint64_t(C) * eb, cuuint64_t(T) * cuuint64_t(C) * eb};
+    const cuuint32_t box[3] = {cuuint32_t(CB), cuuint32_t(TT), 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, dtype == WKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// TMA needs 16-byte aligned bases and row strides, and coordinates in int32.
+bool tma_eligible(int V, int dtype, int64_t B, int64_t T, int64_t C, const void* k, const void* v, const void* r,
+                  const float* w, const float* u, const float* s_in) {
+    // w, u and the initial state travel as bulk copies of whole rows
+    if (C % 4 != 0 || !aligned(w, 16) || !aligned(u, 16) || (s_in && !aligned(s_in, 16))) return false;
+    if (V != 2) return false;
+    const int64_t eb = static_cast<int64_t>(elem_bytes(dtype));
+    if ((C * eb) % 16 != 0) return false;
+    if (B >= (int64_t(1) << 31) || T >= (int64_t(1) << 31) || C >= (int64_t(1) << 31)) return false;
+    if (!aligned(k, 16) || !aligned(v, 16) || (r && !aligned(r, 16))) return false;
+    return encode_fn() != nullptr;
+}
+
+// Kernel choice: 0 = automatic; the environment variable WKV_FORWARD_KERNEL
+// (seq | chunk | tma) forces one, for ablation measurements.
+int forced_kernel() {
+    static int f = []() {
+        const char* e = std::getenv("WKV_FORWARD_KERNEL");
+        if (e == nullptr) return 0;
+        if (std::strcmp(e, "seq") == 0) return 1;
+        if (std::strcmp(e, "chunk") == 0) return 2;
+        if (std::strcmp(e, "tma") == 0) return 3;
+        return 0;
+    }();
+    return f;
+}
+
+template <typename IO, bool GATE, int STAGES>
+int launch_tma(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
+    using G = wkv::WsGeometry<IO, 2, GATE, kWsW, kLS, STAGES>;
+    auto kern = wkv::chunk_ws_kernel<IO, 2, GATE, kWsW, kLS, STAGES>;
+    static int capacity[kMaxDevices] = {0};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (capacity[dev] == 0) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        int per_sm = 0;
+        rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+    }
+    CUtensorMap tk, tv, tr;
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
+        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT))
+        return WKV_ERR_CUDA;
+    if (GATE) {
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT)) return WKV_ERR_CUDA;
+    } else {
+        tr = tv;
+    }
+    const int64_t grid = a.units < capacity[dev] ? a.units : capacity[dev];
+    kern<<<static_cast<unsigned>(grid), G::THREADS, G::SMEM, st>>>(tk, tv, tr, a);
+    return check_launch();
+}
+
+template <typename IO>
+int dispatch_tma(bool gate, const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
+    constexpr int S = kWsStages;
+    return gate ? launch_tma<IO, true, S>(a, dtype, st) : launch_tma<IO, false, S>(a, dtype, st);
 }
 
 template <typename IO, int V>
@@ -176,7 +285,7 @@ size_t wkv_forward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype) {
     if (n == 0 || use_sequential(T)) return 0;
     // the larger of the two vector widths' layouts, so the size does not
     // depend on pointer alignment
-    const size_t a = chunk_geom(B, T, C, 1).bytes, b = chunk_geom(B, T, C, 2).bytes;
+    const size_t a = chunk_geom(B, T, C, 1, kMinTT).bytes, b = chunk_geom(B, T, C, 2, kMinTT).bytes;
     return a > b ? a : b;
 }
 
@@ -241,7 +350,8 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     const void* io[] = {k, v, r, y};
     const float* f32[] = {w, u, state_in, state_out};
     const int V = pick_vec(C, dtype, io, 4, f32, 4);
-    const bool seq = use_sequential(T);
+    const int force = forced_kernel();
+    const bool seq = force == 1 || (force == 0 && use_sequential(T));
 
     wkv::ChunkArgs a{};
     a.w = w;
@@ -258,7 +368,8 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     a.wait_limit_ns = kWaitLimitNs;
     int64_t grid = 0;
     if (!seq) {
-        const ChunkGeom g = chunk_geom(B, T, C, V);
+        const bool tma = force != 2 && tma_eligible(V, dtype, B, T, C, k, v, r, w, u, state_in);
+        const ChunkGeom g = chunk_geom(B, T, C, V, (tma ? kWsW : kW) * kLS);
         a.nCB = g.nCB;
         a.nLB = g.nLB;
         a.nchunks = g.nchunks;
@@ -271,9 +382,12 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
             if (workspace_bytes < wkv_forward_workspace_bytes(B, T, C, dtype)) return WKV_ERR_WORKSPACE;
             char* ws = static_cast<char*>(workspace);
             a.hdr = reinterpret_cast<wkv::WsHeader*>(ws);
-            a.status = reinterpret_cast<unsigned long long*>(ws + g.status_off);
-            a.agg = reinterpret_cast<float*>(ws + g.agg_off);
-            a.inc = reinterpret_cast<float*>(ws + g.inc_off);
+            a.aggw = reinterpret_cast<wkv::Word*>(ws + g.aggw_off);
+            a.incw = reinterpret_cast<wkv::Word*>(ws + g.incw_off);
+        }
+        if (tma) {
+            return dtype == WKV_F32 ? dispatch_tma<float>(r != nullptr, a, dtype, stream)
+                                    : dispatch_tma<__nv_bfloat16>(r != nullptr, a, dtype, stream);
         }
     }
     if (seq && B * (C / V) > int64_t(0x7fffffff) * 256) return WKV_ERR_SHAPE;

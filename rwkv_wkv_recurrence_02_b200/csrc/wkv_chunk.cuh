@@ -29,25 +29,42 @@
 //           cached exponentials (one more ex2 for the gate, one rcp); the
 //           exact path walks the running-max recurrence.
 //
-// Cross-CTA waits are bounded in time; on expiry the kernel records an error
-// in the workspace and writes NaN for the affected outputs instead of waiting.
+// Cross-chunk protocol: every published state is a 16-byte word per channel
+// carrying the launch epoch and its kind, so readers validate what they read
+// without flags or fences.  Cross-CTA waits are bounded in time; on expiry the
+// kernel records an error in the workspace and writes NaN for the affected
+// outputs instead of waiting.
 #pragma once
+
+#include <cuda.h>
 
 #include "wkv_common.cuh"
 
 namespace wkv {
 
-constexpr uint32_t kStatusAgg = 1;  // chunk summary published
-constexpr uint32_t kStatusInc = 2;  // inclusive state (state after the chunk) published
+constexpr uint32_t kKindAgg = 1;  // chunk summary (from the empty state)
+constexpr uint32_t kKindInc = 2;  // inclusive state (state after the chunk)
 constexpr uint32_t kErrTimeout = 1;
 
 // First 256 bytes of a workspace.
 struct WsHeader {
-    uint32_t epoch;     // launch counter: status words carry it, so no reset is needed between calls
+    uint32_t epoch;     // launch counter: words carry it, so no reset is needed between calls
     uint32_t done;      // CTAs finished in the current launch
     uint32_t error;     // kErrTimeout bits, sticky until the workspace is re-initialised
     uint32_t err_unit;  // a unit that hit the error
+    uint32_t ticket;    // next unit to claim (persistent kernel)
 };
+
+// One published state of one channel, (p, a, b) as is, plus a tag = (launch
+// epoch mod 2^30) << 2 | kind.  Written and read as one aligned 16-byte
+// access, so a reader sees either the whole word or none of it and needs no
+// separate flag or fence.
+struct alignas(16) Word {
+    float p, a, b;
+    uint32_t tag;
+};
+
+__device__ __forceinline__ uint32_t word_tag(uint32_t epoch, uint32_t kind) { return (epoch << 2) | kind; }
 
 struct ChunkArgs {
     const float* w;
@@ -64,22 +81,11 @@ struct ChunkArgs {
     int64_t nchunks;    // ceil(T / TT)
     int64_t units;      // nLB * nchunks
     WsHeader* hdr;      // null when nchunks == 1
-    unsigned long long* status;  // [units]  (epoch << 32) | kind
-    float* agg;         // [units][3][CB]  chunk summaries
-    float* inc;         // [units][3][CB]  states after each chunk
+    Word* aggw;         // [units][CB] chunk summaries
+    Word* incw;         // [units][CB] states after each chunk
     int64_t unit_offset;
     uint64_t wait_limit_ns;
 };
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
     uint32_t v;
@@ -93,94 +99,139 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Spin (with backoff) until the status word of a chunk carries this launch's
-// epoch and a non-zero kind.  Gives up after `limit_ns` of wall time or 2^26
-// polls and returns 0.
-__device__ __noinline__ unsigned long long wait_status(const unsigned long long* addr, uint32_t epoch,
-                                                      uint64_t limit_ns) {
+__device__ __forceinline__ void st_word(Word* dst, St s, uint32_t tag) {
+    asm volatile("st.relaxed.gpu.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(__float_as_uint(s.p)),
+                 "r"(__float_as_uint(s.a)), "r"(__float_as_uint(s.b)), "r"(tag)
+                 : "memory");
+}
+
+__device__ __forceinline__ Word ld_word(const Word* src) {
+    uint32_t p, a, b, t;
+    asm volatile("ld.relaxed.gpu.global.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(p), "=r"(a), "=r"(b), "=r"(t)
+                 : "l"(src)
+                 : "memory");
+    return Word{__uint_as_float(p), __uint_as_float(a), __uint_as_float(b), t};
+}
+
+__device__ __forceinline__ St word_state(const Word& w) { return St{w.p, w.a, w.b}; }
+
+// Each lane publishes the words of its own V channels.
+template <int V>
+__device__ __forceinline__ void publish(Word* dst, const St* val, uint32_t epoch, uint32_t kind, int lane) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) st_word(dst + lane * V + j, val[j], word_tag(epoch, kind));
+}
+
+// Windowed decoupled look-back state, kept by the warp that looks back for
+// one unit: `acc` summarises the chunks already folded (from chunk `cur`+1
+// up to the unit), `span` their token count, `x` the result once `done`.
+template <int V>
+struct LookState {
+    St acc[V];
+    St x[V];
+    int64_t cur;
+    int64_t span;
+    bool done;
+};
+
+constexpr int kWin = 4;
+
+// One round of the look-back: every lane reads the summary and inclusive
+// words of its own channels for chunks cur, cur-1, ..., cur-kWin+1 (one
+// round trip), then the warp walks them nearest first.  A chunk counts as
+// published only if every lane saw its word with this launch's epoch, so all
+// lanes take the same path with data they observed themselves.  The walk
+// stops at the first inclusive state (or at the start of the sequence, where
+// `sin` takes its place) and otherwise folds summaries into acc.  Returns
+// true if it made progress.
+template <int V, int TT>
+__device__ __forceinline__ bool lookback_round(const ChunkArgs& A, int64_t lb, uint32_t epoch, const float* w2,
+                                               const St* sin, LookState<V>& L, int lane) {
+    constexpr int CB = 32 * V;
+    Word wi[kWin][V], wa[kWin][V];
+#pragma unroll
+    for (int l = 0; l < kWin; ++l) {
+        const int64_t c = L.cur - l;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            if (c >= 0) {
+                const int64_t off = (c * A.nLB + lb) * CB + lane * V + j;
+                wi[l][j] = ld_word(A.incw + off);
+                wa[l][j] = ld_word(A.aggw + off);
+            } else {
+                wi[l][j] = Word{0.f, 0.f, 0.f, 0u};
+                wa[l][j] = Word{0.f, 0.f, 0.f, 0u};
+            }
+        }
+    }
+    bool progressed = false;
+#pragma unroll
+    for (int l = 0; l < kWin; ++l) {
+        if (L.cur < 0) {
+#pragma unroll
+            for (int j = 0; j < V; ++j) L.x[j] = st_combine(sin[j], L.acc[j], static_cast<float>(L.span) * w2[j]);
+            L.done = true;
+            return true;
+        }
+        bool inc = true, agg = true;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            inc = inc && wi[l][j].tag == word_tag(epoch, kKindInc);
+            agg = agg && wa[l][j].tag == word_tag(epoch, kKindAgg);
+        }
+        if (__all_sync(0xffffffffu, inc)) {
+#pragma unroll
+            for (int j = 0; j < V; ++j)
+                L.x[j] = st_combine(word_state(wi[l][j]), L.acc[j], static_cast<float>(L.span) * w2[j]);
+            L.done = true;
+            return true;
+        }
+        if (!__all_sync(0xffffffffu, agg)) return progressed;
+#pragma unroll
+        for (int j = 0; j < V; ++j)
+            L.acc[j] = st_combine(word_state(wa[l][j]), L.acc[j], static_cast<float>(L.span) * w2[j]);
+        L.span += TT;
+        L.cur -= 1;
+        progressed = true;
+    }
+    return progressed;
+}
+
+// Blocking look-back: rounds with backoff until the start state is known or
+// `limit_ns` passes (then x is NaN and the function returns false).
+template <int V, int TT>
+__device__ __forceinline__ bool lookback_finish(const ChunkArgs& A, int64_t lb, uint32_t epoch, const float* w2,
+                                                const St* sin, LookState<V>& L, int lane) {
     const uint64_t t0 = global_ns();
     unsigned sleep_ns = 32;
-    for (uint32_t it = 0; it < (1u << 26); ++it) {
-        const unsigned long long s = ld_acquire_u64(addr);
-        if (static_cast<uint32_t>(s >> 32) == epoch && (s & 3ull) != 0ull) return s;
-        if ((it & 7u) == 7u && global_ns() - t0 > limit_ns) return 0ull;
-        __nanosleep(sleep_ns);
-        if (sleep_ns < 512) sleep_ns <<= 1;
-    }
-    return 0ull;
-}
-
-template <int V>
-__device__ __forceinline__ void publish(float* dst, const St* val, unsigned long long* status,
-                                        uint32_t epoch, uint32_t kind, int lane) {
-    constexpr int CB = 32 * V;
+    while (!L.done) {
+        if (!lookback_round<V, TT>(A, lb, epoch, w2, sin, L, lane)) {
+            if (global_ns() - t0 > A.wait_limit_ns) {
+                const float nan = __int_as_float(0x7fc00000);
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-        __stcg(dst + 0 * CB + lane * V + j, val[j].p);
-        __stcg(dst + 1 * CB + lane * V + j, val[j].a);
-        __stcg(dst + 2 * CB + lane * V + j, val[j].b);
-    }
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release_u64(status, (static_cast<unsigned long long>(epoch) << 32) | kind);
-}
-
-template <int V>
-__device__ __forceinline__ void fetch(const float* src, St* val, int lane) {
-    constexpr int CB = 32 * V;
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-        val[j].p = __ldcg(src + 0 * CB + lane * V + j);
-        val[j].a = __ldcg(src + 1 * CB + lane * V + j);
-        val[j].b = __ldcg(src + 2 * CB + lane * V + j);
-    }
-}
-
-// Decoupled look-back, run by one warp: the state at the start of `chunk`
-// for this lane block.  `sin` is the state before chunk 0.
-template <int V, int TT>
-__device__ __forceinline__ void lookback(const ChunkArgs& A, int64_t chunk, int64_t lb, uint32_t epoch,
-                                      const float* w2, const St* sin, St* x, int lane) {
-    constexpr int CB = 32 * V;
-    St acc[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) acc[j] = st_identity();
-    int64_t span = 0;  // tokens summarised by acc (between the found state and `chunk`)
-    for (int64_t c = chunk - 1;; --c) {
-        if (c < 0) {
-#pragma unroll
-            for (int j = 0; j < V; ++j) x[j] = st_combine(sin[j], acc[j], static_cast<float>(span) * w2[j]);
-            return;
-        }
-        const int64_t uj = c * A.nLB + lb;
-        unsigned long long s = 0ull;
-        if (lane == 0) s = wait_status(A.status + uj, epoch, A.wait_limit_ns);
-        s = __shfl_sync(0xffffffffu, s, 0);
-        if (s == 0ull) {
-            if (lane == 0) {
-                atomicOr(&A.hdr->error, kErrTimeout);
-                atomicExch(&A.hdr->err_unit, static_cast<uint32_t>(chunk * A.nLB + lb));
+                for (int j = 0; j < V; ++j) L.x[j] = St{nan, nan, nan};
+                return false;
             }
-#pragma unroll
-            for (int j = 0; j < V; ++j) x[j] = St{__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
-                                                  __int_as_float(0x7fc00000)};
-            return;
+            __nanosleep(sleep_ns);
+            if (sleep_ns < 256) sleep_ns <<= 1;
         }
-        // every lane re-reads the (now ready) word with acquire semantics, so
-        // its own payload loads below are ordered after the producer's stores
-        s = ld_acquire_u64(A.status + uj);
-        const uint32_t kind = static_cast<uint32_t>(s & 3ull);
-        St g[V];
-        fetch<V>((kind == kStatusInc ? A.inc : A.agg) + uj * 3 * CB, g, lane);
-        if (kind == kStatusInc) {
-#pragma unroll
-            for (int j = 0; j < V; ++j) x[j] = st_combine(g[j], acc[j], static_cast<float>(span) * w2[j]);
-            return;
-        }
-#pragma unroll
-        for (int j = 0; j < V; ++j) acc[j] = st_combine(g[j], acc[j], static_cast<float>(span) * w2[j]);
-        span += TT;
     }
+    return true;
+}
+
+template <int V>
+__device__ __forceinline__ void look_init(LookState<V>& L, int64_t chunk) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) L.acc[j] = st_identity();
+    L.cur = chunk - 1;
+    L.span = 0;
+    L.done = false;
+}
+
+__device__ __forceinline__ void record_timeout(const ChunkArgs& A, int64_t unit) {
+    atomicOr(&A.hdr->error, kErrTimeout);
+    atomicExch(&A.hdr->err_unit, static_cast<uint32_t>(unit));
 }
 
 // Thresholds of the fixed-reference fast path, in base-2 exponent units.
@@ -192,15 +243,24 @@ constexpr float kFastSpan = 96.f;
 // stays >= 2^-100 times the current token's term.
 constexpr float kFastState = 100.f;
 
-template <typename IO, int V, bool GATE, int W, int LS, bool FULL>
-__device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V][32], St (&s_x)[V][32]) {
+// One unit (CB channels of one sequence x one chunk of TT tokens), run by
+// the whole CTA.  SMEM selects where the rows come from: false = straight
+// from global memory into registers (all loads issued up front); true = a
+// shared-memory stage that a TMA copy filled (rows read as they are used).
+// `stage` points at the stage's k tile; v and r tiles follow it.
+template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool SMEM>
+__device__ __forceinline__ void unit_body(const ChunkArgs& A, int64_t unit, uint32_t epoch,
+                                          const unsigned char* stage, St (&s_agg)[W][V][32],
+                                          St (&s_x)[V][32]) {
     constexpr int CB = 32 * V;
     constexpr int TT = W * LS;
+    constexpr int ROW = CB * static_cast<int>(sizeof(IO));     // bytes of one tile row
+    constexpr int TILE = TT * ROW;
     using Ld = Vec<IO, V>;
     using Lf = Vec<float, V>;
+    using Raw = typename Ld::raw;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t unit = A.unit_offset + blockIdx.x;
     const int64_t chunk = unit / A.nLB;
     const int64_t lb = unit % A.nLB;
     const int64_t b = lb / A.nCB;
@@ -212,12 +272,6 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
     const int64_t chunk_rows = min(static_cast<int64_t>(TT), T - chunk * TT);
     const int nvalid = FULL ? LS : static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), T - t_seg)));
     const bool need_ws = A.nchunks > 1;
-
-    uint32_t epoch = 0;
-    if (need_ws && warp == W - 1) {
-        if (lane == 0) epoch = ld_relaxed_u32(&A.hdr->epoch);
-        epoch = __shfl_sync(0xffffffffu, epoch, 0);
-    }
 
     // ---- per-channel parameters (base 2) ----
     float w2[V], u2[V], dk[V], eu[V];
@@ -236,24 +290,39 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
         }
     }
 
-    // ---- loads: LS rows x V channels of k, v, r ----
+    // ---- row access ----
     const int64_t base = (b * T + t_seg) * C + c;
     const IO* kp = static_cast<const IO*>(A.k) + base;
     const IO* vp = static_cast<const IO*>(A.v) + base;
     const IO* rp = GATE ? static_cast<const IO*>(A.r) + base : nullptr;
-    typename Ld::raw kr[LS], vr[LS], rr[LS];
+    const unsigned char* srow = stage + warp * LS * ROW + lane * V * static_cast<int>(sizeof(IO));
+    Raw kr[LS], vr[LS], rr[LS];
+    if constexpr (!SMEM) {
 #pragma unroll
-    for (int i = 0; i < LS; ++i) {
-        if (cvalid && (FULL || i < nvalid)) {
-            kr[i] = Ld::load(kp + i * C);
-            vr[i] = Ld::load(vp + i * C);
-            if (GATE) rr[i] = Ld::load(rp + i * C);
-        } else {
-            kr[i] = typename Ld::raw{};
-            vr[i] = typename Ld::raw{};
-            rr[i] = typename Ld::raw{};
+        for (int i = 0; i < LS; ++i) {
+            if (cvalid && (FULL || i < nvalid)) {
+                kr[i] = Ld::load(kp + i * C);
+                vr[i] = Ld::load(vp + i * C);
+                if (GATE) rr[i] = Ld::load(rp + i * C);
+            } else {
+                kr[i] = Raw{};
+                vr[i] = Raw{};
+                rr[i] = Raw{};
+            }
         }
     }
+    auto krow = [&](int i) -> Raw {
+        if constexpr (SMEM) return *reinterpret_cast<const Raw*>(srow + i * ROW);
+        else return kr[i];
+    };
+    auto vrow = [&](int i) -> Raw {
+        if constexpr (SMEM) return *reinterpret_cast<const Raw*>(srow + TILE + i * ROW);
+        else return vr[i];
+    };
+    auto rrow = [&](int i) -> Raw {
+        if constexpr (SMEM) return *reinterpret_cast<const Raw*>(srow + 2 * TILE + i * ROW);
+        else return rr[i];
+    };
 
     // ---- pass 0: key range and running-max exponent of the segment ----
     float kf[LS][V];
@@ -267,9 +336,10 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
 #pragma unroll
     for (int i = 0; i < LS; ++i) {
         if (FULL || i < nvalid) {
+            const Raw kk = krow(i);
 #pragma unroll
             for (int j = 0; j < V; ++j) {
-                const float k2 = Ld::get(kr[i], j) * kLog2e;
+                const float k2 = Ld::get(kk, j) * kLog2e;
                 kf[i][j] = k2;
                 kmax[j] = fmaxf(kmax[j], k2);
                 kmin[j] = fminf(kmin[j], k2);
@@ -293,19 +363,20 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < nvalid) {
+                const Raw vv = vrow(i);
 #pragma unroll
                 for (int j = 0; j < V; ++j) {
                     const float ek = ex2(kf[i][j] - kmax[j]);
                     kf[i][j] = ek;
-                    n[j] = fmaf(n[j], dk[j], ek * Ld::get(vr[i], j));
+                    n[j] = fmaf(n[j], dk[j], ek * Ld::get(vv, j));
                     db[j] = fmaf(db[j], dk[j], ek);
                 }
             }
         }
 #pragma unroll
         for (int j = 0; j < V; ++j) {
-            const float s = ex2(kmax[j] - q[j]);
-            seg[j] = St{q[j], n[j] * s, db[j] * s};
+            const float sc = ex2(kmax[j] - q[j]);
+            seg[j] = St{q[j], n[j] * sc, db[j] * sc};
         }
     } else {
 #pragma unroll
@@ -313,9 +384,10 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < nvalid) {
+                const Raw vr_ = vrow(i);
 #pragma unroll
                 for (int j = 0; j < V; ++j) {
-                    const float vv = Ld::get(vr[i], j);
+                    const float vv = Ld::get(vr_, j);
                     const float pd = seg[j].p - w2[j];
                     const float d2 = pd - kf[i][j];
                     const float e = ex2(-fabsf(d2));
@@ -340,10 +412,10 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
     St lp[V];  // summary of segments 0..warp-1
 #pragma unroll
     for (int j = 0; j < V; ++j) lp[j] = st_identity();
-    for (int s = 0; s < warp; ++s) {
-        const int len = FULL ? LS : static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), chunk_rows - s * LS)));
+    for (int sg = 0; sg < warp; ++sg) {
+        const int len = FULL ? LS : static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), chunk_rows - sg * LS)));
 #pragma unroll
-        for (int j = 0; j < V; ++j) lp[j] = st_combine(lp[j], s_agg[s][j][lane], static_cast<float>(len) * w2[j]);
+        for (int j = 0; j < V; ++j) lp[j] = st_combine(lp[j], s_agg[sg][j][lane], static_cast<float>(len) * w2[j]);
     }
     if (warp == W - 1) {
         St agg[V], sin[V], x[V];
@@ -358,18 +430,22 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
             }
         }
         const bool last = chunk == A.nchunks - 1;
-        const int64_t uoff = unit * 3 * CB;
+        const int64_t uoff = unit * CB;
         if (chunk == 0) {
 #pragma unroll
             for (int j = 0; j < V; ++j) x[j] = sin[j];
         } else {
-            if (!last) publish<V>(A.agg + uoff, agg, A.status + unit, epoch, kStatusAgg, lane);
-            lookback<V, TT>(A, chunk, lb, epoch, w2, sin, x, lane);
+            if (!last) publish<V>(A.aggw + uoff, agg, epoch, kKindAgg, lane);
+            LookState<V> L;
+            look_init<V>(L, chunk);
+            if (!lookback_finish<V, TT>(A, lb, epoch, w2, sin, L, lane) && lane == 0) record_timeout(A, unit);
+#pragma unroll
+            for (int j = 0; j < V; ++j) x[j] = L.x[j];
         }
         St incl[V];
 #pragma unroll
         for (int j = 0; j < V; ++j) incl[j] = st_combine(x[j], agg[j], static_cast<float>(chunk_rows) * w2[j]);
-        if (need_ws && !last) publish<V>(A.inc + uoff, incl, A.status + unit, epoch, kStatusInc, lane);
+        if (need_ws && !last) publish<V>(A.incw + uoff, incl, epoch, kKindInc, lane);
         if (last && A.s_out != nullptr && cvalid) {
 #pragma unroll
             for (int j = 0; j < V; ++j) {
@@ -381,15 +457,6 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
         }
 #pragma unroll
         for (int j = 0; j < V; ++j) s_x[j][lane] = x[j];
-        if (need_ws && lane == 0) {
-            const uint32_t before = atomicAdd(&A.hdr->done, 1u);
-            if (before == static_cast<uint32_t>(A.units - 1)) {
-                // every CTA of this launch has read the epoch; start the next one
-                A.hdr->done = 0u;
-                __threadfence();
-                atomicAdd(&A.hdr->epoch, 1u);
-            }
-        }
     }
     __syncthreads();
     if (nvalid == 0 || !cvalid) return;
@@ -420,14 +487,17 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < nvalid) {
+                const Raw vv = vrow(i);
+                Raw rv{};
+                if (GATE) rv = rrow(i);
                 float out[V];
 #pragma unroll
                 for (int j = 0; j < V; ++j) {
                     const float ek = kf[i][j] * sl[j];
-                    const float ekv = ek * Ld::get(vr[i], j);
+                    const float ekv = ek * Ld::get(vv, j);
                     const float num = fmaf(eu[j], ekv, n[j]);
                     float den = fmaf(eu[j], ek, db[j]);
-                    if (GATE) den *= gate_den(Ld::get(rr[i], j));
+                    if (GATE) den *= gate_den(Ld::get(rv, j));
                     out[j] = num * rcp(den);
                     n[j] = fmaf(n[j], dk[j], ekv);
                     db[j] = fmaf(db[j], dk[j], ek);
@@ -441,7 +511,9 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
 #pragma unroll
             for (int i = 0; i < LS; ++i) {
                 if (FULL || i < nvalid) {
-                    const auto kk = Ld::load(kp + i * C);
+                    Raw kk;
+                    if constexpr (SMEM) kk = krow(i);
+                    else kk = Ld::load(kp + i * C);
 #pragma unroll
                     for (int j = 0; j < V; ++j) kf[i][j] = Ld::get(kk, j) * kLog2e;
                 }
@@ -450,12 +522,15 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < nvalid) {
+                const Raw vv = vrow(i);
+                Raw rv{};
+                if (GATE) rv = rrow(i);
                 float out[V];
 #pragma unroll
                 for (int j = 0; j < V; ++j) {
-                    const float gd = GATE ? gate_den(Ld::get(rr[i], j)) : 1.f;
-                    out[j] = lane_token(st[j].a, st[j].b, st[j].p, w2[j], u2[j], kf[i][j],
-                                        Ld::get(vr[i], j), gd, 1.f);
+                    const float gd = GATE ? gate_den(Ld::get(rv, j)) : 1.f;
+                    out[j] = lane_token(st[j].a, st[j].b, st[j].p, w2[j], u2[j], kf[i][j], Ld::get(vv, j), gd,
+                                        1.f);
                 }
                 Ld::store(yp + i * C, out);
             }
@@ -463,18 +538,86 @@ __device__ __forceinline__ void chunk_body(const ChunkArgs& A, St (&s_agg)[W][V]
     }
 }
 
+// Last CTA of a launch (by the count of finished CTAs) starts the next
+// launch's epoch and resets the counters.  Every CTA read the epoch before
+// it counted itself, so no CTA of this launch can see the new value.
+__device__ __forceinline__ void finish_launch(const ChunkArgs& A, uint32_t ctas) {
+    const uint32_t before = atomicAdd(&A.hdr->done, 1u);
+    if (before == ctas - 1u) {
+        A.hdr->done = 0u;
+        A.hdr->ticket = 0u;
+        __threadfence();
+        atomicAdd(&A.hdr->epoch, 1u);
+    }
+}
+
+// One unit per CTA, rows loaded from global memory into registers.  Takes
+// any alignment that the vector width allows.
 template <typename IO, int V, bool GATE, int W, int LS>
 __global__ void __launch_bounds__(W * 32)
 chunk_forward_kernel(const ChunkArgs A) {
     __shared__ St s_agg[W][V][32];
     __shared__ St s_x[V][32];
+    __shared__ uint32_t s_epoch;
     constexpr int TT = W * LS;
     const int64_t unit = A.unit_offset + blockIdx.x;
     const int64_t chunk = unit / A.nLB;
+    const bool need_ws = A.nchunks > 1;
+    if (threadIdx.x == 0) s_epoch = need_ws ? ld_relaxed_u32(&A.hdr->epoch) : 0u;
+    __syncthreads();
+    const uint32_t epoch = s_epoch;
     if ((chunk + 1) * TT <= A.T)
-        chunk_body<IO, V, GATE, W, LS, true>(A, s_agg, s_x);
+        unit_body<IO, V, GATE, W, LS, true, false>(A, unit, epoch, nullptr, s_agg, s_x);
     else
-        chunk_body<IO, V, GATE, W, LS, false>(A, s_agg, s_x);
+        unit_body<IO, V, GATE, W, LS, false, false>(A, unit, epoch, nullptr, s_agg, s_x);
+    if (need_ws && threadIdx.x == 0) finish_launch(A, static_cast<uint32_t>(A.units));
+}
+
+// ---------------------------------------------------------------------------
+// persistent kernel: TMA tiles into a shared-memory ring, one unit per turn
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for a phase of an mbarrier; false after `limit_ns` (or 2^26 polls).
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 0; it < (1u << 26); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 15u && global_ns() - t0 > limit_ns) return false;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
 }
 
 }  // namespace wkv

@@ -105,13 +105,13 @@ def test_forward_workspace_checks(L):
 def test_workspace_size_rules(L):
     # short sequences take the sequential kernel and need no workspace
     assert L.wkv_forward_workspace_bytes(4, 16, 128, F32) == 0
-    assert L.wkv_forward_workspace_bytes(4, 64, 128, F32) == 0     # a single chunk
+    assert L.wkv_forward_workspace_bytes(4, 32, 128, F32) == 0     # a single chunk
     assert L.wkv_forward_workspace_bytes(-1, 64, 128, F32) == 0
     small = L.wkv_forward_workspace_bytes(8, 1024, 2048, F32)
     big = L.wkv_forward_workspace_bytes(8, 4096, 2048, F32)
     assert 0 < small < big
-    # bounded by a few bytes per element: 2 states of 12 B per lane per chunk
-    assert small < 8 * 1024 * 2048
+    # two 16-byte words per lane per 32-token chunk: about one byte per element
+    assert small < 2 * 8 * 1024 * 2048
 
 
 def test_workspace_init_and_status_validation(L):

@@ -251,8 +251,7 @@ def test_stream_1m_chunked_equals_single_pass():
         wkv.wkv_forward(w, u, k[:, sl], v[:, sl], None, state, y=y_chain[:, sl], state_out=state)
     torch.cuda.synchronize()
     idx = sample_channels(C, n=24)
-    ds = dict(w=w[idx].cpu(), u=u[idx].cpu(), k=k[..., idx].cpu(), v=v[..., idx].cpu(), r=None, state=None)
-    y_ref, s_ref, scale = oracle_forward(**ds)
+    y_ref, s_ref, scale = oracle_forward(w[idx].cpu(), u[idx].cpu(), k[..., idx].cpu(), v[..., idx].cpu())
     dv = idx.to(DEV)
     assert output_error(y_single[..., dv], y_ref, scale) <= 1e-2
     assert output_error(y_chain[..., dv], y_ref, scale) <= 1e-2
