@@ -14,6 +14,7 @@
 #include "../../include/wkv.h"
 #include "wkv_chunk.cuh"
 #include "wkv_chunk_ws.cuh"
+#include "wkv_lane.cuh"
 #include "wkv_seq.cuh"
 #include "wkv_step.cuh"
 
@@ -180,7 +181,9 @@ bool tma_eligible(int V, int dtype, int64_t B, int64_t T, int64_t C, const void*
 }
 
 // Kernel choice: 0 = automatic; the environment variable WKV_FORWARD_KERNEL
-// (seq | chunk | tma) forces one, for ablation measurements.
+// (seq | chunk | tma | lookback) forces one, for ablation measurements:
+// chunk = register-load look-back kernel, lookback = TMA look-back kernel
+// even where the lane-resident one would run.
 int forced_kernel() {
     static int f = []() {
         const char* e = std::getenv("WKV_FORWARD_KERNEL");
@@ -188,6 +191,7 @@ int forced_kernel() {
         if (std::strcmp(e, "seq") == 0) return 1;
         if (std::strcmp(e, "chunk") == 0) return 2;
         if (std::strcmp(e, "tma") == 0) return 3;
+        if (std::strcmp(e, "lookback") == 0) return 4;
         return 0;
     }();
     return f;
@@ -222,6 +226,45 @@ int launch_tma(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
     const int64_t grid = a.units < capacity[dev] ? a.units : capacity[dev];
     kern<<<static_cast<unsigned>(grid), G::THREADS, G::SMEM, st>>>(tk, tv, tr, a);
     return check_launch();
+}
+
+// Lane-resident kernel: each CTA owns whole lane blocks; grid = min(lane
+// blocks, resident capacity).
+template <typename IO, bool GATE, int STAGES>
+int launch_lane(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
+    using G = wkv::LaneGeometry<IO, 2, GATE, kW, kLS, STAGES>;
+    auto kern = wkv::lane_forward_kernel<IO, 2, GATE, kW, kLS, STAGES>;
+    static int capacity[kMaxDevices] = {0};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (capacity[dev] == 0) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        int per_sm = 0;
+        rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+    }
+    CUtensorMap tk, tv, tr;
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
+        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT))
+        return WKV_ERR_CUDA;
+    if (GATE) {
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT)) return WKV_ERR_CUDA;
+    } else {
+        tr = tv;
+    }
+    const int64_t grid = a.nLB < capacity[dev] ? a.nLB : capacity[dev];
+    kern<<<static_cast<unsigned>(grid), G::THREADS, G::SMEM, st>>>(tk, tv, tr, a);
+    return check_launch();
+}
+
+template <typename IO>
+int dispatch_lane(bool gate, const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
+    constexpr int S = sizeof(IO) == 4 ? 2 : 3;   // two CTAs per SM either way
+    return gate ? launch_lane<IO, true, S>(a, dtype, st) : launch_lane<IO, false, S>(a, dtype, st);
 }
 
 template <typename IO>
@@ -369,6 +412,17 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     int64_t grid = 0;
     if (!seq) {
         const bool tma = force != 2 && tma_eligible(V, dtype, B, T, C, k, v, r, w, u, state_in);
+        // enough lane blocks to give every SM its own: no cross-CTA split
+        const bool lane_resident = tma && force != 4 && B * ((C + 63) / 64) >= sm_count();
+        if (lane_resident) {
+            const ChunkGeom g = chunk_geom(B, T, C, 2, kW * kLS);
+            a.nCB = g.nCB;
+            a.nLB = g.nLB;
+            a.nchunks = g.nchunks;
+            a.units = g.units;
+            return dtype == WKV_F32 ? dispatch_lane<float>(r != nullptr, a, dtype, stream)
+                                    : dispatch_lane<__nv_bfloat16>(r != nullptr, a, dtype, stream);
+        }
         const ChunkGeom g = chunk_geom(B, T, C, V, (tma ? kWsW : kW) * kLS);
         a.nCB = g.nCB;
         a.nLB = g.nLB;

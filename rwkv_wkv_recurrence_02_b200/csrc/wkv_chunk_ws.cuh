@@ -67,8 +67,24 @@ struct SegCtx {
     bool cvalid, fast1;
 };
 
+// Per-channel parameters of this thread's V channels (base 2): w2, u2 and
+// the per-step decay 2^-w2 and bonus factor 2^u2.  Channels past C get
+// harmless stand-ins.
+template <int V, int LS>
+__device__ __forceinline__ void set_params(SegCtx<V, LS>& cx, const float* w, const float* u) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        cx.w2[j] = cx.cvalid ? w[j] * kLog2e : 1.f;
+        cx.u2[j] = cx.cvalid ? u[j] * kLog2e : 0.f;
+        cx.dk[j] = ex2(-cx.w2[j]);
+        cx.eu[j] = ex2(cx.u2[j]);
+    }
+}
+
 // Pass 0 + pass 1 of one warp's segment; returns the segment summary.
-template <typename IO, int V, bool GATE, int W, int LS, bool FULL>
+// PARAMS_IN_STAGE: read w, u from the stage's parameter area (else the
+// caller has set them in cx already).
+template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool PARAMS_IN_STAGE = true>
 __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t unit, const unsigned char* stage,
                                            SegCtx<V, LS>& cx, St* seg) {
     constexpr int CB = 32 * V;
@@ -76,7 +92,6 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t unit, con
     constexpr int ROW = CB * static_cast<int>(sizeof(IO));
     constexpr int TILE = TT * ROW;
     using Ld = Vec<IO, V>;
-    using Lf = Vec<float, V>;
     using Raw = typename Ld::raw;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t chunk = unit / A.nLB, lb = unit % A.nLB;
@@ -86,16 +101,8 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t unit, con
     const int64_t t_seg = chunk * TT + static_cast<int64_t>(warp) * LS;
     cx.nvalid = FULL ? LS : static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), A.T - t_seg)));
     cx.base = (b * A.T + t_seg) * A.C + c;
-    {
-        const float* prm = reinterpret_cast<const float*>(stage + NARR_OF<GATE>() * TILE);
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            cx.w2[j] = cx.cvalid ? prm[lane * V + j] * kLog2e : 1.f;
-            cx.u2[j] = cx.cvalid ? prm[CB + lane * V + j] * kLog2e : 0.f;
-            cx.dk[j] = ex2(-cx.w2[j]);
-            cx.eu[j] = ex2(cx.u2[j]);
-        }
-    }
+    if (PARAMS_IN_STAGE) set_params<V>(cx, reinterpret_cast<const float*>(stage + NARR_OF<GATE>() * TILE) + lane * V,
+                                       reinterpret_cast<const float*>(stage + NARR_OF<GATE>() * TILE) + CB + lane * V);
     const unsigned char* srow = stage + warp * LS * ROW + lane * V * static_cast<int>(sizeof(IO));
     float q[V];
 #pragma unroll
@@ -266,7 +273,10 @@ __device__ __forceinline__ bool compute_front(const ChunkArgs& A, int64_t it, un
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int s = static_cast<int>(it % S);
     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-    if (!mbar_wait(&full[s], ph, A.wait_limit_ns)) return false;
+    if (!mbar_wait(&full[s], ph, A.wait_limit_ns)) {
+        if (threadIdx.x == 0 && A.hdr != nullptr) record_timeout(A, -1);
+        return false;
+    }
     const int64_t u = unitbuf[s];
     if (u >= A.units) return false;
     const unsigned char* stage = smem + s * G::STAGE;
@@ -293,6 +303,7 @@ __device__ __forceinline__ bool compute_back(const ChunkArgs& A, int64_t it, uns
     const int s = static_cast<int>(it % S);
     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
     const bool ok = mbar_wait(&xready[s], ph, A.wait_limit_ns);
+    if (!ok && threadIdx.x == 0 && A.hdr != nullptr) record_timeout(A, -1);
     const int64_t u = unitbuf[s];
     const int64_t chunk = u / A.nLB;
     if (ok && cx.nvalid > 0 && cx.cvalid) {
@@ -322,6 +333,21 @@ __device__ __forceinline__ bool compute_back(const ChunkArgs& A, int64_t it, uns
     return ok;
 }
 
+// Scan warps skip ring positions (each takes every SCAN-th), so the end of
+// the stream can land on a position another warp owns: wait for a phase OR
+// for the producer's end position to be at or before `it`.  1 = phase
+// complete, 0 = end of stream, -1 = timed out.
+__device__ __noinline__ int mbar_wait_or_end(uint64_t* bar, uint32_t parity, const volatile int64_t* endpos,
+                                             int64_t it, uint64_t limit_ns) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t n = 0; n < (1u << 26); ++n) {
+        if (mbar_try_wait(bar, parity)) return 1;
+        if (*endpos <= it) return 0;
+        if ((n & 15u) == 15u && global_ns() - t0 > limit_ns) return -1;
+    }
+    return -1;
+}
+
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                      smem_u32(dst)),
@@ -339,6 +365,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[S], empty[S], aggready[S], xready[S], foldready[S];
     __shared__ int64_t unitbuf[S];
+    __shared__ int64_t s_endpos;   // first ring position with no unit (set by the producer)
     __shared__ uint32_t s_epoch;
     St* aggbuf = reinterpret_cast<St*>(smem + S * G::STAGE);                 // [S][W][V][32]
     St* xbuf = reinterpret_cast<St*>(smem + S * (G::STAGE + G::AGGBUF));     // [S][V][32]
@@ -358,9 +385,11 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_epoch = ticket ? ld_relaxed_u32(&A.hdr->epoch) : 0u;
+        s_endpos = INT64_MAX;
     }
     __syncthreads();
     const uint32_t epoch = s_epoch;
+    volatile int64_t* endpos = &s_endpos;
 
     if (warp == kProducer) {
         // ---------------- producer ----------------
@@ -370,15 +399,15 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                 const int s = static_cast<int>(it % S);
                 if (it >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((it / S) - 1) & 1), A.wait_limit_ns)) {
                     if (ticket) record_timeout(A, -1);
-                    unitbuf[s] = A.units;
-                    mbar_arrive(&full[s]);
+                    *endpos = it;
                     break;
                 }
                 const int64_t u = ticket ? static_cast<int64_t>(atomicAdd(&A.hdr->ticket, 1u))
                                          : static_cast<int64_t>(blockIdx.x) + it * gridDim.x;
                 unitbuf[s] = u;
                 if (u >= A.units) {
-                    mbar_arrive(&full[s]);  // end of the stream for this CTA
+                    *endpos = it;           // end of the stream for this CTA
+                    mbar_arrive(&full[s]);
                     break;
                 }
                 const int64_t chunk = u / A.nLB, lb = u % A.nLB;
@@ -413,7 +442,10 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         for (int64_t it = 0;; ++it) {
             const int s = static_cast<int>(it % S);
             const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-            if (!mbar_wait(&full[s], ph, A.wait_limit_ns)) break;
+            if (!mbar_wait(&full[s], ph, A.wait_limit_ns)) {
+                if (lane == 0 && ticket) record_timeout(A, -1);
+                break;
+            }
             const int64_t u = unitbuf[s];
             if (u >= A.units) break;
             const int64_t chunk = u / A.nLB, lb = u % A.nLB;
@@ -425,6 +457,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
 #pragma unroll
             for (int j = 0; j < V; ++j) w2[j] = cvalid ? prm[lane * V + j] * kLog2e : 1.f;
             const bool ok = mbar_wait(&aggready[s], ph, A.wait_limit_ns);
+            if (!ok && lane == 0 && ticket) record_timeout(A, -1);
             St agg[V];
             const St* ab = aggbuf + static_cast<int64_t>(s) * W * V * 32;
 #pragma unroll
@@ -451,7 +484,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         for (int64_t it = warp - W;; it += G::SCAN) {
             const int s = static_cast<int>(it % S);
             const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-            if (!mbar_wait(&full[s], ph, A.wait_limit_ns)) break;
+            const int got = mbar_wait_or_end(&full[s], ph, endpos, it, A.wait_limit_ns);
+            if (got < 0 && lane == 0 && ticket) record_timeout(A, -1);
+            if (got <= 0) break;
             const int64_t u = unitbuf[s];
             if (u >= A.units) break;
             const int64_t chunk = u / A.nLB, lb = u % A.nLB;

@@ -73,6 +73,25 @@ def test_small_shapes(B, T, C, dtype, gate, state):
     check_forward(d, y, s)
 
 
+# Shapes with at least one 64-channel block per SM take the lane-resident
+# kernel (each CTA walks whole sequences of its channels).
+LANE = [
+    # B, T, C, dtype, gate, state
+    (4, 333, 2436, torch.float32, True, True),     # ragged channel block and ragged last chunk
+    (40, 130, 256, torch.bfloat16, True, False),
+    (3, 1000, 3200, torch.bfloat16, False, True),
+    (160, 64, 64, torch.float32, False, True),     # exactly one chunk per lane block
+    (300, 40, 64, torch.bfloat16, True, True),     # more lane blocks than CTA slots, short T
+]
+
+
+@pytest.mark.parametrize("B,T,C,dtype,gate,state", LANE)
+def test_lane_resident_shapes(B, T, C, dtype, gate, state):
+    d = gen_case(B, T, C, dtype, gate, state, seed=B * 7 + T + C)
+    y, s = run_forward(d)
+    check_forward(d, y, s)
+
+
 def test_tiny_workload_against_brute_force():
     d = I.make_forward_inputs("tiny", device=DEV)
     y, s = run_forward(d)
@@ -185,6 +204,25 @@ def test_guard_bands_untouched(dtype):
     assert torch.all(ybuf[:pad] == 12345.0) and torch.all(ybuf[pad + n:] == 12345.0)
     assert torch.all(sbuf[:pad] == 777.0) and torch.all(sbuf[pad + 3 * B * C:] == 777.0)
     check_forward(d, y, s)
+
+
+def test_calls_finish_promptly():
+    """No launch ends by a bounded wait running out: 16 chained calls on a
+    many-chunk shape finish far inside one wait limit (1 s), and the
+    workspace reports no error."""
+    d = gen_case(1, 2048, 4096, torch.bfloat16, False, False, seed=29)
+    ws = wkv.Workspace()
+    st = I.fresh_state(1, 4096, device=DEV)
+    wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], None, st, state_out=st, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(16):
+        wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], None, st, state_out=st, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    assert e0.elapsed_time(e1) < 200.0
+    assert ws.status() == 0
 
 
 def test_workspace_reuse_across_shapes():
