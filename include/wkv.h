@@ -63,7 +63,8 @@ typedef enum {
     WKV_ERR_ALIAS = -5,      /* an output overlaps an input or another output */
     WKV_ERR_CUDA = -6,       /* CUDA launch error; see wkv_last_cuda_error() */
     WKV_ERR_TIMEOUT = -7,    /* a cross-block wait on the GPU gave up (from wkv_workspace_status) */
-    WKV_ERR_WORKSPACE = -8   /* workspace NULL or smaller than wkv_forward_workspace_bytes() */
+    WKV_ERR_WORKSPACE = -8,  /* workspace NULL or smaller than wkv_forward_workspace_bytes() */
+    WKV_ERR_SCRATCH = -9     /* wkv_forward_noalloc: problem needs more than its built-in scratch */
 } wkv_status;
 
 /*
@@ -134,6 +135,44 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype,
              const float* w, const float* u,
              const void* k, const void* v, const void* r,
              float* state, void* y, cudaStream_t stream);
+
+/*
+ * wkv_forward_noalloc -- wkv_forward for callers that cannot allocate device
+ * memory: code running where cudaMalloc is unavailable or forbidden (a
+ * plug-in inside a host application that owns every allocation, a runtime
+ * that hands out only pre-registered buffers, or a pre-recorded launch
+ * sequence that must not touch the allocator).  The paper has no counterpart
+ * to this entry point; it only changes where the scratch memory comes from.
+ *
+ * Same arguments and results as wkv_forward, without the workspace.  The
+ * cross-block scratch the chunked kernel needs comes from a fixed array
+ * inside the library (WKV_NOALLOC_SCRATCH_BYTES bytes of device memory that
+ * every GPU which loads the library keeps until the process exits), so
+ * nothing is allocated.
+ *
+ *   - Limit: problems whose scratch need (wkv_forward_noalloc_scratch_bytes)
+ *     exceeds WKV_NOALLOC_SCRATCH_BYTES are rejected with WKV_ERR_SCRATCH
+ *     before anything runs.  Sequences of at most 64 tokens need none.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing a stream into a graph.
+ *   - Every call on a device shares the one array and clears the part it
+ *     uses at the start (a cudaMemsetAsync on `stream`).  Calls that may
+ *     overlap on the GPU (different streams without ordering) race on it
+ *     and give wrong results; order them.
+ *   - A cross-block wait that runs out is recorded in the array like in a
+ *     workspace; the next call clears it.
+ */
+#define WKV_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype,
+                        const float* w, const float* u,
+                        const void* k, const void* v, const void* r,
+                        const float* state_in, void* y, float* state_out,
+                        cudaStream_t stream);
+
+/* Scratch bytes wkv_forward_noalloc would use for these sizes (0: none). */
+size_t wkv_forward_noalloc_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype);
 
 /* Static English text for a wkv_status value. */
 const char* wkv_strerror(int status);

@@ -26,11 +26,12 @@ WKV_BF16 = 1
 STATUS = {
     0: "WKV_OK", -1: "WKV_ERR_NULLPTR", -2: "WKV_ERR_SHAPE", -3: "WKV_ERR_DTYPE",
     -4: "WKV_ERR_ALIGN", -5: "WKV_ERR_ALIAS", -6: "WKV_ERR_CUDA", -7: "WKV_ERR_TIMEOUT",
-    -8: "WKV_ERR_WORKSPACE",
+    -8: "WKV_ERR_WORKSPACE", -9: "WKV_ERR_SCRATCH",
 }
 # the functions include/wkv.h declares
 EXPORTS = ("wkv_forward", "wkv_forward_workspace_bytes", "wkv_workspace_init", "wkv_workspace_status",
-           "wkv_step", "wkv_strerror", "wkv_last_cuda_error", "wkv_abi_version")
+           "wkv_step", "wkv_forward_noalloc", "wkv_forward_noalloc_scratch_bytes", "wkv_strerror",
+           "wkv_last_cuda_error", "wkv_abi_version")
 
 _lib = None
 _lock = threading.Lock()
@@ -69,6 +70,10 @@ def lib():
         L.wkv_workspace_status.restype = i32
         L.wkv_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.wkv_step.restype = i32
+        L.wkv_forward_noalloc.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.wkv_forward_noalloc.restype = i32
+        L.wkv_forward_noalloc_scratch_bytes.argtypes = [i64, i64, i64, i32]
+        L.wkv_forward_noalloc_scratch_bytes.restype = sz
         L.wkv_strerror.argtypes = [i32]
         L.wkv_strerror.restype = ctypes.c_char_p
         L.wkv_last_cuda_error.argtypes = []
@@ -206,6 +211,27 @@ def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, wa
     ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
     _check(lib().wkv_forward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
                              _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, _stream_ptr(stream)), "wkv_forward")
+    return y, state_out
+
+
+def wkv_forward_noalloc(w, u, k, v, r=None, state_in=None, *, y, state_out=None, stream=None):
+    """wkv_forward without a workspace, for callers that cannot allocate device
+    memory: the scratch comes from a fixed array inside the library.  The
+    caller supplies every output buffer (y, and state_out if wanted); this
+    function allocates nothing.  Raises WkvError(WKV_ERR_SCRATCH) for problems
+    larger than the built-in scratch.  Calls must be ordered on the GPU."""
+    torch = _torch()
+    B, T, C = k.shape
+    dev = k.device
+    code = _dtype_code(k)
+    for t, name in ((v, "v"), (r, "r"), (y, "y")):
+        _need(t, name, (B, T, C), k.dtype, dev)
+    _need(w, "w", (C,), torch.float32, dev)
+    _need(u, "u", (C,), torch.float32, dev)
+    _need(state_in, "state_in", (3, B, C), torch.float32, dev)
+    _need(state_out, "state_out", (3, B, C), torch.float32, dev)
+    _check(lib().wkv_forward_noalloc(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
+                                     _ptr(y), _ptr(state_out), _stream_ptr(stream)), "wkv_forward_noalloc")
     return y, state_out
 
 

@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/wkv.h"
 #include "wkv_chunk.cuh"
@@ -316,6 +317,7 @@ const char* wkv_strerror(int status) {
         case WKV_ERR_CUDA: return "CUDA error (see wkv_last_cuda_error)";
         case WKV_ERR_TIMEOUT: return "a cross-block wait on the GPU gave up; affected outputs are NaN";
         case WKV_ERR_WORKSPACE: return "workspace missing or smaller than wkv_forward_workspace_bytes()";
+        case WKV_ERR_SCRATCH: return "problem needs more scratch than wkv_forward_noalloc's built-in array";
         default: return "unknown wkv status";
     }
 }
@@ -493,4 +495,131 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype, const float* w, const f
     return check_launch();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant of wkv_forward.  The chunked look-back kernel's
+// cross-block scratch lives in this fixed device array instead of a caller
+// workspace.  Host code cannot use the array's name as a device address, so
+// the address is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
 }  // extern "C"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[WKV_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on the current device (looked up on
+// the first call per device, with that device current).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        rc = record_cuda(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+        if (rc != WKV_OK) return rc;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return WKV_OK;
+}
+
+// Scratch of the register-load look-back kernel (chunks of kW * kLS tokens)
+// at the vector width the call will use; 0 when one chunk covers T.
+size_t noalloc_need(int64_t B, int64_t T, int64_t C, int V) {
+    if (T <= kSeqMaxT) return 0;
+    return chunk_geom(B, T, C, V, kW * kLS).bytes;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wkv_forward_noalloc_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype) {
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n) || n == 0 || (dtype != WKV_F32 && dtype != WKV_BF16)) return 0;
+    const size_t a = noalloc_need(B, T, C, 1), b = noalloc_need(B, T, C, 2);
+    return a > b ? a : b;
+}
+
+int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                        const void* k, const void* v, const void* r, const float* state_in, void* y,
+                        float* state_out, cudaStream_t stream) {
+    if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
+    if (B == 0 || C == 0 || T <= kSeqMaxT) {
+        // nothing to do, or a sequence short enough for the kernel that needs
+        // no scratch: the regular entry point does exactly that
+        return wkv_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, nullptr, 0, stream);
+    }
+    if (!w || !u || !k || !v || !y) return WKV_ERR_NULLPTR;
+    const size_t eb = elem_bytes(dtype);
+    if (!aligned(w, 4) || !aligned(u, 4) || !aligned(k, eb) || !aligned(v, eb) || !aligned(y, eb) ||
+        (r && !aligned(r, eb)) || (state_in && !aligned(state_in, 4)) || (state_out && !aligned(state_out, 4)))
+        return WKV_ERR_ALIGN;
+    const size_t io_bytes = size_t(n) * eb, st_bytes = size_t(B * C) * 3 * 4, p_bytes = size_t(C) * 4;
+    const void* ins[] = {k, v, r};
+    for (const void* p : ins)
+        if (overlaps(y, io_bytes, p, io_bytes) || (state_out && overlaps(state_out, st_bytes, p, io_bytes)))
+            return WKV_ERR_ALIAS;
+    if (overlaps(y, io_bytes, w, p_bytes) || overlaps(y, io_bytes, u, p_bytes) ||
+        overlaps(y, io_bytes, state_in, st_bytes) || overlaps(y, io_bytes, state_out, st_bytes))
+        return WKV_ERR_ALIAS;
+    if (state_out && (overlaps(state_out, st_bytes, w, p_bytes) || overlaps(state_out, st_bytes, u, p_bytes) ||
+                      (state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes))))
+        return WKV_ERR_ALIAS;
+
+    const void* io[] = {k, v, r, y};
+    const float* f32[] = {w, u, state_in, state_out};
+    const int V = pick_vec(C, dtype, io, 4, f32, 4);
+    const ChunkGeom g = chunk_geom(B, T, C, V, kW * kLS);
+    if (g.units > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    if (g.bytes > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_SCRATCH;
+
+    wkv::ChunkArgs a{};
+    a.w = w;
+    a.u = u;
+    a.k = k;
+    a.v = v;
+    a.r = r;
+    a.s_in = state_in;
+    a.y = y;
+    a.s_out = state_out;
+    a.B = B;
+    a.T = T;
+    a.C = C;
+    a.nCB = g.nCB;
+    a.nLB = g.nLB;
+    a.nchunks = g.nchunks;
+    a.units = g.units;
+    a.wait_limit_ns = kWaitLimitNs;
+    if (g.bytes > 0) {
+        void* ws = nullptr;
+        int rc = noalloc_scratch(&ws);
+        if (rc != WKV_OK) return rc;
+        // every call starts from a zeroed header and zeroed words: counters,
+        // error word and epoch at 0, and no word left over from an earlier call
+        rc = record_cuda(cudaMemsetAsync(ws, 0, g.bytes, stream));
+        if (rc != WKV_OK) return rc;
+        char* base = static_cast<char*>(ws);
+        a.hdr = reinterpret_cast<wkv::WsHeader*>(base);
+        a.aggw = reinterpret_cast<wkv::Word*>(base + g.aggw_off);
+        a.incw = reinterpret_cast<wkv::Word*>(base + g.incw_off);
+    }
+    if (dtype == WKV_F32) {
+        if (V == 2) dispatch_forward<float, 2>(r != nullptr, false, a, g.units, stream);
+        else dispatch_forward<float, 1>(r != nullptr, false, a, g.units, stream);
+    } else {
+        if (V == 2) dispatch_forward<__nv_bfloat16, 2>(r != nullptr, false, a, g.units, stream);
+        else dispatch_forward<__nv_bfloat16, 1>(r != nullptr, false, a, g.units, stream);
+    }
+    return check_launch();
+}
+
+}  // extern "C"
+
