@@ -38,7 +38,20 @@ constexpr int kWsStages = 4;
 constexpr int kMinTT = (kW < kWsW ? kW : kWsW) * kLS;
 // Sequences at most this long take the sequential kernel.
 constexpr int64_t kSeqMaxT = 16;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per cross-CTA wait
+// Limit of every bounded wait on the GPU: 1 s, or WKV_WAIT_LIMIT_NS (read once
+// per process; used by the tests to make waits run out on purpose).
+uint64_t wait_limit_ns() {
+    static const uint64_t v = []() -> uint64_t {
+        const char* e = std::getenv("WKV_WAIT_LIMIT_NS");
+        if (e != nullptr && *e != '\0') {
+            char* end = nullptr;
+            const unsigned long long x = std::strtoull(e, &end, 10);
+            if (end != e) return x;
+        }
+        return 1000000000ull;
+    }();
+    return v;
+}
 
 int record_cuda(cudaError_t e) {
     if (e == cudaSuccess) return WKV_OK;
@@ -232,7 +245,7 @@ int launch_tma(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
 // Lane-resident kernel: each CTA owns whole lane blocks; grid = min(lane
 // blocks, resident capacity).
 template <typename IO, bool GATE, int STAGES>
-int launch_lane(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
+int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
     using G = wkv::LaneGeometry<IO, 2, GATE, kW, kLS, STAGES>;
     auto kern = wkv::lane_forward_kernel<IO, 2, GATE, kW, kLS, STAGES>;
     static int capacity[kMaxDevices] = {0};
@@ -258,14 +271,30 @@ int launch_lane(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
         tr = tv;
     }
     const int64_t grid = a.nLB < capacity[dev] ? a.nLB : capacity[dev];
+    // fewer CTAs than lane blocks: equal shares of the chunk order, with one
+    // state handed between neighbouring CTAs through the workspace
+    if (grid < a.nLB && a.nchunks > 1) {
+        if (workspace == nullptr) return WKV_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
+        if (workspace_bytes < 256 + size_t(a.nLB) * G::CB * sizeof(wkv::Word) ||
+            workspace_bytes < wkv_forward_workspace_bytes(a.B, a.T, a.C, dtype))
+            return WKV_ERR_WORKSPACE;
+        a.hdr = reinterpret_cast<wkv::WsHeader*>(workspace);
+        a.incw = reinterpret_cast<wkv::Word*>(static_cast<char*>(workspace) + 256);
+    } else {
+        a.hdr = nullptr;
+        a.incw = nullptr;
+    }
+    a.aggw = nullptr;
     kern<<<static_cast<unsigned>(grid), G::THREADS, G::SMEM, st>>>(tk, tv, tr, a);
     return check_launch();
 }
 
 template <typename IO>
-int dispatch_lane(bool gate, const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
+int dispatch_lane(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
     constexpr int S = sizeof(IO) == 4 ? 2 : 3;   // two CTAs per SM either way
-    return gate ? launch_lane<IO, true, S>(a, dtype, st) : launch_lane<IO, false, S>(a, dtype, st);
+    return gate ? launch_lane<IO, true, S>(a, dtype, ws, ws_bytes, st)
+                : launch_lane<IO, false, S>(a, dtype, ws, ws_bytes, st);
 }
 
 template <typename IO>
@@ -410,7 +439,7 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     a.B = B;
     a.T = T;
     a.C = C;
-    a.wait_limit_ns = kWaitLimitNs;
+    a.wait_limit_ns = wait_limit_ns();
     int64_t grid = 0;
     if (!seq) {
         const bool tma = force != 2 && tma_eligible(V, dtype, B, T, C, k, v, r, w, u, state_in);
@@ -422,8 +451,9 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
             a.nLB = g.nLB;
             a.nchunks = g.nchunks;
             a.units = g.units;
-            return dtype == WKV_F32 ? dispatch_lane<float>(r != nullptr, a, dtype, stream)
-                                    : dispatch_lane<__nv_bfloat16>(r != nullptr, a, dtype, stream);
+            return dtype == WKV_F32
+                       ? dispatch_lane<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
+                       : dispatch_lane<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
         }
         const ChunkGeom g = chunk_geom(B, T, C, V, (tma ? kWsW : kW) * kLS);
         a.nCB = g.nCB;
@@ -597,7 +627,7 @@ int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype, const float*
     a.nLB = g.nLB;
     a.nchunks = g.nchunks;
     a.units = g.units;
-    a.wait_limit_ns = kWaitLimitNs;
+    a.wait_limit_ns = wait_limit_ns();
     if (g.bytes > 0) {
         void* ws = nullptr;
         int rc = noalloc_scratch(&ws);

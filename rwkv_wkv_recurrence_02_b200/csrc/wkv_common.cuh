@@ -147,6 +147,47 @@ __device__ __forceinline__ float lane_token(float& a, float& b, float& p, float 
     return y;
 }
 
+// ---------------------------------------------------------------------------
+// packed fp32 pairs (sm_100 f32x2 arithmetic): the two channels a thread owns
+// ---------------------------------------------------------------------------
+struct F2 {
+    unsigned long long v;
+};
+
+__device__ __forceinline__ F2 f2(float a, float b) {
+    F2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ F2 f2s(float a) { return f2(a, a); }
+__device__ __forceinline__ float f2lo(F2 x) {
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(x.v));
+    return a;
+}
+__device__ __forceinline__ float f2hi(F2 x) {
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(x.v));
+    return b;
+}
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
+    F2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+    return d;
+}
+__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
+    F2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+    return d;
+}
+__device__ __forceinline__ F2 add2(F2 a, F2 b) {
+    F2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+    return d;
+}
+__device__ __forceinline__ F2 ex2x2(F2 x) { return f2(ex2(f2lo(x)), ex2(f2hi(x))); }
+__device__ __forceinline__ F2 rcpx2(F2 x) { return f2(rcp(f2lo(x)), rcp(f2hi(x))); }
+
 // 1 + e^-r, the denominator factor of sigmoid(r) = 1 / (1 + e^-r).
 __device__ __forceinline__ float gate_den(float r) { return 1.f + ex2(-r * kLog2e); }
 

@@ -1,10 +1,13 @@
 // wkv_lane.cuh -- lane-resident chunked forward kernel.
 //
-// Each CTA owns whole lane blocks (CB = 32*V channels of one sequence) and
-// walks their chunks in order, so the state carried from one chunk to the
-// next never leaves the CTA: no workspace and no waiting on other CTAs.  It
-// is the path when there are enough lane blocks to fill every CTA slot of
-// the GPU; the look-back kernels split the sequence across CTAs otherwise.
+// Each CTA owns lane blocks (CB = 32*V channels of one sequence) and walks
+// their chunks in order, so the state carried from one chunk to the next
+// stays in the CTA.  To balance the work, CTA g takes an equal share of the
+// lane-major (lane block, chunk) order: at most the head of its last lane
+// block and the tail of its first one are partial, and the head's end state
+// is handed to the next CTA as one 16-byte word per channel (see LaneRange).
+// It is the path when there are at least as many lane blocks as SMs; the
+// look-back kernels split single sequences across CTAs otherwise.
 //
 // Warps 0..W-1 compute, warp W is the producer.  Per chunk of TT = W*LS
 // tokens: the producer streams the k, v, r tiles into a ring of S shared-
@@ -33,6 +36,117 @@ struct LaneGeometry {
     static constexpr int THREADS = (W + 1) * 32;
 };
 
+// The contiguous range [s, e) of the lane-major (lane block, chunk) order a
+// CTA owns, as work items in processing order: the head of its last lane
+// block (chunks from 0, ending inside the block; its end state is handed to
+// the next CTA), then whole lane blocks, then the tail of its first lane
+// block (starting inside the block from the state the previous CTA handed
+// over).  With at least as many lane blocks as CTAs every range spans a lane
+// block boundary, so a CTA has at most one head and one tail and no hand-off
+// depends on another.
+struct LaneRange {
+    int64_t nc;            // chunks per lane block
+    int64_t f0, nfull;     // whole lane blocks [f0, f0 + nfull)
+    int64_t lb_head, head_end, lb_tail, tail_begin;
+    bool head, tail;
+    int count;
+
+    __device__ __forceinline__ void init(int64_t nLB, int64_t nchunks, int64_t g, int64_t G) {
+        nc = nchunks;
+        const int64_t U = nLB * nchunks;
+        const int64_t s = g * U / G, e = (g + 1) * U / G;
+        tail = s % nc != 0;
+        lb_tail = s / nc;
+        tail_begin = s % nc;
+        head = e % nc != 0;
+        lb_head = e / nc;
+        head_end = e % nc;
+        f0 = (s + nc - 1) / nc;
+        nfull = e / nc - f0;
+        if (nfull < 0) nfull = 0;
+        count = static_cast<int>(nfull) + (head ? 1 : 0) + (tail ? 1 : 0);
+    }
+    // item i: lane block, chunk range [c0, c1), whether its start state comes
+    // from the previous CTA and whether its end state goes to the next one
+    __device__ __forceinline__ void item(int i, int64_t& lb, int64_t& c0, int64_t& c1, bool& from_prev,
+                                         bool& to_next) const {
+        from_prev = false;
+        to_next = false;
+        if (head) {
+            if (i == 0) {
+                lb = lb_head;
+                c0 = 0;
+                c1 = head_end;
+                to_next = true;
+                return;
+            }
+            --i;
+        }
+        if (i < nfull) {
+            lb = f0 + i;
+            c0 = 0;
+            c1 = nc;
+            return;
+        }
+        lb = lb_tail;
+        c0 = tail_begin;
+        c1 = nc;
+        from_prev = true;
+    }
+};
+
+// State entering work item i (called by one warp, once per item): the
+// sequence's initial state, or the state the previous CTA handed over
+// (waited for with a time bound; NaN and a recorded error on expiry).
+template <int V>
+__device__ __noinline__ void lane_entry_state(const ChunkArgs& A, const LaneRange& R, int i, uint32_t epoch,
+                                              St* out) {
+    constexpr int CB = 32 * V;
+    const int lane = threadIdx.x & 31;
+    const int64_t lanes = A.B * A.C;
+    int64_t lb, c0, c1;
+    bool from_prev, to_next;
+    R.item(i, lb, c0, c1, from_prev, to_next);
+    const int64_t cb = (lb % A.nCB) * CB + lane * V;
+    if (!from_prev) {
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            out[j] = st_identity();
+            if (A.s_in != nullptr && cb + j < A.C) {
+                const int64_t li = (lb / A.nCB) * A.C + cb + j;
+                out[j] = St{A.s_in[2 * lanes + li] * kLog2e, A.s_in[li], A.s_in[lanes + li]};
+            }
+        }
+        return;
+    }
+    const Word* src = A.incw + lb * CB + lane * V;
+    const uint64_t t0 = global_ns();
+    unsigned sleep_ns = 32;
+    for (;;) {
+        Word wv[V];
+        bool mine = true;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            wv[j] = ld_word(src + j);
+            mine = mine && wv[j].tag == word_tag(epoch, kKindInc);
+        }
+        if (__all_sync(0xffffffffu, mine)) {
+#pragma unroll
+            for (int j = 0; j < V; ++j) out[j] = word_state(wv[j]);
+            return;
+        }
+        if (global_ns() - t0 > A.wait_limit_ns) {
+            if (lane == 0) record_timeout(A, lb);
+            const float nan = __int_as_float(0x7fc00000);
+#pragma unroll
+            for (int j = 0; j < V; ++j) out[j] = St{nan, nan, nan};
+            return;
+        }
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 256) sleep_ns <<= 1;
+    }
+}
+
 __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -48,8 +162,10 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     __shared__ __align__(8) uint64_t full[S], empty[S];
     __shared__ St s_seg[2][W][V][32];   // segment summaries, double-buffered by chunk parity
     __shared__ St s_carry[2][V][32];    // state at the start of a chunk, double-buffered
+    __shared__ LaneRange s_range;       // this CTA's share of the chunk order
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
+        s_range.init(A.nLB, A.nchunks, blockIdx.x, gridDim.x);
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], W);
@@ -61,11 +177,15 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     if (warp == W) {
         // ---------------- producer ----------------
         if (lane == 0) {
+            const LaneRange& R = s_range;
             int64_t it = 0;
-            for (int64_t lb = blockIdx.x; lb < A.nLB; lb += gridDim.x) {
+            for (int item = 0; item < R.count; ++item) {
+                int64_t lb, c0, c1;
+                bool from_prev, to_next;
+                R.item(item, lb, c0, c1, from_prev, to_next);
                 const int x = static_cast<int>((lb % A.nCB) * CB);
                 const int z = static_cast<int>(lb / A.nCB);
-                for (int64_t chunk = 0; chunk < A.nchunks; ++chunk, ++it) {
+                for (int64_t chunk = c0; chunk < c1; ++chunk, ++it) {
                     const int s = static_cast<int>(it % S);
                     if (it >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((it / S) - 1) & 1), A.wait_limit_ns))
                         return;  // the compute warps stopped; they time out on full[] as well
@@ -84,23 +204,24 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 
     // ---------------- compute ----------------
     // Shared buffers alternate with the parity of the running chunk count it
-    // (continuous across lane blocks).  The state entering a lane block is
+    // (continuous across work items).  The state entering a work item is
     // written by warp W-1 where it would otherwise write the carried state,
     // so every slot is written and read in the same barrier order.
     const int64_t lanes = A.B * A.C;
-    auto initial_state = [&](int64_t lbx, int j) -> St {
-        if (lbx >= A.nLB) return st_identity();
-        const int64_t cc = (lbx % A.nCB) * CB + lane * V + j;
-        if (A.s_in == nullptr || cc >= A.C) return st_identity();
-        const int64_t li = (lbx / A.nCB) * A.C + cc;
-        return St{A.s_in[2 * lanes + li] * kLog2e, A.s_in[li], A.s_in[lanes + li]};
-    };
-    if (warp == W - 1 && static_cast<int64_t>(blockIdx.x) < A.nLB) {
+    const uint32_t epoch = A.hdr != nullptr ? ld_relaxed_u32(&A.hdr->epoch) : 0u;
+    const LaneRange& R = s_range;
+    bool ok = true;
+    if (warp == W - 1 && R.count > 0) {
+        St x0[V];
+        lane_entry_state<V>(A, R, 0, epoch, x0);
 #pragma unroll
-        for (int j = 0; j < V; ++j) s_carry[0][j][lane] = initial_state(blockIdx.x, j);
+        for (int j = 0; j < V; ++j) s_carry[0][j][lane] = x0[j];
     }
     int64_t it = 0;
-    for (int64_t lb = blockIdx.x; lb < A.nLB; lb += gridDim.x) {
+    for (int item = 0; item < R.count && ok; ++item) {
+        int64_t lb, c0, c1;
+        bool from_prev, to_next;
+        R.item(item, lb, c0, c1, from_prev, to_next);
         const int64_t b = lb / A.nCB;
         const int64_t c = (lb % A.nCB) * CB + lane * V;
         SegCtx<V, LS> cx;
@@ -114,12 +235,13 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
             }
             set_params<V, LS>(cx, wv, uv);
         }
-        for (int64_t chunk = 0; chunk < A.nchunks; ++chunk, ++it) {
+        for (int64_t chunk = c0; chunk < c1; ++chunk, ++it) {
             const int s = static_cast<int>(it % S);
             const int par = static_cast<int>(it & 1);
             if (!mbar_wait(&full[s], static_cast<uint32_t>((it / S) & 1), A.wait_limit_ns)) {
                 if (threadIdx.x == 0 && A.hdr != nullptr) record_timeout(A, -1);
-                return;
+                ok = false;
+                break;
             }
             const unsigned char* stage = smem + s * G::STAGE;
             const int64_t unit = chunk * A.nLB + lb;
@@ -143,17 +265,25 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
             }
             if (warp == W - 1) {
                 // state after the chunk: this warp's start, then its own segment
-                const bool last = chunk == A.nchunks - 1;
-                for (int j = 0; j < V; ++j) {
-                    const St nx = st_combine(st[j], seg[j], static_cast<float>(cx.nvalid) * cx.w2[j]);
-                    s_carry[par ^ 1][j][lane] = last ? initial_state(lb + gridDim.x, j) : nx;
-                    if (last && A.s_out != nullptr && cx.cvalid) {
-                        const int64_t li = b * A.C + c + j;
-                        A.s_out[li] = nx.a;
-                        A.s_out[lanes + li] = nx.b;
-                        A.s_out[2 * lanes + li] = nx.p * kLn2;
+                St nx[V];
+#pragma unroll
+                for (int j = 0; j < V; ++j) nx[j] = st_combine(st[j], seg[j], static_cast<float>(cx.nvalid) * cx.w2[j]);
+                if (chunk == c1 - 1) {
+                    if (to_next) {
+                        publish<V>(A.incw + lb * CB, nx, epoch, kKindInc, lane);
+                    } else if (A.s_out != nullptr && cx.cvalid) {
+#pragma unroll
+                        for (int j = 0; j < V; ++j) {
+                            const int64_t li = b * A.C + c + j;
+                            A.s_out[li] = nx[j].a;
+                            A.s_out[lanes + li] = nx[j].b;
+                            A.s_out[2 * lanes + li] = nx[j].p * kLn2;
+                        }
                     }
+                    if (item + 1 < R.count) lane_entry_state<V>(A, R, item + 1, epoch, nx);
                 }
+#pragma unroll
+                for (int j = 0; j < V; ++j) s_carry[par ^ 1][j][lane] = nx[j];
             }
             if (cx.nvalid > 0 && cx.cvalid) {
                 if (full_chunk) seg_pass2<IO, V, GATE, W, LS, true>(A, stage, cx, st);
@@ -163,6 +293,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
             if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
+    if (threadIdx.x == 0 && A.hdr != nullptr) finish_launch(A, gridDim.x);
 }
 
 }  // namespace wkv

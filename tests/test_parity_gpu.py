@@ -82,6 +82,11 @@ LANE = [
     (3, 1000, 3200, torch.bfloat16, False, True),
     (160, 64, 64, torch.float32, False, True),     # exactly one chunk per lane block
     (300, 40, 64, torch.bfloat16, True, True),     # more lane blocks than CTA slots, short T
+    # more lane blocks than CTA slots with several chunks each: CTAs take
+    # equal shares of the chunk order and hand one state to their neighbour
+    (5, 200, 3840, torch.float32, True, True),
+    (7, 130, 2724, torch.bfloat16, True, True),   # ragged channel block and last chunk
+    (6, 555, 3200, torch.bfloat16, False, False),
 ]
 
 
