@@ -36,6 +36,12 @@ constexpr int kLS = 8;
 constexpr int kWsW = 4;
 constexpr int kWsStages = 4;
 constexpr int kMinTT = (kW < kWsW ? kW : kWsW) * kLS;
+// Lane-resident kernel: compute warps and tokens per warp segment (64-token
+// chunks).
+constexpr int kLaneW = 4;
+constexpr int kLaneLS = 16;
+// Fewest 64-channel lane blocks for which the lane-resident kernel is used.
+constexpr int64_t kLaneMinBlocks = 32;
 // Sequences at most this long take the sequential kernel.
 constexpr int64_t kSeqMaxT = 16;
 // Limit of every bounded wait on the GPU: 1 s, or WKV_WAIT_LIMIT_NS (read once
@@ -246,8 +252,8 @@ int launch_tma(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
 // blocks, resident capacity).
 template <typename IO, bool GATE, int STAGES>
 int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
-    using G = wkv::LaneGeometry<IO, 2, GATE, kW, kLS, STAGES>;
-    auto kern = wkv::lane_forward_kernel<IO, 2, GATE, kW, kLS, STAGES>;
+    using G = wkv::LaneGeometry<IO, 2, GATE, kLaneW, kLaneLS, STAGES>;
+    auto kern = wkv::lane_forward_kernel<IO, 2, GATE, kLaneW, kLaneLS, STAGES>;
     static int capacity[kMaxDevices] = {0};
     int dev = 0;
     int rc = record_cuda(cudaGetDevice(&dev));
@@ -292,7 +298,8 @@ int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
 
 template <typename IO>
 int dispatch_lane(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
-    constexpr int S = sizeof(IO) == 4 ? 2 : 3;   // two CTAs per SM either way
+    // ring depth: two CTAs per SM for either dtype
+    constexpr int S = sizeof(IO) == 4 ? 2 : 3;
     return gate ? launch_lane<IO, true, S>(a, dtype, ws, ws_bytes, st)
                 : launch_lane<IO, false, S>(a, dtype, ws, ws_bytes, st);
 }
@@ -443,10 +450,11 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     int64_t grid = 0;
     if (!seq) {
         const bool tma = force != 2 && tma_eligible(V, dtype, B, T, C, k, v, r, w, u, state_in);
-        // enough lane blocks to give every SM its own: no cross-CTA split
-        const bool lane_resident = tma && force != 4 && B * ((C + 63) / 64) >= sm_count();
+        // enough lane blocks to keep a good share of the SMs busy walking whole
+        // sequences; below that the look-back kernel splits sequences along T
+        const bool lane_resident = tma && force != 4 && B * ((C + 63) / 64) >= kLaneMinBlocks;
         if (lane_resident) {
-            const ChunkGeom g = chunk_geom(B, T, C, 2, kW * kLS);
+            const ChunkGeom g = chunk_geom(B, T, C, 2, kLaneW * kLaneLS);
             a.nCB = g.nCB;
             a.nLB = g.nLB;
             a.nchunks = g.nchunks;

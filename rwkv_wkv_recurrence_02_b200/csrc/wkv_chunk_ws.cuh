@@ -115,19 +115,16 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
 // scales every token by the largest key: one ex2 per token, whose argument
 // fuses the base-2 conversion.
 template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool PARAMS_IN_STAGE = true>
-__device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t unit, const unsigned char* stage,
-                                           SegCtx<V, LS>& cx, St* seg) {
+__device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, int64_t b, int64_t c,
+                                           const unsigned char* stage, SegCtx<V, LS>& cx, St* seg) {
     constexpr int CB = 32 * V;
     constexpr int TT = W * LS;
     constexpr int ROW = CB * static_cast<int>(sizeof(IO));
     constexpr int TILE = TT * ROW;
     using Raw = typename Vec<IO, V>::raw;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t chunk = unit / A.nLB, lb = unit % A.nLB;
-    const int64_t b = lb / A.nCB;
-    const int64_t c = (lb % A.nCB) * CB + lane * V;
     cx.cvalid = c < A.C;
-    const int64_t t_seg = chunk * TT + static_cast<int64_t>(warp) * LS;
+    const int64_t t_seg = chunk * TT + warp * LS;
     cx.nvalid = FULL ? LS : static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), A.T - t_seg)));
     cx.base = (b * A.T + t_seg) * A.C + c;
     if (PARAMS_IN_STAGE) set_params<V>(cx, reinterpret_cast<const float*>(stage + NARR_OF<GATE>() * TILE) + lane * V,
@@ -298,13 +295,18 @@ __device__ __forceinline__ void seg_pass2(const ChunkArgs& A, const unsigned cha
     }
 }
 
+// (chunk, lane block, sequence, first channel) of a unit.
+struct UnitCoord {
+    int64_t chunk, lb, b, c0;
+};
+
 // Compute warps, first half of a unit: wait for its tiles, pass 0/1, hand
 // the segment summary to the scan warp.  False at the end of the stream (or
 // on a timeout).
 template <typename IO, int V, bool GATE, int W, int LS, int S>
 __device__ __forceinline__ bool compute_front(const ChunkArgs& A, int64_t it, unsigned char* smem, uint64_t* full,
-                                              uint64_t* aggready, const int64_t* unitbuf, St* aggbuf,
-                                              SegCtx<V, LS>& cx) {
+                                              uint64_t* aggready, const int64_t* unitbuf, const UnitCoord* coord,
+                                              St* aggbuf, SegCtx<V, LS>& cx) {
     using G = WsGeometry<IO, V, GATE, W, LS, S>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int s = static_cast<int>(it % S);
@@ -317,8 +319,9 @@ __device__ __forceinline__ bool compute_front(const ChunkArgs& A, int64_t it, un
     if (u >= A.units) return false;
     const unsigned char* stage = smem + s * G::STAGE;
     St seg[V];
-    if ((u / A.nLB + 1) * G::TT <= A.T) seg_pass01<IO, V, GATE, W, LS, true>(A, u, stage, cx, seg);
-    else seg_pass01<IO, V, GATE, W, LS, false>(A, u, stage, cx, seg);
+    const int64_t chunk = coord[s].chunk, b = coord[s].b, c = coord[s].c0 + lane * V;
+    if ((chunk + 1) * G::TT <= A.T) seg_pass01<IO, V, GATE, W, LS, true>(A, chunk, b, c, stage, cx, seg);
+    else seg_pass01<IO, V, GATE, W, LS, false>(A, chunk, b, c, stage, cx, seg);
     St* ab = aggbuf + static_cast<int64_t>(s) * W * V * 32;
 #pragma unroll
     for (int j = 0; j < V; ++j) ab[(warp * V + j) * 32 + lane] = seg[j];
@@ -331,8 +334,8 @@ __device__ __forceinline__ bool compute_front(const ChunkArgs& A, int64_t it, un
 // release the stage.  False on a timeout.
 template <typename IO, int V, bool GATE, int W, int LS, int S>
 __device__ __forceinline__ bool compute_back(const ChunkArgs& A, int64_t it, unsigned char* smem, uint64_t* xready,
-                                             uint64_t* empty, const int64_t* unitbuf, const St* aggbuf,
-                                             const St* xbuf, SegCtx<V, LS>& cx) {
+                                             uint64_t* empty, const int64_t* unitbuf, const UnitCoord* coord,
+                                             const St* aggbuf, const St* xbuf, SegCtx<V, LS>& cx) {
     using G = WsGeometry<IO, V, GATE, W, LS, S>;
     constexpr int TT = G::TT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -340,8 +343,7 @@ __device__ __forceinline__ bool compute_back(const ChunkArgs& A, int64_t it, uns
     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
     const bool ok = mbar_wait(&xready[s], ph, A.wait_limit_ns);
     if (!ok && threadIdx.x == 0 && A.hdr != nullptr) record_timeout(A, -1);
-    const int64_t u = unitbuf[s];
-    const int64_t chunk = u / A.nLB;
+    const int64_t chunk = coord[s].chunk;
     if (ok && cx.nvalid > 0 && cx.cvalid) {
         const int64_t chunk_rows = min(static_cast<int64_t>(TT), A.T - chunk * TT);
         const St* ab = aggbuf + static_cast<int64_t>(s) * W * V * 32;
@@ -401,6 +403,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[S], empty[S], aggready[S], xready[S], foldready[S];
     __shared__ int64_t unitbuf[S];
+    __shared__ UnitCoord coord[S];   // decoded by the producer: no divisions in the other warps
     __shared__ int64_t s_endpos;   // first ring position with no unit (set by the producer)
     __shared__ uint32_t s_epoch;
     St* aggbuf = reinterpret_cast<St*>(smem + S * G::STAGE);                 // [S][W][V][32]
@@ -449,6 +452,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                 const int64_t chunk = u / A.nLB, lb = u % A.nLB;
                 const int64_t c0 = (lb % A.nCB) * CB;
                 const int64_t b = lb / A.nCB;
+                coord[s] = UnitCoord{chunk, lb, b, c0};
                 // channels of this block inside C; a multiple of 4 because C is
                 const uint32_t pbytes = static_cast<uint32_t>(min(static_cast<int64_t>(CB), A.C - c0)) * 4u;
                 const bool first = chunk == 0 && A.s_in != nullptr;
@@ -484,8 +488,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
             }
             const int64_t u = unitbuf[s];
             if (u >= A.units) break;
-            const int64_t chunk = u / A.nLB, lb = u % A.nLB;
-            const int64_t c = (lb % A.nCB) * CB + lane * V;
+            const int64_t chunk = coord[s].chunk;
+            const int64_t c = coord[s].c0 + lane * V;
             const bool cvalid = c < A.C;
             const int64_t chunk_rows = min(static_cast<int64_t>(TT), A.T - chunk * TT);
             const float* prm = reinterpret_cast<const float*>(smem + s * G::STAGE + G::TILES);
@@ -525,9 +529,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
             if (got <= 0) break;
             const int64_t u = unitbuf[s];
             if (u >= A.units) break;
-            const int64_t chunk = u / A.nLB, lb = u % A.nLB;
-            const int64_t b = lb / A.nCB;
-            const int64_t c = (lb % A.nCB) * CB + lane * V;
+            const int64_t chunk = coord[s].chunk, lb = coord[s].lb;
+            const int64_t b = coord[s].b;
+            const int64_t c = coord[s].c0 + lane * V;
             const bool cvalid = c < A.C;
             const int64_t chunk_rows = min(static_cast<int64_t>(TT), A.T - chunk * TT);
             const bool last = chunk == A.nchunks - 1;
@@ -593,12 +597,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         // are out before this CTA waits for the start state of the previous
         // unit.  Two register contexts, unrolled by two.
         SegCtx<V, LS> cxa, cxb;
-        bool end_a = !compute_front<IO, V, GATE, W, LS, S>(A, 0, smem, full, aggready, unitbuf, aggbuf, cxa);
+        bool end_a = !compute_front<IO, V, GATE, W, LS, S>(A, 0, smem, full, aggready, unitbuf, coord, aggbuf, cxa);
         for (int64_t it = 0; !end_a; it += 2) {
-            const bool end_b = !compute_front<IO, V, GATE, W, LS, S>(A, it + 1, smem, full, aggready, unitbuf, aggbuf, cxb);
-            if (!compute_back<IO, V, GATE, W, LS, S>(A, it, smem, xready, empty, unitbuf, aggbuf, xbuf, cxa) || end_b) break;
-            end_a = !compute_front<IO, V, GATE, W, LS, S>(A, it + 2, smem, full, aggready, unitbuf, aggbuf, cxa);
-            if (!compute_back<IO, V, GATE, W, LS, S>(A, it + 1, smem, xready, empty, unitbuf, aggbuf, xbuf, cxb)) break;
+            const bool end_b = !compute_front<IO, V, GATE, W, LS, S>(A, it + 1, smem, full, aggready, unitbuf, coord, aggbuf, cxb);
+            if (!compute_back<IO, V, GATE, W, LS, S>(A, it, smem, xready, empty, unitbuf, coord, aggbuf, xbuf, cxa) || end_b) break;
+            end_a = !compute_front<IO, V, GATE, W, LS, S>(A, it + 2, smem, full, aggready, unitbuf, coord, aggbuf, cxa);
+            if (!compute_back<IO, V, GATE, W, LS, S>(A, it + 1, smem, xready, empty, unitbuf, coord, aggbuf, xbuf, cxb)) break;
         }
     }
     __syncthreads();

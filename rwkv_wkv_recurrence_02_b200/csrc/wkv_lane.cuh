@@ -151,8 +151,8 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-template <typename IO, int V, bool GATE, int W, int LS, int S>
-__global__ void __launch_bounds__(LaneGeometry<IO, V, GATE, W, LS, S>::THREADS, 2)
+template <typename IO, int V, bool GATE, int W, int LS, int S, int MINB = 2>
+__global__ void __launch_bounds__(LaneGeometry<IO, V, GATE, W, LS, S>::THREADS, MINB)
 lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const __grid_constant__ CUtensorMap tr, const ChunkArgs A) {
     using G = LaneGeometry<IO, V, GATE, W, LS, S>;
@@ -178,7 +178,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
         // ---------------- producer ----------------
         if (lane == 0) {
             const LaneRange& R = s_range;
-            int64_t it = 0;
+            uint32_t it = 0;
             for (int item = 0; item < R.count; ++item) {
                 int64_t lb, c0, c1;
                 bool from_prev, to_next;
@@ -187,7 +187,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
                 const int z = static_cast<int>(lb / A.nCB);
                 for (int64_t chunk = c0; chunk < c1; ++chunk, ++it) {
                     const int s = static_cast<int>(it % S);
-                    if (it >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((it / S) - 1) & 1), A.wait_limit_ns))
+                    if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1u, A.wait_limit_ns))
                         return;  // the compute warps stopped; they time out on full[] as well
                     unsigned char* st = smem + s * G::STAGE;
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -217,7 +217,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 #pragma unroll
         for (int j = 0; j < V; ++j) s_carry[0][j][lane] = x0[j];
     }
-    int64_t it = 0;
+    uint32_t it = 0;
     for (int item = 0; item < R.count && ok; ++item) {
         int64_t lb, c0, c1;
         bool from_prev, to_next;
@@ -237,31 +237,39 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
         }
         for (int64_t chunk = c0; chunk < c1; ++chunk, ++it) {
             const int s = static_cast<int>(it % S);
-            const int par = static_cast<int>(it & 1);
-            if (!mbar_wait(&full[s], static_cast<uint32_t>((it / S) & 1), A.wait_limit_ns)) {
+            const int par = static_cast<int>(it & 1u);
+            if (!mbar_wait(&full[s], (it / S) & 1u, A.wait_limit_ns)) {
                 if (threadIdx.x == 0 && A.hdr != nullptr) record_timeout(A, -1);
                 ok = false;
                 break;
             }
             const unsigned char* stage = smem + s * G::STAGE;
-            const int64_t unit = chunk * A.nLB + lb;
             const bool full_chunk = (chunk + 1) * TT <= A.T;
             St seg[V];
-            if (full_chunk) seg_pass01<IO, V, GATE, W, LS, true, false>(A, unit, stage, cx, seg);
-            else seg_pass01<IO, V, GATE, W, LS, false, false>(A, unit, stage, cx, seg);
+            if (full_chunk) seg_pass01<IO, V, GATE, W, LS, true, false>(A, chunk, b, c, stage, cx, seg);
+            else seg_pass01<IO, V, GATE, W, LS, false, false>(A, chunk, b, c, stage, cx, seg);
 #pragma unroll
             for (int j = 0; j < V; ++j) s_seg[par][warp][j][lane] = seg[j];
             named_sync(1, W * 32);
             // start state of this warp's segment: carried state, then the
             // segments before this one
-            const int64_t chunk_rows = min(static_cast<int64_t>(TT), A.T - chunk * TT);
+            // rows of this chunk (all TT but in a sequence's last, partial chunk)
+            const int chunk_rows = full_chunk ? TT : static_cast<int>(A.T - chunk * TT);
             St st[V];
 #pragma unroll
             for (int j = 0; j < V; ++j) st[j] = s_carry[par][j][lane];
-            for (int sg = 0; sg < warp; ++sg) {
-                const int len = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), chunk_rows - sg * LS)));
+            float seglen[V];
 #pragma unroll
-                for (int j = 0; j < V; ++j) st[j] = st_combine(st[j], s_seg[par][sg][j][lane], static_cast<float>(len) * cx.w2[j]);
+            for (int j = 0; j < V; ++j) seglen[j] = static_cast<float>(LS) * cx.w2[j];
+            for (int sg = 0; sg < warp; ++sg) {
+                // segments before this one are full unless the chunk is short
+                if (!full_chunk) {
+                    const int len = max(0, min(LS, chunk_rows - sg * LS));
+#pragma unroll
+                    for (int j = 0; j < V; ++j) seglen[j] = static_cast<float>(len) * cx.w2[j];
+                }
+#pragma unroll
+                for (int j = 0; j < V; ++j) st[j] = st_combine(st[j], s_seg[par][sg][j][lane], seglen[j]);
             }
             if (warp == W - 1) {
                 // state after the chunk: this warp's start, then its own segment
