@@ -16,6 +16,7 @@
 #include "wkv_chunk.cuh"
 #include "wkv_chunk_ws.cuh"
 #include "wkv_lane.cuh"
+#include "wkv_part.cuh"
 #include "wkv_seq.cuh"
 #include "wkv_step.cuh"
 
@@ -40,12 +41,21 @@ constexpr int kMinTT = (kW < kWsW ? kW : kWsW) * kLS;
 // chunks).
 constexpr int kLaneW = 4;
 constexpr int kLaneLS = 16;
-// Fewest 64-channel lane blocks for which the lane-resident kernel is used.
-constexpr int64_t kLaneMinBlocks = 32;
+// Part kernel: compute warps and tokens per warp segment (128-token parts).
+// It runs when there are fewer 64-channel lane blocks than SMs; the
+// lane-resident kernel from there on.
+constexpr int kPartW = 8;
+constexpr int kPartLS = 16;
+constexpr int kPartMinBlocks = 2;
+// look-back window (parts per round trip) and whether pass 1 keeps its
+// exponentials in registers for pass 2
+constexpr int kPartWin = 1;
+constexpr bool kPartCache = true;
 // Sequences at most this long take the sequential kernel.
 constexpr int64_t kSeqMaxT = 16;
-// Limit of every bounded wait on the GPU: 1 s, or WKV_WAIT_LIMIT_NS (read once
-// per process; used by the tests to make waits run out on purpose).
+// Limit of every wait on another CTA's result: 1 s, or WKV_WAIT_LIMIT_NS (read
+// once per process; used by the tests to make waits run out on purpose).
+// Waits for a CTA's own TMA copies have a fixed limit (kCopyWaitNs).
 uint64_t wait_limit_ns() {
     static const uint64_t v = []() -> uint64_t {
         const char* e = std::getenv("WKV_WAIT_LIMIT_NS");
@@ -201,9 +211,10 @@ bool tma_eligible(int V, int dtype, int64_t B, int64_t T, int64_t C, const void*
 }
 
 // Kernel choice: 0 = automatic; the environment variable WKV_FORWARD_KERNEL
-// (seq | chunk | tma | lookback) forces one, for ablation measurements:
-// chunk = register-load look-back kernel, lookback = TMA look-back kernel
-// even where the lane-resident one would run.
+// (seq | chunk | tma | lookback | part | lane) forces one, for ablation
+// measurements: chunk = register-load look-back kernel, lookback = TMA
+// look-back kernel, part = part kernel, lane = lane-resident kernel, each
+// even where another would run.
 int forced_kernel() {
     static int f = []() {
         const char* e = std::getenv("WKV_FORWARD_KERNEL");
@@ -212,9 +223,31 @@ int forced_kernel() {
         if (std::strcmp(e, "chunk") == 0) return 2;
         if (std::strcmp(e, "tma") == 0) return 3;
         if (std::strcmp(e, "lookback") == 0) return 4;
+        if (std::strcmp(e, "part") == 0) return 5;
+        if (std::strcmp(e, "lane") == 0) return 6;
         return 0;
     }();
     return f;
+}
+
+// Launch of a TMA kernel with programmatic stream serialization: its CTAs
+// may be scheduled while the previous kernel of the stream drains; the
+// kernel waits for that kernel (griddepcontrol.wait) before its first
+// global memory access.
+template <typename... P>
+int launch_pdl(void (*kern)(P...), int64_t grid, int threads, uint32_t smem, cudaStream_t st,
+               const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tr, const wkv::ChunkArgs& a) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tk, tv, tr, a));
 }
 
 template <typename IO, bool GATE, int STAGES>
@@ -292,8 +325,73 @@ int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
         a.incw = nullptr;
     }
     a.aggw = nullptr;
-    kern<<<static_cast<unsigned>(grid), G::THREADS, G::SMEM, st>>>(tk, tv, tr, a);
-    return check_launch();
+    return launch_pdl(kern, grid, G::THREADS, G::SMEM, st, tk, tv, tr, a);
+}
+
+// Part kernel: lane blocks cut into parts along T, claimed in order from the
+// workspace's ticket counter; grid = min(parts, resident capacity).
+template <typename IO, bool GATE, int NB>
+int launch_part(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+    using G = wkv::PartGeometry<IO, 2, GATE, kPartW, kPartLS, NB>;
+    auto kern = wkv::part_forward_kernel<IO, 2, GATE, kPartW, kPartLS, NB, kPartMinBlocks, kPartWin, kPartCache>;
+    static int capacity[kMaxDevices] = {0};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (capacity[dev] == 0) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        int per_sm = 0;
+        rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+    }
+    const ChunkGeom g = chunk_geom(a.B, a.T, a.C, 2, G::PT);
+    a.nCB = g.nCB;
+    a.nLB = g.nLB;
+    a.nchunks = g.nchunks;
+    a.units = g.units;
+    if (g.nchunks > 1) {
+        if (workspace == nullptr) return WKV_ERR_WORKSPACE;
+        if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
+        if (workspace_bytes < g.bytes || workspace_bytes < wkv_forward_workspace_bytes(a.B, a.T, a.C, dtype))
+            return WKV_ERR_WORKSPACE;
+        char* ws = static_cast<char*>(workspace);
+        a.hdr = reinterpret_cast<wkv::WsHeader*>(ws);
+        a.aggw = reinterpret_cast<wkv::Word*>(ws + g.aggw_off);
+        a.incw = reinterpret_cast<wkv::Word*>(ws + g.incw_off);
+    } else {
+        a.hdr = nullptr;
+        a.aggw = nullptr;
+        a.incw = nullptr;
+    }
+    CUtensorMap tk, tv, tr;
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::PT) ||
+        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::PT))
+        return WKV_ERR_CUDA;
+    if (GATE) {
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
+    } else {
+        tr = tv;
+    }
+    const int64_t grid = a.units < capacity[dev] ? a.units : capacity[dev];
+    return launch_pdl(kern, grid, G::THREADS, G::SMEM, st, tk, tv, tr, a);
+}
+
+// Part buffers per CTA: as many as fit beside kPartMinBlocks CTAs per SM
+// (up to three), at least one.
+template <typename IO, bool GATE>
+constexpr int part_buffers() {
+    constexpr int budget = 225 * 1024 / kPartMinBlocks - 8 * 1024;   // static shared memory and slack
+    constexpr int part = wkv::PartGeometry<IO, 2, GATE, kPartW, kPartLS, 1>::PART;
+    return budget / part < 1 ? 1 : (budget / part > 3 ? 3 : budget / part);
+}
+
+template <typename IO>
+int dispatch_part(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
+    return gate ? launch_part<IO, true, part_buffers<IO, true>()>(a, dtype, ws, ws_bytes, st)
+                : launch_part<IO, false, part_buffers<IO, false>()>(a, dtype, ws, ws_bytes, st);
 }
 
 template <typename IO>
@@ -450,9 +548,19 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     int64_t grid = 0;
     if (!seq) {
         const bool tma = force != 2 && tma_eligible(V, dtype, B, T, C, k, v, r, w, u, state_in);
-        // enough lane blocks to keep a good share of the SMs busy walking whole
-        // sequences; below that the look-back kernel splits sequences along T
-        const bool lane_resident = tma && force != 4 && B * ((C + 63) / 64) >= kLaneMinBlocks;
+        // at least one lane block per SM: CTAs walk whole sequences; fewer:
+        // the part kernel cuts them along T.  The ticket counter is 32 bits.
+        const int64_t nLB = B * ((C + 63) / 64);
+        const int64_t nparts = nLB * ((T + kPartW * kPartLS - 1) / (kPartW * kPartLS));
+        const bool part_ok = tma && nparts < (int64_t(1) << 31);
+        const bool part = part_ok && (force == 5 || (force == 0 && nLB < sm_count()));
+        if (part) {
+            a.nLB = nLB;
+            return dtype == WKV_F32
+                       ? dispatch_part<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
+                       : dispatch_part<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
+        }
+        const bool lane_resident = tma && force != 4;
         if (lane_resident) {
             const ChunkGeom g = chunk_geom(B, T, C, 2, kLaneW * kLaneLS);
             a.nCB = g.nCB;

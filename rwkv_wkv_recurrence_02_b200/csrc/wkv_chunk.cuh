@@ -45,6 +45,10 @@ namespace wkv {
 constexpr uint32_t kKindAgg = 1;  // chunk summary (from the empty state)
 constexpr uint32_t kKindInc = 2;  // inclusive state (state after the chunk)
 constexpr uint32_t kErrTimeout = 1;
+// Limit of a wait for this CTA's own TMA copies to land.  Unlike the waits on
+// other CTAs it does not follow the configurable limit: a CTA must not exit
+// while a copy into its shared memory is still in flight.
+constexpr uint64_t kCopyWaitNs = 2000000000ull;
 
 // First 256 bytes of a workspace.
 struct WsHeader {
@@ -138,20 +142,20 @@ struct LookState {
 constexpr int kWin = 4;
 
 // One round of the look-back: every lane reads the summary and inclusive
-// words of its own channels for chunks cur, cur-1, ..., cur-kWin+1 (one
+// words of its own channels for chunks cur, cur-1, ..., cur-WIN+1 (one
 // round trip), then the warp walks them nearest first.  A chunk counts as
 // published only if every lane saw its word with this launch's epoch, so all
 // lanes take the same path with data they observed themselves.  The walk
 // stops at the first inclusive state (or at the start of the sequence, where
 // `sin` takes its place) and otherwise folds summaries into acc.  Returns
 // true if it made progress.
-template <int V, int TT>
+template <int V, int TT, int WIN = kWin>
 __device__ __forceinline__ bool lookback_round(const ChunkArgs& A, int64_t lb, uint32_t epoch, const float* w2,
                                                const St* sin, LookState<V>& L, int lane) {
     constexpr int CB = 32 * V;
-    Word wi[kWin][V], wa[kWin][V];
+    Word wi[WIN][V], wa[WIN][V];
 #pragma unroll
-    for (int l = 0; l < kWin; ++l) {
+    for (int l = 0; l < WIN; ++l) {
         const int64_t c = L.cur - l;
 #pragma unroll
         for (int j = 0; j < V; ++j) {
@@ -167,7 +171,7 @@ __device__ __forceinline__ bool lookback_round(const ChunkArgs& A, int64_t lb, u
     }
     bool progressed = false;
 #pragma unroll
-    for (int l = 0; l < kWin; ++l) {
+    for (int l = 0; l < WIN; ++l) {
         if (L.cur < 0) {
 #pragma unroll
             for (int j = 0; j < V; ++j) L.x[j] = st_combine(sin[j], L.acc[j], static_cast<float>(L.span) * w2[j]);
@@ -200,13 +204,13 @@ __device__ __forceinline__ bool lookback_round(const ChunkArgs& A, int64_t lb, u
 
 // Blocking look-back: rounds with backoff until the start state is known or
 // `limit_ns` passes (then x is NaN and the function returns false).
-template <int V, int TT>
+template <int V, int TT, int WIN = kWin>
 __device__ __forceinline__ bool lookback_finish(const ChunkArgs& A, int64_t lb, uint32_t epoch, const float* w2,
                                                 const St* sin, LookState<V>& L, int lane) {
     const uint64_t t0 = global_ns();
     unsigned sleep_ns = 32;
     while (!L.done) {
-        if (!lookback_round<V, TT>(A, lb, epoch, w2, sin, L, lane)) {
+        if (!lookback_round<V, TT, WIN>(A, lb, epoch, w2, sin, L, lane)) {
             if (global_ns() - t0 > A.wait_limit_ns) {
                 const float nan = __int_as_float(0x7fc00000);
 #pragma unroll
@@ -616,6 +620,21 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     return mbar_wait_slow(bar, parity, limit_ns);
+}
+
+// Programmatic dependent launch: let the next kernel of the stream be
+// scheduled as this one's CTAs retire, then wait until the previous kernel
+// of the stream has finished and its writes are visible.  Nothing before
+// this may read or write global memory (kernel parameters, tensor maps
+// included, are not global memory).  Without the launch attribute both are
+// no-ops.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,

@@ -107,14 +107,16 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
 
 // Pass 0 + pass 1 of one warp's segment; returns the segment summary.
 // PARAMS_IN_STAGE: read w, u from the stage's parameter area (else the
-// caller has set them in cx already).
+// caller has set them in cx already).  CACHE: keep the per-token
+// exponentials of the fast path in cx.kf for pass 2 (else pass 2 recomputes
+// them from the keys in the stage, and kf is dead after pass 1).
 //
 // Pass 0 works on raw keys: the key range (max, min) and the segment's
 // running-max exponent q = max_i (k2_i + i w2) - (n-1) w2, which equals the
 // recurrence p <- max(p - w2, k2) over the segment.  Pass 1 (fast path)
 // scales every token by the largest key: one ex2 per token, whose argument
 // fuses the base-2 conversion.
-template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool PARAMS_IN_STAGE = true>
+template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool PARAMS_IN_STAGE = true, bool CACHE = true>
 __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, int64_t b, int64_t c,
                                            const unsigned char* stage, SegCtx<V, LS>& cx, St* seg) {
     constexpr int CB = 32 * V;
@@ -177,7 +179,7 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, in
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < cx.nvalid) {
                 const F2 ek = ex2x2(fma2(cx.kf[i], L2, KM));
-                cx.kf[i] = ek;
+                if (CACHE) cx.kf[i] = ek;
                 const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + TILE + i * ROW)));
                 n = fma2(n, DK, ekv);
                 db = fma2(db, DK, ek);
@@ -217,9 +219,10 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, in
 }
 // Pass 2 of one warp's segment: outputs from the segment's start state st.
 // Fast path: every term rescaled to R = max(kmax, p) and the cached
-// exponentials reused; one ex2 (gate) and one rcp per output.  Otherwise
-// the exact running-max recurrence from keys read again from the stage.
-template <typename IO, int V, bool GATE, int W, int LS, bool FULL>
+// exponentials reused (CACHE; else one more ex2 per token, straight to the
+// scale R); one ex2 (gate) and one rcp per output.  Otherwise the exact
+// running-max recurrence from keys read again from the stage.
+template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool CACHE = true>
 __device__ __forceinline__ void seg_pass2(const ChunkArgs& A, const unsigned char* stage, SegCtx<V, LS>& cx,
                                           St* st) {
     constexpr int CB = 32 * V;
@@ -240,14 +243,17 @@ __device__ __forceinline__ void seg_pass2(const ChunkArgs& A, const unsigned cha
     IO* yp = static_cast<IO*>(A.y) + cx.base;
     const int64_t C = A.C;
     if (fast2) {
-        float sl[V], ss[V];
+        float sl[V], ss[V], nr[V];
 #pragma unroll
         for (int j = 0; j < V; ++j) {
             const float R = fmaxf(cx.kmax[j], st[j].p);
-            sl[j] = ex2(cx.kmax[j] - R);
+            sl[j] = CACHE ? ex2(cx.kmax[j] - R) : 0.f;
             ss[j] = ex2(st[j].p - R);
+            nr[j] = -R;
         }
         const F2 SL = f2(sl[0], sl[1]);
+        const F2 NR = f2(nr[0], nr[1]);
+        const F2 L2 = f2s(kLog2e);
         const F2 EU = f2(cx.eu[0], cx.eu[1]);
         const F2 DK = f2(cx.dk[0], cx.dk[1]);
         const F2 NL = f2s(-kLog2e);
@@ -256,7 +262,8 @@ __device__ __forceinline__ void seg_pass2(const ChunkArgs& A, const unsigned cha
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < cx.nvalid) {
-                const F2 ek = mul2(cx.kf[i], SL);
+                const F2 ek = CACHE ? mul2(cx.kf[i], SL)
+                                    : ex2x2(fma2(raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + i * ROW)), L2, NR));
                 const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + TILE + i * ROW)));
                 const F2 num = fma2(EU, ekv, n);
                 F2 den = fma2(EU, ek, db);
@@ -311,7 +318,7 @@ __device__ __forceinline__ bool compute_front(const ChunkArgs& A, int64_t it, un
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int s = static_cast<int>(it % S);
     const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-    if (!mbar_wait(&full[s], ph, A.wait_limit_ns)) {
+    if (!mbar_wait(&full[s], ph, kCopyWaitNs)) {
         if (threadIdx.x == 0 && A.hdr != nullptr) record_timeout(A, -1);
         return false;
     }
@@ -482,7 +489,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         for (int64_t it = 0;; ++it) {
             const int s = static_cast<int>(it % S);
             const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-            if (!mbar_wait(&full[s], ph, A.wait_limit_ns)) {
+            if (!mbar_wait(&full[s], ph, kCopyWaitNs)) {
                 if (lane == 0 && ticket) record_timeout(A, -1);
                 break;
             }
@@ -524,7 +531,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         for (int64_t it = warp - W;; it += G::SCAN) {
             const int s = static_cast<int>(it % S);
             const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-            const int got = mbar_wait_or_end(&full[s], ph, endpos, it, A.wait_limit_ns);
+            const int got = mbar_wait_or_end(&full[s], ph, endpos, it, kCopyWaitNs);
             if (got < 0 && lane == 0 && ticket) record_timeout(A, -1);
             if (got <= 0) break;
             const int64_t u = unitbuf[s];

@@ -147,8 +147,19 @@ __device__ __noinline__ void lane_entry_state(const ChunkArgs& A, const LaneRang
     }
 }
 
-__device__ __forceinline__ void named_sync(int id, int threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+// Named barrier over `threads` threads that also ANDs a flag over them, so
+// every participating thread takes the same branch afterwards.
+__device__ __forceinline__ bool named_sync_and(int id, int threads, bool flag) {
+    uint32_t all;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(all)
+        : "r"(static_cast<uint32_t>(flag)), "r"(id), "r"(threads)
+        : "memory");
+    return all != 0;
 }
 
 template <typename IO, int V, bool GATE, int W, int LS, int S, int MINB = 2>
@@ -164,6 +175,12 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     __shared__ St s_carry[2][V][32];    // state at the start of a chunk, double-buffered
     __shared__ LaneRange s_range;       // this CTA's share of the chunk order
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tk);
+        prefetch_tensormap(&tv);
+        if (GATE) prefetch_tensormap(&tr);
+    }
+    pdl_begin();
     if (threadIdx.x == 0) {
         s_range.init(A.nLB, A.nchunks, blockIdx.x, gridDim.x);
         for (int s = 0; s < S; ++s) {
@@ -238,19 +255,22 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
         for (int64_t chunk = c0; chunk < c1; ++chunk, ++it) {
             const int s = static_cast<int>(it % S);
             const int par = static_cast<int>(it & 1u);
-            if (!mbar_wait(&full[s], (it / S) & 1u, A.wait_limit_ns)) {
+            const bool got = mbar_wait(&full[s], (it / S) & 1u, kCopyWaitNs);
+            const unsigned char* stage = smem + s * G::STAGE;
+            const bool full_chunk = (chunk + 1) * TT <= A.T;
+            St seg[V];
+            if (got) {
+                if (full_chunk) seg_pass01<IO, V, GATE, W, LS, true, false>(A, chunk, b, c, stage, cx, seg);
+                else seg_pass01<IO, V, GATE, W, LS, false, false>(A, chunk, b, c, stage, cx, seg);
+#pragma unroll
+                for (int j = 0; j < V; ++j) s_seg[par][warp][j][lane] = seg[j];
+            }
+            // a copy that did not land stops every compute warp together
+            if (!named_sync_and(1, W * 32, got)) {
                 if (threadIdx.x == 0 && A.hdr != nullptr) record_timeout(A, -1);
                 ok = false;
                 break;
             }
-            const unsigned char* stage = smem + s * G::STAGE;
-            const bool full_chunk = (chunk + 1) * TT <= A.T;
-            St seg[V];
-            if (full_chunk) seg_pass01<IO, V, GATE, W, LS, true, false>(A, chunk, b, c, stage, cx, seg);
-            else seg_pass01<IO, V, GATE, W, LS, false, false>(A, chunk, b, c, stage, cx, seg);
-#pragma unroll
-            for (int j = 0; j < V; ++j) s_seg[par][warp][j][lane] = seg[j];
-            named_sync(1, W * 32);
             // start state of this warp's segment: carried state, then the
             // segments before this one
             // rows of this chunk (all TT but in a sequence's last, partial chunk)

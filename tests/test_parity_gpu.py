@@ -97,6 +97,27 @@ def test_lane_resident_shapes(B, T, C, dtype, gate, state):
     check_forward(d, y, s)
 
 
+# Fewer 64-channel blocks than SMs: the part kernel cuts every sequence into
+# 128-token parts that find their entering state by look-back.
+PART = [
+    # B, T, C, dtype, gate, state
+    (1, 17, 64, torch.float32, True, True),        # a single part, shorter than a part
+    (1, 128, 64, torch.bfloat16, False, True),     # exactly one part
+    (1, 129, 128, torch.float32, True, False),     # one token in the second part
+    (2, 1000, 72, torch.bfloat16, True, True),     # ragged channel block and last part
+    (1, 5000, 256, torch.float32, False, True),    # many parts per lane block
+    (2, 2000, 4096, torch.bfloat16, True, False),  # more parts than CTA slots: claimed in ticket order
+    (3, 777, 1000, torch.bfloat16, False, True),
+]
+
+
+@pytest.mark.parametrize("B,T,C,dtype,gate,state", PART)
+def test_part_shapes(B, T, C, dtype, gate, state):
+    d = gen_case(B, T, C, dtype, gate, state, seed=B * 13 + T + C)
+    y, s = run_forward(d)
+    check_forward(d, y, s)
+
+
 def test_tiny_workload_against_brute_force():
     d = I.make_forward_inputs("tiny", device=DEV)
     y, s = run_forward(d)
@@ -131,9 +152,11 @@ def test_extreme_keys(kval, dtype):
     check_forward(d, y, s)
 
 
-def test_state_in_place_and_chaining():
-    """state_out == state_in is allowed; chaining calls reproduces one pass."""
-    d = gen_case(2, 300, 130, torch.float32, True, True, seed=11)
+@pytest.mark.parametrize("C", [130, 128])
+def test_state_in_place_and_chaining(C):
+    """state_out == state_in is allowed; chaining calls reproduces one pass
+    (C = 130: register-load kernel; C = 128: part kernel)."""
+    d = gen_case(2, 300, C, torch.float32, True, True, seed=11)
     y_full, s_full = run_forward(d)
     st = d["state"].clone()
     parts = []
@@ -194,11 +217,13 @@ def test_empty_and_degenerate_sizes():
     assert torch.all(st[0] == 0) and torch.all(st[1] == 0) and torch.all(st[2] == -1e38)
 
 
+@pytest.mark.parametrize("C", [70, 72])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_guard_bands_untouched(dtype):
+def test_guard_bands_untouched(dtype, C):
     """Outputs land exactly in their buffers: sentinel padding around y and
-    the state survives (bounds check without a sanitizer)."""
-    B, T, C, pad = 2, 333, 70, 4096
+    the state survives (bounds check without a sanitizer).  C = 70 takes the
+    register-load kernel, C = 72 the part kernel."""
+    B, T, pad = 2, 333, 4096
     d = gen_case(B, T, C, dtype, True, True, seed=23)
     n = B * T * C
     ybuf = torch.full((n + 2 * pad,), 12345.0, dtype=dtype, device=DEV)
