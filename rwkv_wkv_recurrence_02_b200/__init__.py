@@ -15,6 +15,7 @@ Two layers:
   non-zero status.
 """
 import ctypes
+import functools
 import os
 import threading
 
@@ -105,10 +106,13 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def _stream_ptr(stream):
+def _stream_ptr(stream, device=None):
+    """cudaStream_t of `stream`, or of the current stream of `device`."""
     torch = _torch()
-    s = torch.cuda.current_stream() if stream is None else stream
-    return s.cuda_stream
+    if stream is not None:
+        return stream.cuda_stream
+    idx = device.index if device is not None and device.index is not None else torch.cuda.current_device()
+    return torch._C._cuda_getCurrentRawStream(idx)
 
 
 def _check(status, where):
@@ -118,6 +122,8 @@ def _check(status, where):
 
 def _need(t, name, shape, dtype, device):
     if t is None:
+        return
+    if t.shape == shape and t.dtype == dtype and t.device == device and t.is_contiguous():
         return
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
@@ -147,7 +153,7 @@ class Workspace:
         if self.buf is None or self.buf.numel() < nbytes:
             dev = self.device if self.device is not None else torch.device("cuda", torch.cuda.current_device())
             self.buf = torch.empty(int(nbytes) + 256, dtype=torch.uint8, device=dev)
-            _check(lib().wkv_workspace_init(self._aligned_ptr(), self.buf.numel() - 256, _stream_ptr(stream)),
+            _check(lib().wkv_workspace_init(self._aligned_ptr(), self.buf.numel() - 256, _stream_ptr(stream, self.buf.device)),
                    "wkv_workspace_init")
         return self._aligned_ptr(), self.buf.numel() - 256
 
@@ -158,11 +164,11 @@ class Workspace:
     def status(self, stream=None) -> int:
         if self.buf is None:
             return 0
-        return lib().wkv_workspace_status(self._aligned_ptr(), _stream_ptr(stream))
+        return lib().wkv_workspace_status(self._aligned_ptr(), _stream_ptr(stream, self.buf.device))
 
     def reset(self, stream=None):
         if self.buf is not None:
-            _check(lib().wkv_workspace_init(self._aligned_ptr(), self.buf.numel() - 256, _stream_ptr(stream)),
+            _check(lib().wkv_workspace_init(self._aligned_ptr(), self.buf.numel() - 256, _stream_ptr(stream, self.buf.device)),
                    "wkv_workspace_init")
 
 
@@ -177,6 +183,7 @@ def default_workspace(device) -> Workspace:
     return ws
 
 
+@functools.lru_cache(maxsize=1024)
 def workspace_bytes(B: int, T: int, C: int, dtype_code: int) -> int:
     return int(lib().wkv_forward_workspace_bytes(B, T, C, dtype_code))
 
@@ -208,9 +215,10 @@ def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, wa
         state_out = torch.empty((3, B, C), dtype=torch.float32, device=dev)
     _need(state_out, "state_out", (3, B, C), torch.float32, dev)
     ws = workspace if workspace is not None else default_workspace(dev)
+    sp = _stream_ptr(stream, dev)
     ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
     _check(lib().wkv_forward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
-                             _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, _stream_ptr(stream)), "wkv_forward")
+                             _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, sp), "wkv_forward")
     return y, state_out
 
 
@@ -231,7 +239,7 @@ def wkv_forward_noalloc(w, u, k, v, r=None, state_in=None, *, y, state_out=None,
     _need(state_in, "state_in", (3, B, C), torch.float32, dev)
     _need(state_out, "state_out", (3, B, C), torch.float32, dev)
     _check(lib().wkv_forward_noalloc(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
-                                     _ptr(y), _ptr(state_out), _stream_ptr(stream)), "wkv_forward_noalloc")
+                                     _ptr(y), _ptr(state_out), _stream_ptr(stream, dev)), "wkv_forward_noalloc")
     return y, state_out
 
 
@@ -255,5 +263,5 @@ def wkv_step(w, u, k, v, state, r=None, *, y=None, stream=None):
         y = torch.empty((Lr, B, C), dtype=k.dtype, device=dev)
     _need(y, "y", (Lr, B, C), k.dtype, dev)
     _check(lib().wkv_step(Lr, B, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state), _ptr(y),
-                          _stream_ptr(stream)), "wkv_step")
+                          _stream_ptr(stream, dev)), "wkv_step")
     return y

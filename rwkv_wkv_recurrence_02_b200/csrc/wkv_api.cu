@@ -41,12 +41,12 @@ constexpr int kMinTT = (kW < kWsW ? kW : kWsW) * kLS;
 // chunks).
 constexpr int kLaneW = 4;
 constexpr int kLaneLS = 16;
-// Part kernel: compute warps and tokens per warp segment (128-token parts).
-// It runs when there are fewer 64-channel lane blocks than SMs; the
-// lane-resident kernel from there on.
-constexpr int kPartW = 8;
+// Part kernel: compute warps and tokens per warp segment (64-token parts),
+// four CTAs per SM.  It runs when there are fewer 64-channel lane blocks
+// than SMs; the lane-resident kernel from there on.
+constexpr int kPartW = 4;
 constexpr int kPartLS = 16;
-constexpr int kPartMinBlocks = 2;
+constexpr int kPartMinBlocks = 4;
 // look-back window (parts per round trip) and whether pass 1 keeps its
 // exponentials in registers for pass 2
 constexpr int kPartWin = 1;

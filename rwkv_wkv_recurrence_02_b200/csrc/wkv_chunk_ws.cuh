@@ -179,7 +179,7 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, in
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < cx.nvalid) {
                 const F2 ek = ex2x2(fma2(cx.kf[i], L2, KM));
-                if (CACHE) cx.kf[i] = ek;
+                if constexpr (CACHE) cx.kf[i] = ek;
                 const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + TILE + i * ROW)));
                 n = fma2(n, DK, ekv);
                 db = fma2(db, DK, ek);
@@ -262,8 +262,9 @@ __device__ __forceinline__ void seg_pass2(const ChunkArgs& A, const unsigned cha
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < cx.nvalid) {
-                const F2 ek = CACHE ? mul2(cx.kf[i], SL)
-                                    : ex2x2(fma2(raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + i * ROW)), L2, NR));
+                F2 ek;
+                if constexpr (CACHE) ek = mul2(cx.kf[i], SL);
+                else ek = ex2x2(fma2(raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + i * ROW)), L2, NR));
                 const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + TILE + i * ROW)));
                 const F2 num = fma2(EU, ekv, n);
                 F2 den = fma2(EU, ek, db);

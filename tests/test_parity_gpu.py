@@ -98,12 +98,14 @@ def test_lane_resident_shapes(B, T, C, dtype, gate, state):
 
 
 # Fewer 64-channel blocks than SMs: the part kernel cuts every sequence into
-# 128-token parts that find their entering state by look-back.
+# 64-token parts that find their entering state by look-back.
 PART = [
     # B, T, C, dtype, gate, state
     (1, 17, 64, torch.float32, True, True),        # a single part, shorter than a part
-    (1, 128, 64, torch.bfloat16, False, True),     # exactly one part
-    (1, 129, 128, torch.float32, True, False),     # one token in the second part
+    (1, 64, 64, torch.bfloat16, False, True),      # exactly one part
+    (1, 65, 128, torch.float32, True, False),      # one token in the second part
+    (1, 128, 64, torch.bfloat16, False, True),
+    (1, 129, 128, torch.float32, True, False),
     (2, 1000, 72, torch.bfloat16, True, True),     # ragged channel block and last part
     (1, 5000, 256, torch.float32, False, True),    # many parts per lane block
     (2, 2000, 4096, torch.bfloat16, True, False),  # more parts than CTA slots: claimed in ticket order
