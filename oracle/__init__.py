@@ -32,6 +32,7 @@ def lib():
         L.oracle_wkv_step.argtypes = [i64, i64, i64, p, p, p, p, p, p, p, i32]
         L.oracle_wkv_summary.argtypes = [d, i64, p, p, p]
         L.oracle_wkv_combine.argtypes = [d, d, d, d, d, d, d, i64, p]
+        L.oracle_wkv_backward.argtypes = [i64, i64, i64, p, p, p, p, p, p, p, p, p, p, p, p, p, p, i32]
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -102,6 +103,31 @@ def wkv_step(w, u, k, v, state, r=None, nthreads=0):
     lib().oracle_wkv_step(Lr, B, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
                           _ptr(state), _ptr(y), int(nthreads))
     return y
+
+
+def wkv_backward(w, u, k, v, r=None, state_in=None, dy=None, dstate_out=None, nthreads=0):
+    """Gradients of wkv_forward: given dy (B, T, C) and dstate_out (3, B, C)
+    (dL/d(a, b) of the returned state; its p plane is not read), returns
+    (dk, dv, dr, dw, du, dstate_in) as float64; dr is None without a gate,
+    dw and du are (C,) sums over sequences and tokens, dstate_in is
+    dL/d(a0, b0, p0) of state_in (zeros for the empty state)."""
+    w, u, k, v, r, state_in = _f32(w), _f32(u), _f32(k), _f32(v), _f32(r), _f64(state_in)
+    B, T, C = _check_forward_args(k, w, u, v, r, state_in)
+    dy, dstate_out = _f64(dy), _f64(dstate_out)
+    if dy is None or dy.shape != (B, T, C):
+        raise ValueError("dy must be (B, T, C)")
+    if dstate_out is not None and dstate_out.shape != (3, B, C):
+        raise ValueError("dstate_out must be (3, B, C)")
+    dk = np.empty((B, T, C), np.float64)
+    dv = np.empty((B, T, C), np.float64)
+    dr = np.empty((B, T, C), np.float64) if r is not None else None
+    dw = np.empty(C, np.float64)
+    du = np.empty(C, np.float64)
+    ds = np.empty((3, B, C), np.float64)
+    lib().oracle_wkv_backward(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
+                              _ptr(dy), _ptr(dstate_out), _ptr(dk), _ptr(dv), _ptr(dr), _ptr(dw), _ptr(du),
+                              _ptr(ds), int(nthreads))
+    return dk, dv, dr, dw, du, ds
 
 
 def fresh_state(B, C):

@@ -245,3 +245,119 @@ void oracle_wkv_combine(double w, double p, double a, double b,
     out[1] = e1 * a + e2 * A;
     out[2] = e1 * b + e2 * Bd;
 }
+
+/*
+ * Reverse mode (gradients) of oracle_wkv_forward over one chunk.  The pages
+ * state that the parallel mode trains the model but print no gradient; this
+ * is the chain rule applied to the recurrence of "リカレント定式化" in the
+ * output-then-update order of "並列学習の定式化", per lane (0-based t):
+ *
+ *   N_{t+1} = lam N_t + e^{k_t} v_t,   D_{t+1} = lam D_t + e^{k_t},   lam = e^{-w}
+ *   num_t = N_t + e^{u+k_t} v_t,  den_t = D_t + e^{u+k_t},  wkv_t = num_t / den_t
+ *   y_t = g_t wkv_t,  g_t = sigmoid(r_t) (1 without a gate)
+ *
+ * with (N_0, D_0) = (a0 e^{p0}, b0 e^{p0}) from state_in.  Given dy = dL/dy
+ * and ds_out = dL/d(a_T, b_T) for the state the forward returns (its p plane
+ * is not read: later uses of a state depend on it only through N = a e^p and
+ * D = b e^p, so dL/dN_T = dL/da_T e^{-p_T}), with gN_t = dL/dN_t, gD_t =
+ * dL/dD_t summed over every later use:
+ *
+ *   dnum_t = g_t dy_t / den_t,  dden_t = -g_t dy_t wkv_t / den_t
+ *   gN_t = dnum_t + lam gN_{t+1},   gD_t = dden_t + lam gD_{t+1}
+ *   dv_t = dnum_t e^{u+k_t} + gN_{t+1} e^{k_t}
+ *   dk_t = (dnum_t v_t + dden_t) e^{u+k_t} + (gN_{t+1} v_t + gD_{t+1}) e^{k_t}
+ *   du  += (dnum_t v_t + dden_t) e^{u+k_t}
+ *   dw  += -lam (gN_{t+1} N_t + gD_{t+1} D_t)
+ *   dr_t = dy_t wkv_t g_t (1 - g_t)
+ *   ds_in = (gN_0 e^{p0}, gD_0 e^{p0}, a0 gN_0 e^{p0} + b0 gD_0 e^{p0})
+ *
+ * dw and du are summed over every sequence and token of their channel.
+ * Arithmetic: plain IEEE double, with every exponent of a lane shifted by
+ * the lane's largest weight exponent (all gradients are invariant to that
+ * shift), so weights are <= 1.  Valid while the smallest terms that matter
+ * stay inside double range, which holds for the test inputs (|k| <= 60,
+ * T up to a few thousand).  p_T, the scale of the returned state, is taken
+ * from the same log-space recurrence as oracle_wkv_forward.
+ *
+ * dr may be NULL (no gate); ds_out NULL means zero; ds_in may be NULL.
+ */
+void oracle_wkv_backward(int64_t B, int64_t T, int64_t C,
+                         const float* w, const float* u,
+                         const float* k, const float* v, const float* r,
+                         const double* state_in, const double* dy, const double* ds_out,
+                         double* dk, double* dv, double* dr, double* dw, double* du,
+                         double* ds_in, int nthreads) {
+    set_threads(nthreads);
+    const int64_t lanes = B * C;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        const double wc = (double)w[c], uc = (double)u[c], lam = exp(-wc);
+        double* Nt = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        double* Dt = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        double dw_c = 0.0, du_c = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            const int64_t lane = b * C + c;
+            double a0 = 0.0, b0 = 0.0, p0 = ORACLE_FRESH_P;
+            if (state_in) {
+                a0 = state_in[0 * lanes + lane];
+                b0 = state_in[1 * lanes + lane];
+                p0 = state_in[2 * lanes + lane];
+            }
+            /* the lane's largest weight exponent, and p_T of the forward */
+            double m = p0, sa = a0, sb = b0, sp = p0, sc = 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t it = (b * T + t) * C + c;
+                const double kt = (double)k[it];
+                if (kt > m) m = kt;
+                if (uc + kt > m) m = uc + kt;
+                lane_step(wc, uc, kt, (double)v[it], &sa, &sb, &sp, &sc, NULL);
+            }
+            const double pT = sp;
+            /* forward: N_t, D_t before token t, shifted by e^{-m} */
+            double N = a0 * exp(p0 - m), D = b0 * exp(p0 - m);
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t it = (b * T + t) * C + c;
+                Nt[t] = N;
+                Dt[t] = D;
+                const double et = exp((double)k[it] - m);
+                N = lam * N + et * (double)v[it];
+                D = lam * D + et;
+            }
+            /* reverse: gN, gD = dL/dN_{t+1}, dL/dD_{t+1} (shifted by e^{+m}) */
+            double gN = 0.0, gD = 0.0;
+            if (ds_out) {
+                const double s = exp(m - pT);
+                gN = ds_out[0 * lanes + lane] * s;
+                gD = ds_out[1 * lanes + lane] * s;
+            }
+            for (int64_t t = T - 1; t >= 0; --t) {
+                const int64_t it = (b * T + t) * C + c;
+                const double kt = (double)k[it], vt = (double)v[it];
+                const double et = exp(kt - m), Et = exp(uc + kt - m);
+                const double num = Nt[t] + Et * vt, den = Dt[t] + Et;
+                const double wkv = num / den;
+                const double g = r ? sigmoid_f64((double)r[it]) : 1.0;
+                const double h = g * dy[it];
+                const double dnum = h / den, dden = -h * wkv / den;
+                dv[it] = dnum * Et + gN * et;
+                dk[it] = (dnum * vt + dden) * Et + (gN * vt + gD) * et;
+                du_c += (dnum * vt + dden) * Et;
+                dw_c += -lam * (gN * Nt[t] + gD * Dt[t]);
+                if (dr) dr[it] = dy[it] * wkv * g * (1.0 - g);
+                gN = dnum + lam * gN;
+                gD = dden + lam * gD;
+            }
+            if (ds_in) {
+                const double s = exp(p0 - m);
+                const double ga = gN * s, gb = gD * s;
+                ds_in[0 * lanes + lane] = ga;
+                ds_in[1 * lanes + lane] = gb;
+                ds_in[2 * lanes + lane] = a0 * ga + b0 * gb;
+            }
+        }
+        dw[c] = dw_c;
+        du[c] = du_c;
+        free(Nt);
+        free(Dt);
+    }
+}
