@@ -174,6 +174,60 @@ int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype,
 /* Scratch bytes wkv_forward_noalloc would use for these sizes (0: none). */
 size_t wkv_forward_noalloc_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype);
 
+/*
+ * wkv_backward -- gradients of wkv_forward over one chunk (reverse mode).
+ * The pages state that the parallel mode is what trains the model (article
+ * section "並列学習の定式化") but print no gradient; this is the chain rule
+ * through the recurrence of "リカレント定式化", per lane, with N_t, D_t the
+ * state's numerator and denominator before token t, lam = e^{-w},
+ * den_t = D_t + e^{u+k_t}, wkv_t = (N_t + e^{u+k_t} v_t) / den_t:
+ *
+ *   dnum_t = g_t dy_t / den_t,  dden_t = -dnum_t wkv_t   (g_t = sigmoid(r_t), or 1)
+ *   gN_t = dnum_t + lam gN_{t+1},  gD_t = dden_t + lam gD_{t+1}     (dL/dN_t, dL/dD_t)
+ *   dv_t = dnum_t e^{u+k_t} + gN_{t+1} e^{k_t}
+ *   dk_t = (dnum_t v_t + dden_t) e^{u+k_t} + (gN_{t+1} v_t + gD_{t+1}) e^{k_t}
+ *   du = sum (dnum_t v_t + dden_t) e^{u+k_t},   dw = -lam sum (gN_{t+1} N_t + gD_{t+1} D_t)
+ *   dr_t = dy_t wkv_t g_t (1 - g_t)
+ *
+ * Same sizes, dtype, layouts and state semantics as wkv_forward.
+ *   w, u, k, v, r, state_in   the forward's inputs (r NULL: no gate; state_in
+ *                             NULL: the empty state).
+ *   dy                        (B,T,C) dL/dy, in `dtype`.
+ *   dstate_out                (3,B,C) float32 dL/d(a, b) of the state the
+ *                             forward returned, or NULL (zero).  Its p plane
+ *                             is not read: every later use of a state depends
+ *                             on it only through N = a e^p and D = b e^p, so
+ *                             the chain continues through dL/dN = dL/da e^{-p}.
+ *   dk, dv                    (B,T,C) outputs in `dtype`.
+ *   dr                        (B,T,C) output in `dtype`; NULL exactly when r is.
+ *   dw, du                    (C,) float32 outputs: sums over every sequence
+ *                             and token of the channel (written, not added to).
+ *                             dw is dL/dw; with w = exp(decay) the decay's
+ *                             gradient is dw * w.
+ *   dstate_in                 (3,B,C) float32 output dL/d(a0, b0, p0), or NULL;
+ *                             dL/dp0 = a0 dL/da0 + b0 dL/db0.  Feeding its a, b
+ *                             planes as dstate_out of the previous chunk
+ *                             chains chunks exactly.
+ *   workspace                 at least wkv_backward_workspace_bytes() bytes,
+ *                             256-byte aligned, zeroed once by
+ *                             wkv_workspace_init() before its first use (a
+ *                             wkv_forward workspace of that size serves too).
+ * Requirements of this version: every array 16-byte aligned and C a multiple
+ * of 4 (WKV_ERR_ALIGN otherwise).  No output may overlap an input or another
+ * output (WKV_ERR_ALIAS).  T == 0: dw = du = 0 and dstate_in passes
+ * dstate_out through.  Asynchronous on `stream` like every call.
+ */
+int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype,
+                 const float* w, const float* u,
+                 const void* k, const void* v, const void* r,
+                 const float* state_in, const void* dy, const float* dstate_out,
+                 void* dk, void* dv, void* dr, float* dw, float* du, float* dstate_in,
+                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of workspace wkv_backward needs for these sizes (0 for invalid sizes
+ * or no elements). */
+size_t wkv_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype);
+
 /* Static English text for a wkv_status value. */
 const char* wkv_strerror(int status);
 

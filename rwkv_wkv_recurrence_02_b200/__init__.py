@@ -31,8 +31,8 @@ STATUS = {
 }
 # the functions include/wkv.h declares
 EXPORTS = ("wkv_forward", "wkv_forward_workspace_bytes", "wkv_workspace_init", "wkv_workspace_status",
-           "wkv_step", "wkv_forward_noalloc", "wkv_forward_noalloc_scratch_bytes", "wkv_strerror",
-           "wkv_last_cuda_error", "wkv_abi_version")
+           "wkv_step", "wkv_forward_noalloc", "wkv_forward_noalloc_scratch_bytes", "wkv_backward",
+           "wkv_backward_workspace_bytes", "wkv_strerror", "wkv_last_cuda_error", "wkv_abi_version")
 
 _lib = None
 _lock = threading.Lock()
@@ -75,6 +75,11 @@ def lib():
         L.wkv_forward_noalloc.restype = i32
         L.wkv_forward_noalloc_scratch_bytes.argtypes = [i64, i64, i64, i32]
         L.wkv_forward_noalloc_scratch_bytes.restype = sz
+        L.wkv_backward.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                   vp, sz, vp]
+        L.wkv_backward.restype = i32
+        L.wkv_backward_workspace_bytes.argtypes = [i64, i64, i64, i32]
+        L.wkv_backward_workspace_bytes.restype = sz
         L.wkv_strerror.argtypes = [i32]
         L.wkv_strerror.restype = ctypes.c_char_p
         L.wkv_last_cuda_error.argtypes = []
@@ -241,6 +246,56 @@ def wkv_forward_noalloc(w, u, k, v, r=None, state_in=None, *, y, state_out=None,
     _check(lib().wkv_forward_noalloc(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
                                      _ptr(y), _ptr(state_out), _stream_ptr(stream, dev)), "wkv_forward_noalloc")
     return y, state_out
+
+
+@functools.lru_cache(maxsize=1024)
+def backward_workspace_bytes(B: int, T: int, C: int, dtype_code: int) -> int:
+    return int(lib().wkv_backward_workspace_bytes(B, T, C, dtype_code))
+
+
+def wkv_backward(w, u, k, v, r=None, state_in=None, *, dy, dstate_out=None, dk=None, dv=None, dr=None,
+                 dw=None, du=None, dstate_in=None, want_dstate_in=True, workspace: Workspace = None, stream=None):
+    """Gradients of wkv_forward.  dy: (B, T, C) like k; dstate_out: (3, B, C)
+    float32 dL/d(a, b) of the returned state, or None.  Returns (dk, dv, dr,
+    dw, du, dstate_in); dr is None without a gate, dw and du are (C,) float32
+    sums over sequences and tokens."""
+    torch = _torch()
+    B, T, C = k.shape
+    dev = k.device
+    if dev.type != "cuda":
+        raise ValueError("wkv_backward runs on CUDA tensors only")
+    code = _dtype_code(k)
+    for t, name in ((v, "v"), (r, "r"), (dy, "dy")):
+        _need(t, name, (B, T, C), k.dtype, dev)
+    _need(w, "w", (C,), torch.float32, dev)
+    _need(u, "u", (C,), torch.float32, dev)
+    _need(k, "k", (B, T, C), k.dtype, dev)
+    _need(state_in, "state_in", (3, B, C), torch.float32, dev)
+    _need(dstate_out, "dstate_out", (3, B, C), torch.float32, dev)
+    if dk is None:
+        dk = torch.empty((B, T, C), dtype=k.dtype, device=dev)
+    if dv is None:
+        dv = torch.empty((B, T, C), dtype=k.dtype, device=dev)
+    if dr is None and r is not None:
+        dr = torch.empty((B, T, C), dtype=k.dtype, device=dev)
+    if dw is None:
+        dw = torch.empty((C,), dtype=torch.float32, device=dev)
+    if du is None:
+        du = torch.empty((C,), dtype=torch.float32, device=dev)
+    if dstate_in is None and want_dstate_in:
+        dstate_in = torch.empty((3, B, C), dtype=torch.float32, device=dev)
+    for t, name in ((dk, "dk"), (dv, "dv"), (dr, "dr")):
+        _need(t, name, (B, T, C), k.dtype, dev)
+    _need(dw, "dw", (C,), torch.float32, dev)
+    _need(du, "du", (C,), torch.float32, dev)
+    _need(dstate_in, "dstate_in", (3, B, C), torch.float32, dev)
+    ws = workspace if workspace is not None else default_workspace(dev)
+    sp = _stream_ptr(stream, dev)
+    ws_ptr, ws_bytes = ws.get(backward_workspace_bytes(B, T, C, code), stream)
+    _check(lib().wkv_backward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
+                              _ptr(dy), _ptr(dstate_out), _ptr(dk), _ptr(dv), _ptr(dr), _ptr(dw), _ptr(du),
+                              _ptr(dstate_in), ws_ptr, ws_bytes, sp), "wkv_backward")
+    return dk, dv, dr, dw, du, dstate_in
 
 
 def wkv_step(w, u, k, v, state, r=None, *, y=None, stream=None):

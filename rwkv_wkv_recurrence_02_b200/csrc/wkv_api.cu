@@ -17,6 +17,7 @@
 #include "wkv_chunk_ws.cuh"
 #include "wkv_lane.cuh"
 #include "wkv_part.cuh"
+#include "wkv_backward.cuh"
 #include "wkv_seq.cuh"
 #include "wkv_step.cuh"
 
@@ -283,10 +284,10 @@ int launch_tma(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
 
 // Lane-resident kernel: each CTA owns whole lane blocks; grid = min(lane
 // blocks, resident capacity).
-template <typename IO, bool GATE, int STAGES>
+template <typename IO, bool GATE, int STAGES, bool CKPT = false>
 int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
     using G = wkv::LaneGeometry<IO, 2, GATE, kLaneW, kLaneLS, STAGES>;
-    auto kern = wkv::lane_forward_kernel<IO, 2, GATE, kLaneW, kLaneLS, STAGES>;
+    auto kern = wkv::lane_forward_kernel<IO, 2, GATE, kLaneW, kLaneLS, STAGES, 2, CKPT>;
     static int capacity[kMaxDevices] = {0};
     int dev = 0;
     int rc = record_cuda(cudaGetDevice(&dev));
@@ -316,7 +317,7 @@ int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
         if (workspace == nullptr) return WKV_ERR_WORKSPACE;
         if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
         if (workspace_bytes < 256 + size_t(a.nLB) * G::CB * sizeof(wkv::Word) ||
-            workspace_bytes < wkv_forward_workspace_bytes(a.B, a.T, a.C, dtype))
+            (!CKPT && workspace_bytes < wkv_forward_workspace_bytes(a.B, a.T, a.C, dtype)))
             return WKV_ERR_WORKSPACE;
         a.hdr = reinterpret_cast<wkv::WsHeader*>(workspace);
         a.incw = reinterpret_cast<wkv::Word*>(static_cast<char*>(workspace) + 256);
@@ -769,3 +770,197 @@ int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype, const float*
 
 }  // extern "C"
 
+
+// ---------------------------------------------------------------------------
+// reverse mode
+// ---------------------------------------------------------------------------
+namespace {
+
+// Backward kernel: 8 compute warps x 8-token segments, the 64-token chunks
+// of the checkpoint sweep.
+constexpr int kBwdW = 8;
+constexpr int kBwdLS = 8;
+static_assert(kBwdW * kBwdLS == kLaneW * kLaneLS, "the backward walks the checkpoint sweep's chunks");
+
+struct BwdLayout {
+    int64_t nCB, nLB, nchunks;
+    size_t ckpt_off, part_off, bytes;
+};
+
+// Workspace of wkv_backward: header, the checkpoint sweep's hand-off words,
+// the checkpoints, the dw/du partials.
+BwdLayout bwd_layout(int64_t B, int64_t T, int64_t C) {
+    BwdLayout L{};
+    constexpr int64_t CB = 64;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    L.nCB = (C + CB - 1) / CB;
+    L.nLB = B * L.nCB;
+    L.nchunks = (T + kBwdW * kBwdLS - 1) / (kBwdW * kBwdLS);
+    L.ckpt_off = 256 + up(size_t(L.nLB) * CB * sizeof(wkv::Word));
+    L.part_off = L.ckpt_off + up(size_t(L.nchunks + 1) * size_t(L.nLB) * CB * sizeof(wkv::St));
+    L.bytes = L.part_off + up(2 * size_t(L.nLB) * CB * sizeof(float));
+    return L;
+}
+
+template <typename IO, bool GATE, int S, int MINB>
+int launch_backward(const wkv::BwdArgs& a, int dtype, cudaStream_t st) {
+    using G = wkv::BwdGeometry<IO, GATE, kBwdW, kBwdLS, S>;
+    auto kern = wkv::lane_backward_kernel<IO, GATE, kBwdW, kBwdLS, S, MINB>;
+    static bool ready[kMaxDevices] = {false};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (!ready[dev]) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        ready[dev] = true;
+    }
+    CUtensorMap tk, tv, tdy, tr;
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
+        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
+        !encode_map(&tdy, a.dy, dtype, a.B, a.T, a.C, G::CB, G::TT))
+        return WKV_ERR_CUDA;
+    if (GATE) {
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT)) return WKV_ERR_CUDA;
+    } else {
+        tr = tk;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.nLB));
+    cfg.blockDim = dim3(G::THREADS);
+    cfg.dynamicSmemBytes = G::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tk, tv, tdy, tr, a));
+}
+
+template <typename IO>
+int run_backward(const wkv::BwdArgs& b, wkv::ChunkArgs f, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
+    // checkpoint sweep (ring depth as in the forward), then the reverse walk
+    constexpr int SF = sizeof(IO) == 4 ? 2 : 3;
+    int rc = launch_lane<IO, false, SF, true>(f, dtype, ws, ws_bytes, st);
+    if (rc != WKV_OK) return rc;
+    // stages: three with one CTA per SM for fp32, two with two CTAs for bf16
+    if constexpr (sizeof(IO) == 4)
+        return b.r != nullptr ? launch_backward<IO, true, 3, 1>(b, dtype, st) : launch_backward<IO, false, 3, 1>(b, dtype, st);
+    else
+        return b.r != nullptr ? launch_backward<IO, true, 2, 2>(b, dtype, st) : launch_backward<IO, false, 2, 2>(b, dtype, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wkv_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype) {
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n) || (dtype != WKV_F32 && dtype != WKV_BF16)) return 0;
+    if (n == 0) return 0;
+    return bwd_layout(B, T, C).bytes;
+}
+
+int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                 const void* k, const void* v, const void* r, const float* state_in, const void* dy,
+                 const float* dstate_out, void* dk, void* dv, void* dr, float* dw, float* du, float* dstate_in,
+                 void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
+    if (C == 0) return WKV_OK;
+    if (!dw || !du) return WKV_ERR_NULLPTR;
+    const int64_t lanes = B * C;
+    const size_t eb = elem_bytes(dtype);
+    const size_t io_bytes = size_t(n) * eb, st_bytes = size_t(lanes) * 3 * 4, p_bytes = size_t(C) * 4;
+    if (!aligned(dw, 4) || !aligned(du, 4)) return WKV_ERR_ALIGN;
+    if (overlaps(dw, p_bytes, du, p_bytes)) return WKV_ERR_ALIAS;
+    if (n == 0) {
+        // no token: dw = du = 0, and the returned state's gradient passes through
+        int rc = record_cuda(cudaMemsetAsync(dw, 0, p_bytes, stream));
+        if (rc != WKV_OK) return rc;
+        rc = record_cuda(cudaMemsetAsync(du, 0, p_bytes, stream));
+        if (rc != WKV_OK || dstate_in == nullptr || lanes == 0) return rc;
+        if (!aligned(dstate_in, 4) || (state_in && !aligned(state_in, 4)) || (dstate_out && !aligned(dstate_out, 4)))
+            return WKV_ERR_ALIGN;
+        wkv::bwd_passthrough_kernel<<<static_cast<unsigned>((lanes + 255) / 256), 256, 0, stream>>>(
+            lanes, state_in, dstate_out, dstate_in);
+        return check_launch();
+    }
+    if (!w || !u || !k || !v || !dy || !dk || !dv) return WKV_ERR_NULLPTR;
+    if ((r == nullptr) != (dr == nullptr)) return WKV_ERR_NULLPTR;
+    // TMA tiles and paired-channel stores: 16-byte aligned arrays, C a multiple of 4
+    const void* arrs[] = {k, v, r, dy, dk, dv, dr, w, u, state_in, dstate_out, dstate_in};
+    for (const void* p : arrs)
+        if (p && !aligned(p, 16)) return WKV_ERR_ALIGN;
+    if (C % 4 != 0 || (C * int64_t(eb)) % 16 != 0) return WKV_ERR_ALIGN;
+    if (B >= (int64_t(1) << 31) || T >= (int64_t(1) << 31) || C >= (int64_t(1) << 31)) return WKV_ERR_SHAPE;
+    // outputs overlap no input and no other output
+    struct Span { const void* p; size_t n; };
+    const Span ins[] = {{w, p_bytes}, {u, p_bytes}, {k, io_bytes}, {v, io_bytes}, {r, io_bytes},
+                        {state_in, st_bytes}, {dy, io_bytes}, {dstate_out, st_bytes}};
+    const Span outs[] = {{dk, io_bytes}, {dv, io_bytes}, {dr, io_bytes}, {dw, p_bytes}, {du, p_bytes},
+                         {dstate_in, st_bytes}};
+    for (const Span& o : outs) {
+        for (const Span& i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return WKV_ERR_ALIAS;
+        for (const Span& o2 : outs)
+            if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return WKV_ERR_ALIAS;
+    }
+    const BwdLayout L = bwd_layout(B, T, C);
+    if (workspace == nullptr || workspace_bytes < L.bytes) return WKV_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
+    char* ws = static_cast<char*>(workspace);
+    if (L.nLB > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    if (encode_fn() == nullptr) return WKV_ERR_CUDA;   // no driver entry point for tensor maps
+
+    wkv::ChunkArgs f{};
+    f.w = w;
+    f.u = u;
+    f.k = k;
+    f.v = v;
+    f.s_in = state_in;
+    f.B = B;
+    f.T = T;
+    f.C = C;
+    f.nCB = L.nCB;
+    f.nLB = L.nLB;
+    f.nchunks = L.nchunks;
+    f.units = L.nLB * L.nchunks;
+    f.ckpt = reinterpret_cast<wkv::St*>(ws + L.ckpt_off);
+    f.wait_limit_ns = wait_limit_ns();
+
+    wkv::BwdArgs b{};
+    b.w = w;
+    b.u = u;
+    b.k = k;
+    b.v = v;
+    b.r = r;
+    b.dy = dy;
+    b.s_in = state_in;
+    b.ds_out = dstate_out;
+    b.dk = dk;
+    b.dv = dv;
+    b.dr = dr;
+    b.ds_in = dstate_in;
+    b.ckpt = f.ckpt;
+    b.part = reinterpret_cast<float*>(ws + L.part_off);
+    b.B = B;
+    b.T = T;
+    b.C = C;
+    b.nCB = L.nCB;
+    b.nLB = L.nLB;
+    b.nchunks = L.nchunks;
+    b.wait_limit_ns = f.wait_limit_ns;
+    if (B > 0) {
+        const int rc = dtype == WKV_F32 ? run_backward<float>(b, f, dtype, workspace, workspace_bytes, stream)
+                                        : run_backward<__nv_bfloat16>(b, f, dtype, workspace, workspace_bytes, stream);
+        if (rc != WKV_OK) return rc;
+    }
+    wkv::bwd_reduce_kernel<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(b.part, B, C, L.nCB, dw, du);
+    return check_launch();
+}
+
+}  // extern "C"

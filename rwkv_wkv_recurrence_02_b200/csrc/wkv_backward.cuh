@@ -1,0 +1,433 @@
+// wkv_backward.cuh -- reverse mode (gradients) of the WKV operator.
+//
+// The pages say the parallel mode is what trains the model ("並列学習の定式化")
+// but print no gradient; this is the chain rule through the recurrence of
+// "リカレント定式化" in the output-then-update order, per lane (0-based t,
+// natural units, lam = e^{-w}):
+//
+//   N_{t+1} = lam N_t + e^{k_t} v_t,   D_{t+1} = lam D_t + e^{k_t}
+//   wkv_t = (N_t + e^{u+k_t} v_t) / (D_t + e^{u+k_t}),   y_t = g_t wkv_t
+//
+// With gN_t, gD_t = dL/dN_t, dL/dD_t and c_t = (dnum_t, dden_t) =
+// (g_t dy_t, -g_t dy_t wkv_t) / den_t, the gradients obey the reverse
+// recurrence gN_t = c_t + lam gN_{t+1} (and gD likewise), and
+//
+//   dv_t = dnum_t e^{u+k_t} + gN_{t+1} e^{k_t}
+//   dk_t = (dnum_t v_t + dden_t) e^{u+k_t} + (gN_{t+1} v_t + gD_{t+1}) e^{k_t}
+//   du = sum (dnum_t v_t + dden_t) e^{u+k_t},  dw = -lam sum (gN_{t+1} N_t + gD_{t+1} D_t)
+//   dr_t = dy_t wkv_t g_t (1 - g_t)
+//
+// Everything is kept in base-2 max form like the forward: a forward state is
+// (p, a, b) with N = a 2^p, and a reverse state is (x, A, B) with gN = A 2^x,
+// gD = B 2^x, so st_combine folds both.  Every product of a forward weight
+// and a reverse weight is formed as one 2^(sum of exponents), which stays in
+// range.
+//
+// Work split: one CTA per lane block (64 channels of one sequence) walks its
+// 64-token chunks from the last to the first, carrying the reverse state; a
+// producer warp streams the k, v, dy (and r) tiles of each chunk, and the
+// forward state entering the chunk (from the checkpoint sweep), into a ring
+// of S shared-memory stages with TMA.  Warp s of the W compute warps owns the
+// chunk's segment s of LS tokens:
+//
+//   sweep 0   the segment's forward summary from the empty state; the warps'
+//             summaries meet in shared memory, and each warp's entering
+//             forward state F is the chunk's checkpoint followed by the
+//             summaries before its own.
+//   sweep A   forward from F: outputs, c_t (kept in registers as
+//             (exponent, dnum, dden)), dr_t, du, and the segment's reverse
+//             summary (the reverse state the segment alone produces at its
+//             start).
+//   fold      each warp's reverse state at its segment end is the chunk's
+//             carried reverse state followed by the reverse summaries of the
+//             segments after its own; warp 0 also forms the carry for the
+//             chunk before.
+//   sweep B   backward from there: dk_t, dv_t; the registers of c_t now keep
+//             the reverse state after token t.
+//   sweep C   forward from F again: dw.
+//
+// The checkpoint sweep is the lane-resident forward kernel in its checkpoint
+// mode; a last kernel sums the per-lane-block dw, du partials per channel.
+#pragma once
+
+#include "wkv_lane.cuh"
+
+namespace wkv {
+
+struct BwdArgs {
+    const float* w;
+    const float* u;
+    const void* k;
+    const void* v;
+    const void* r;
+    const void* dy;
+    const float* s_in;
+    const float* ds_out;
+    void* dk;
+    void* dv;
+    void* dr;
+    float* ds_in;
+    const St* ckpt;     // [nchunks + 1][nLB][CB], see ChunkArgs::ckpt
+    float* part;        // [2][nLB][CB]: dw, du of each lane block
+    int64_t B, T, C;
+    int64_t nCB, nLB, nchunks;
+    uint64_t wait_limit_ns;
+};
+
+template <typename IO, bool GATE, int W, int LS, int S>
+struct BwdGeometry {
+    static constexpr int V = 2;
+    static constexpr int CB = 32 * V;
+    static constexpr int TT = W * LS;
+    static constexpr int NARR = GATE ? 4 : 3;   // k, v, dy (, r)
+    static constexpr int ROW = CB * static_cast<int>(sizeof(IO));
+    static constexpr uint32_t TILE = TT * ROW;
+    static constexpr uint32_t CKPT = CB * sizeof(St);
+    static constexpr uint32_t STAGE = NARR * TILE + CKPT;
+    static constexpr uint32_t SMEM = S * STAGE;
+    static constexpr int THREADS = (W + 1) * 32;
+};
+
+// Output of the current (undecayed) state and token, base 2: wkv, 1/den and
+// the scale o of num and den (num = num_hat 2^o), and e2 = 2^(u2+k2-o).
+// One ex2: exactly one of the two scale factors is 1.
+__device__ __forceinline__ void bwd_out(const St& s, float u2, float k2, float v, float& wkv, float& inv_den,
+                                        float& o, float& e2) {
+    const float uk = u2 + k2;
+    const float diff = s.p - uk;
+    const float e = ex2(-fabsf(diff));
+    float num, den;
+    if (diff >= 0.f) {
+        o = s.p;
+        e2 = e;
+        num = fmaf(e, v, s.a);
+        den = s.b + e;
+    } else {
+        o = uk;
+        e2 = 1.f;
+        num = fmaf(e, s.a, v);
+        den = fmaf(e, s.b, 1.f);
+    }
+    inv_den = rcp(den);
+    wkv = num * inv_den;
+}
+
+// State update of the forward recurrence, base 2, one ex2.
+__device__ __forceinline__ void bwd_update(St& s, float w2, float k2, float v) {
+    const float pd = s.p - w2;
+    const float diff = pd - k2;
+    const float e = ex2(-fabsf(diff));
+    if (diff >= 0.f) {
+        s.a = fmaf(e, v, s.a);
+        s.b += e;
+        s.p = pd;
+    } else {
+        s.a = fmaf(e, s.a, v);
+        s.b = fmaf(e, s.b, 1.f);
+        s.p = k2;
+    }
+}
+
+template <typename IO, bool GATE, int W, int LS, int S, int MINB>
+__global__ void __launch_bounds__(BwdGeometry<IO, GATE, W, LS, S>::THREADS, MINB)
+lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                     const __grid_constant__ CUtensorMap tdy, const __grid_constant__ CUtensorMap tr,
+                     const BwdArgs A) {
+    using G = BwdGeometry<IO, GATE, W, LS, S>;
+    constexpr int V = G::V;
+    constexpr int CB = G::CB;
+    constexpr int TT = G::TT;
+    using Raw = typename Vec<IO, V>::raw;
+    using Ld = Vec<IO, V>;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[S], empty[S];
+    __shared__ St s_fseg[W][V][32];     // forward summaries of the segments
+    __shared__ St s_rseg[W][V][32];     // reverse summaries of the segments
+    __shared__ St s_gcarry[2][V][32];   // reverse state at the end of a chunk, by chunk parity
+    // partial sums of dw, du after the last chunk, in the forward summaries' place
+    static_assert(sizeof(s_fseg) >= 2 * W * V * 32 * sizeof(float), "reduction buffer");
+    float(*s_red)[W][V][32] = reinterpret_cast<float(*)[W][V][32]>(&s_fseg[0][0][0]);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t lb = blockIdx.x;
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tk);
+        prefetch_tensormap(&tv);
+        prefetch_tensormap(&tdy);
+        if (GATE) prefetch_tensormap(&tr);
+    }
+    pdl_begin();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], W);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const int64_t nch = A.nchunks;
+    const int64_t bs = lb / A.nCB;
+    const int x0 = static_cast<int>((lb % A.nCB) * CB);
+
+    if (warp == W) {
+        // ---------------- producer: chunks from the last to the first ----------------
+        if (lane == 0) {
+            int64_t issued = 0;
+            for (int64_t it = 0; it < nch; ++it) {
+                const int s = static_cast<int>(it % S);
+                if (it >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((it / S) - 1) & 1), A.wait_limit_ns))
+                    break;
+                const int64_t chunk = nch - 1 - it;
+                unsigned char* st = smem + s * G::STAGE;
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_expect_tx(&full[s], G::NARR * G::TILE + G::CKPT);
+                const int y = static_cast<int>(chunk * TT), z = static_cast<int>(bs);
+                tma_load_3d(st, &tk, x0, y, z, &full[s]);
+                tma_load_3d(st + G::TILE, &tv, x0, y, z, &full[s]);
+                tma_load_3d(st + 2 * G::TILE, &tdy, x0, y, z, &full[s]);
+                if (GATE) tma_load_3d(st + 3 * G::TILE, &tr, x0, y, z, &full[s]);
+                bulk_load(st + G::NARR * G::TILE, A.ckpt + (chunk * A.nLB + lb) * CB, G::CKPT, &full[s]);
+                ++issued;
+            }
+            // every copy issued lands before this warp (and so the CTA) exits
+            for (int64_t q = issued > S ? issued - S : 0; q < issued; ++q)
+                mbar_wait(&full[q % S], static_cast<uint32_t>((q / S) & 1), kCopyWaitNs);
+        }
+        return;
+    }
+
+    // ---------------- compute ----------------
+    const int64_t c = x0 + lane * V;
+    const bool cvalid = c < A.C;
+    float w2[V], u2[V], lam[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        w2[j] = cvalid ? __ldg(A.w + c + j) * kLog2e : 1.f;
+        u2[j] = cvalid ? __ldg(A.u + c + j) * kLog2e : 0.f;
+        lam[j] = ex2(-w2[j]);
+    }
+    const int64_t lanes = A.B * A.C;
+    // reverse state after the sequence: dL/d(a_T, b_T) of the returned state
+    if (warp == 0) {
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            St g0 = st_identity();
+            if (A.ds_out != nullptr && cvalid) {
+                const St fin = A.ckpt[(nch * A.nLB + lb) * CB + lane * V + j];
+                const int64_t li = bs * A.C + c + j;
+                g0 = St{-fin.p, A.ds_out[li], A.ds_out[lanes + li]};
+            }
+            s_gcarry[0][j][lane] = g0;
+        }
+    }
+    float dw_acc[V] = {0.f, 0.f}, du_acc[V] = {0.f, 0.f};
+    bool ok = true;
+    for (int64_t it = 0; it < nch; ++it) {
+        const int s = static_cast<int>(it % S);
+        const int par = static_cast<int>(it & 1);
+        const int64_t chunk = nch - 1 - it;
+        const bool got = mbar_wait(&full[s], static_cast<uint32_t>((it / S) & 1), kCopyWaitNs);
+        const unsigned char* stage = smem + s * G::STAGE;
+        const int64_t t_seg = chunk * TT + warp * LS;
+        const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), A.T - t_seg)));
+        const unsigned char* srow = stage + warp * LS * G::ROW + lane * V * static_cast<int>(sizeof(IO));
+        auto row = [&](int arr, int i) -> F2 {
+            return raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + arr * G::TILE + i * G::ROW));
+        };
+        // ---- sweep 0: forward summary of the segment ----
+        St fs[V] = {st_identity(), st_identity()};
+        if (got) {
+#pragma unroll
+            for (int i = 0; i < LS; ++i) {
+                if (i < n) {
+                    const F2 kk = row(0, i), vv = row(1, i);
+                    bwd_update(fs[0], w2[0], f2lo(kk) * kLog2e, f2lo(vv));
+                    bwd_update(fs[1], w2[1], f2hi(kk) * kLog2e, f2hi(vv));
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < V; ++j) s_fseg[warp][j][lane] = fs[j];
+        }
+        if (!named_sync_and(1, W * 32, got)) {
+            ok = false;
+            break;
+        }
+        // entering forward state of the segment
+        const St* ck = reinterpret_cast<const St*>(stage + G::NARR * G::TILE) + lane * V;
+        St F[V] = {ck[0], ck[1]};
+        for (int sg = 0; sg < warp; ++sg) {
+            const int len = static_cast<int>(max(static_cast<int64_t>(0),
+                                                 min(static_cast<int64_t>(LS), A.T - (chunk * TT + sg * LS))));
+#pragma unroll
+            for (int j = 0; j < V; ++j) F[j] = st_combine(F[j], s_fseg[sg][j][lane], static_cast<float>(len) * w2[j]);
+        }
+        // ---- sweep A: outputs, c_t, dr, du, reverse summary ----
+        float co[LS][V], cn[LS][V], cd[LS][V];
+        St rs[V] = {st_identity(), st_identity()};
+        {
+            St S_[V] = {F[0], F[1]};
+            IO* drp = GATE ? static_cast<IO*>(A.dr) + (bs * A.T + t_seg) * A.C + c : nullptr;
+#pragma unroll
+            for (int i = 0; i < LS; ++i) {
+                if (i < n) {
+                    const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
+                    F2 rr = f2s(0.f);
+                    if (GATE) rr = row(3, i);
+                    float drv[V];
+#pragma unroll
+                    for (int j = 0; j < V; ++j) {
+                        const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                        const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                        const float dyj = j == 0 ? f2lo(dd) : f2hi(dd);
+                        float wkv, inv, o, e2;
+                        bwd_out(S_[j], u2[j], k2, vj, wkv, inv, o, e2);
+                        float g = 1.f;
+                        if (GATE) {
+                            g = rcp(1.f + ex2(-(j == 0 ? f2lo(rr) : f2hi(rr)) * kLog2e));
+                            drv[j] = dyj * wkv * g * (1.f - g);
+                        }
+                        const float dn = g * dyj * inv;
+                        const float dd2 = -dn * wkv;
+                        du_acc[j] = fmaf(fmaf(dn, vj, dd2), e2, du_acc[j]);
+                        co[i][j] = -o;
+                        cn[i][j] = dn;
+                        cd[i][j] = dd2;
+                        rs[j] = st_combine(rs[j], St{-o - static_cast<float>(i) * w2[j], dn, dd2}, 0.f);
+                        bwd_update(S_[j], w2[j], k2, vj);
+                    }
+                    if (GATE && cvalid) Ld::store(drp, drv);
+                }
+                if (GATE) drp += A.C;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < V; ++j) s_rseg[warp][j][lane] = rs[j];
+        named_sync(1, W * 32);
+        // ---- fold: reverse state at the end of this warp's segment ----
+        St gend[V] = {s_gcarry[par][0][lane], s_gcarry[par][1][lane]};
+        for (int sg = W - 1; sg > warp; --sg) {
+            const int len = static_cast<int>(max(static_cast<int64_t>(0),
+                                                 min(static_cast<int64_t>(LS), A.T - (chunk * TT + sg * LS))));
+#pragma unroll
+            for (int j = 0; j < V; ++j) gend[j] = st_combine(gend[j], s_rseg[sg][j][lane], static_cast<float>(len) * w2[j]);
+        }
+        // ---- sweep B: dk, dv from the reverse walk ----
+        {
+            St g[V] = {gend[0], gend[1]};
+            IO* dkp = static_cast<IO*>(A.dk) + (bs * A.T + t_seg) * A.C + c;
+            IO* dvp = static_cast<IO*>(A.dv) + (bs * A.T + t_seg) * A.C + c;
+#pragma unroll
+            for (int i = LS - 1; i >= 0; --i) {
+                if (i < n) {
+                    const F2 kk = row(0, i), vv = row(1, i);
+                    float dkv[V], dvv[V];
+#pragma unroll
+                    for (int j = 0; j < V; ++j) {
+                        const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                        const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                        const float ek = ex2(g[j].p + k2);                 // e^{k_t} gN_{t+1} / A
+                        const float e2 = ex2(u2[j] + k2 + co[i][j]);     // e^{u+k_t} dnum_t / dn
+                        dvv[j] = fmaf(cn[i][j], e2, g[j].a * ek);
+                        dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), e2, fmaf(g[j].a, vj, g[j].b) * ek);
+                        const St gn = st_combine(g[j], St{co[i][j], cn[i][j], cd[i][j]}, w2[j]);
+                        // keep the reverse state after token t for sweep C
+                        co[i][j] = g[j].p;
+                        cn[i][j] = g[j].a;
+                        cd[i][j] = g[j].b;
+                        g[j] = gn;
+                    }
+                    if (cvalid) {
+                        Ld::store(dkp + i * A.C, dkv);
+                        Ld::store(dvp + i * A.C, dvv);
+                    }
+                }
+            }
+            if (warp == 0) {
+#pragma unroll
+                for (int j = 0; j < V; ++j) s_gcarry[par ^ 1][j][lane] = g[j];
+            }
+        }
+        // ---- sweep C: dw from the forward states and the reverse states ----
+        {
+            St S_[V] = {F[0], F[1]};
+#pragma unroll
+            for (int i = 0; i < LS; ++i) {
+                if (i < n) {
+                    const F2 kk = row(0, i), vv = row(1, i);
+#pragma unroll
+                    for (int j = 0; j < V; ++j) {
+                        const float z = fmaf(cn[i][j], S_[j].a, cd[i][j] * S_[j].b) * ex2(co[i][j] + S_[j].p);
+                        dw_acc[j] += z;
+                        bwd_update(S_[j], w2[j], (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e, j == 0 ? f2lo(vv) : f2hi(vv));
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // ---- per-lane-block partial sums of dw, du; gradient of the initial state ----
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        s_red[0][warp][j][lane] = -lam[j] * dw_acc[j];
+        s_red[1][warp][j][lane] = du_acc[j];
+    }
+    named_sync(1, W * 32);
+    if (warp == 0) {
+        const int par = static_cast<int>(nch & 1);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            float sw = 0.f, su = 0.f;
+            for (int q = 0; q < W; ++q) {
+                sw += s_red[0][q][j][lane];
+                su += s_red[1][q][j][lane];
+            }
+            A.part[lb * CB + lane * V + j] = ok ? sw : __int_as_float(0x7fc00000);
+            A.part[(A.nLB + lb) * CB + lane * V + j] = ok ? su : __int_as_float(0x7fc00000);
+            if (A.ds_in != nullptr && cvalid) {
+                const int64_t li = bs * A.C + c + j;
+                const St g = s_gcarry[par][j][lane];
+                float a0 = 0.f, b0 = 0.f, p2 = kFreshP2;
+                if (A.s_in != nullptr) {
+                    a0 = A.s_in[li];
+                    b0 = A.s_in[lanes + li];
+                    p2 = A.s_in[2 * lanes + li] * kLog2e;
+                }
+                const float sc = ex2(g.p + p2);
+                const float ga = ok ? g.a * sc : __int_as_float(0x7fc00000);
+                const float gb = ok ? g.b * sc : __int_as_float(0x7fc00000);
+                A.ds_in[li] = ga;
+                A.ds_in[lanes + li] = gb;
+                A.ds_in[2 * lanes + li] = fmaf(a0, ga, b0 * gb);
+            }
+        }
+    }
+}
+
+// dw[c], du[c]: sums of the lane blocks' partials over the sequences.
+__global__ void bwd_reduce_kernel(const float* part, int64_t B, int64_t C, int64_t nCB, float* dw, float* du) {
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    const int64_t nLB = B * nCB, cb = c / 64, o = c % 64;
+    float sw = 0.f, su = 0.f;
+    for (int64_t b = 0; b < B; ++b) {
+        sw += part[(b * nCB + cb) * 64 + o];
+        su += part[(nLB + b * nCB + cb) * 64 + o];
+    }
+    dw[c] = sw;
+    du[c] = su;
+}
+
+// T == 0: the returned state is the given one, so its gradient passes
+// through; dw = du = 0 are set by the caller.
+__global__ void bwd_passthrough_kernel(int64_t lanes, const float* s_in, const float* ds_out, float* ds_in) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= lanes) return;
+    const float ga = ds_out != nullptr ? ds_out[i] : 0.f;
+    const float gb = ds_out != nullptr ? ds_out[lanes + i] : 0.f;
+    const float a0 = s_in != nullptr ? s_in[i] : 0.f, b0 = s_in != nullptr ? s_in[lanes + i] : 0.f;
+    ds_in[i] = ga;
+    ds_in[lanes + i] = gb;
+    ds_in[2 * lanes + i] = fmaf(a0, ga, b0 * gb);
+}
+
+}  // namespace wkv

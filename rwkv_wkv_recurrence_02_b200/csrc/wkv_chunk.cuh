@@ -87,6 +87,8 @@ struct ChunkArgs {
     WsHeader* hdr;      // null when nchunks == 1
     Word* aggw;         // [units][CB] chunk summaries
     Word* incw;         // [units][CB] states after each chunk
+    St* ckpt;           // lane-resident kernel only, or null: [nchunks + 1][nLB][CB] base-2 states
+                        // entering each chunk, the last one the state after the sequence
     int64_t unit_offset;
     uint64_t wait_limit_ns;
 };

@@ -147,6 +147,10 @@ __device__ __noinline__ void lane_entry_state(const ChunkArgs& A, const LaneRang
     }
 }
 
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Named barrier over `threads` threads that also ANDs a flag over them, so
 // every participating thread takes the same branch afterwards.
 __device__ __forceinline__ bool named_sync_and(int id, int threads, bool flag) {
@@ -162,7 +166,10 @@ __device__ __forceinline__ bool named_sync_and(int id, int threads, bool flag) {
     return all != 0;
 }
 
-template <typename IO, int V, bool GATE, int W, int LS, int S, int MINB = 2>
+// CKPT: checkpoint sweep for the reverse mode instead of outputs: no pass 2,
+// and the state entering every chunk (and the one after the sequence) goes
+// to A.ckpt.
+template <typename IO, int V, bool GATE, int W, int LS, int S, int MINB = 2, bool CKPT = false>
 __global__ void __launch_bounds__(LaneGeometry<IO, V, GATE, W, LS, S>::THREADS, MINB)
 lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const __grid_constant__ CUtensorMap tr, const ChunkArgs A) {
@@ -271,6 +278,11 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
                 ok = false;
                 break;
             }
+            if (CKPT && warp == 0) {
+                St* dst = A.ckpt + (chunk * A.nLB + lb) * CB + lane * V;
+#pragma unroll
+                for (int j = 0; j < V; ++j) dst[j] = s_carry[par][j][lane];
+            }
             // start state of this warp's segment: carried state, then the
             // segments before this one
             // rows of this chunk (all TT but in a sequence's last, partial chunk)
@@ -296,6 +308,11 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
                 St nx[V];
 #pragma unroll
                 for (int j = 0; j < V; ++j) nx[j] = st_combine(st[j], seg[j], static_cast<float>(cx.nvalid) * cx.w2[j]);
+                if (CKPT && chunk == A.nchunks - 1) {
+                    St* dst = A.ckpt + (A.nchunks * A.nLB + lb) * CB + lane * V;
+#pragma unroll
+                    for (int j = 0; j < V; ++j) dst[j] = nx[j];
+                }
                 if (chunk == c1 - 1) {
                     if (to_next) {
                         publish<V>(A.incw + lb * CB, nx, epoch, kKindInc, lane);
@@ -313,7 +330,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 #pragma unroll
                 for (int j = 0; j < V; ++j) s_carry[par ^ 1][j][lane] = nx[j];
             }
-            if (cx.nvalid > 0 && cx.cvalid) {
+            if (!CKPT && cx.nvalid > 0 && cx.cvalid) {
                 if (full_chunk) seg_pass2<IO, V, GATE, W, LS, true>(A, stage, cx, st);
                 else seg_pass2<IO, V, GATE, W, LS, false>(A, stage, cx, st);
             }

@@ -145,3 +145,42 @@ def test_python_front_end_refuses_cpu_tensors():
         wkv.wkv_forward(torch.ones(8), torch.zeros(8), k, k)
     with pytest.raises(ValueError):
         wkv.wkv_step(torch.ones(1, 8), torch.zeros(1, 8), k, k, torch.zeros(1, 3, 4, 8))
+
+
+def bwd(L, B=2, T=100, C=64, dt=F32, w=BASE, u=BASE + 4096, k=BASE + (1 << 30), v=BASE + (2 << 30), r=None,
+        s_in=None, dy=BASE + (8 << 30), ds_out=None, dk=BASE + (9 << 30), dv=BASE + (10 << 30), dr=None,
+        dw=BASE + 8192, du=BASE + 12288, ds_in=None, ws=BASE + (7 << 30), ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = L.wkv_backward_workspace_bytes(B, T, C, dt)
+    return L.wkv_backward(B, T, C, dt, w, u, k, v, r, s_in, dy, ds_out, dk, dv, dr, dw, du, ds_in, ws, ws_bytes,
+                          None)
+
+
+def test_backward_workspace_size(L):
+    assert L.wkv_backward_workspace_bytes(-1, 64, 128, F32) == 0
+    assert L.wkv_backward_workspace_bytes(2, 64, 128, 9) == 0
+    assert L.wkv_backward_workspace_bytes(2, 0, 128, F32) == 0
+    small = L.wkv_backward_workspace_bytes(8, 1024, 2048, F32)
+    big = L.wkv_backward_workspace_bytes(8, 4096, 2048, F32)
+    # one 12-byte checkpoint per lane per 64 tokens, plus fixed parts
+    assert 0 < small < big < 2 * 8 * 4096 * 2048
+
+
+def test_backward_validation(L):
+    assert bwd(L, dt=5) == DTYPE
+    assert bwd(L, T=-1) == SHAPE
+    assert bwd(L, C=0) == OK
+    assert bwd(L, dw=None) == NULLPTR
+    assert bwd(L, dy=None) == NULLPTR
+    assert bwd(L, dk=None) == NULLPTR
+    assert bwd(L, r=BASE + (11 << 30)) == NULLPTR                 # a gate needs dr
+    assert bwd(L, dr=BASE + (11 << 30)) == NULLPTR                # and dr needs a gate
+    assert bwd(L, dk=BASE + (9 << 30) + 4) == ALIGN               # 16-byte aligned arrays
+    assert bwd(L, C=66) == ALIGN                                  # C a multiple of 4
+    assert bwd(L, dk=BASE + (1 << 30)) == ALIAS                   # dk over k
+    assert bwd(L, dv=BASE + (9 << 30) + 1024) == ALIAS            # dv inside dk
+    assert bwd(L, du=BASE + 8192 + 16) == ALIAS                   # du inside dw
+    assert bwd(L, ds_in=BASE + (8 << 30), s_in=BASE + (12 << 30)) == ALIAS   # dstate_in over dy
+    assert bwd(L, ws=None) == WORKSPACE
+    assert bwd(L, ws_bytes=L.wkv_backward_workspace_bytes(2, 100, 64, F32) - 1) == WORKSPACE
+    assert bwd(L, ws=BASE + (7 << 30) + 16) == ALIGN
