@@ -34,6 +34,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "WKV elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
+METRIC_BWD = "WKV backward elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
 UNIT = "elements/s"
 SPEC_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
@@ -68,6 +69,19 @@ def algorithmic_bytes(wl, B, T, C, layers=0) -> int:
     io = n * eb * (3 if wl.gate else 2) + n * eb
     state = B * C * 12 * (2 if wl.random_state or wl.chunk else 1)
     return io + state + C * 8
+
+
+def algorithmic_bytes_backward(wl, B, T, C) -> int:
+    """Bytes one backward call must move at minimum: k, v, dy (and r) read
+    once, dk, dv (and dr) written once, the initial state and dL/d(a, b) of
+    the returned state read, dL/d(initial state) written, w and u read, dw and
+    du written."""
+    eb = wl.elem_bytes
+    n = B * T * C
+    narr = 3 if wl.gate else 2
+    io = n * eb * ((narr + 1) + narr)
+    state = B * C * (12 * (1 if wl.random_state or wl.chunk else 0) + 8 + 12)
+    return io + state + C * 16
 
 
 def max_over_ranks(value: float, dist=None) -> float:
@@ -234,9 +248,49 @@ class DecodeCase:
                      None if self.r is None else self.r[a:a + L], y=self.y)
 
 
-def make_case(name, device, seed_base):
+class BackwardCase:
+    """Backward: one wkv_backward call per step on the workload's shape, inputs
+    (forward inputs, dy, dL/d(returned state)) rotating over sets larger than
+    L2, outputs preallocated."""
+
+    def __init__(self, wl, device, seed_base):
+        import torch
+        from rwkv_wkv_recurrence_02_b200 import inputs as I
+        self.wl = wl
+        T = wl.chunk or wl.T
+        self.B, self.T, self.C = wl.B, T, wl.C
+        one = algorithmic_bytes_backward(wl, self.B, self.T, self.C)
+        nsets = 2
+        while nsets * one < 2 * L2_BYTES:
+            nsets += 1
+        self.sets = []
+        for i in range(nsets):
+            d = I.make_forward_inputs(wl, T=T, device=device, seed_offset=seed_base + i)
+            g = torch.Generator(device="cpu").manual_seed(9000 + seed_base + i)
+            d["dy"] = torch.randn(self.B, T, self.C, generator=g).to(wl.torch_dtype).to(device)
+            d["ds"] = torch.randn(3, self.B, self.C, generator=g).to(device)
+            self.sets.append(d)
+        mk = lambda: torch.empty((self.B, T, self.C), dtype=wl.torch_dtype, device=device)
+        self.out = [dict(dk=mk(), dv=mk(), dr=mk() if wl.gate else None,
+                         dw=torch.empty(self.C, device=device), du=torch.empty(self.C, device=device),
+                         dstate_in=torch.empty((3, self.B, self.C), device=device)) for _ in range(2)]
+        self.elements = self.B * T * self.C
+        self.bytes = algorithmic_bytes_backward(wl, self.B, T, self.C)
+        self.launches_per_step = 3   # checkpoint sweep, reverse walk, dw/du reduction
+
+    def step(self, i, wkv, ws):
+        d = self.sets[i % len(self.sets)]
+        wkv.wkv_backward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"], dy=d["dy"], dstate_out=d["ds"],
+                         workspace=ws, **self.out[i % 2])
+
+
+def make_case(name, device, seed_base, op="forward"):
     from rwkv_wkv_recurrence_02_b200 import inputs as I
     wl = I.WORKLOADS[name]
+    if op == "backward":
+        if wl.layers:
+            raise SystemExit("--op backward takes the forward workloads (the decode step has no reverse mode)")
+        return BackwardCase(wl, device, seed_base)
     if wl.layers:
         return DecodeCase(wl, device, seed_base)
     return ForwardCase(wl, device, seed_base)
@@ -246,6 +300,8 @@ def e2e_measure(case, wkv, ws, steps, warmup, stream):
     """Same metric through the public API with host buffers: each step copies
     its inputs from pinned host memory and reads the result back."""
     import torch
+    if isinstance(case, BackwardCase):
+        return e2e_measure_backward(case, wkv, ws, steps, warmup, stream)
     if not isinstance(case, ForwardCase):
         return None
     d = case.sets[0]
@@ -276,6 +332,72 @@ def e2e_measure(case, wkv, ws, steps, warmup, stream):
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) / 1e3
     return {"seconds": sec, "steps": steps, "h2d": h2d, "d2h": d2h}
+
+
+def e2e_measure_backward(case, wkv, ws, steps, warmup, stream):
+    """The backward through the public API with host buffers: every step copies
+    k, v, r, dy, the state and dL/d(returned state) from pinned host memory and
+    reads every gradient back."""
+    import torch
+    d = case.sets[0]
+    names = ("w", "u", "k", "v", "r", "state", "dy", "ds")
+    host = {n: (None if d[n] is None else d[n].to("cpu").pin_memory()) for n in names}
+    dev = {n: (None if v is None else torch.empty_like(v, device=d["k"].device)) for n, v in host.items()}
+    outs = case.out[0]
+    back = {n: (None if v is None else torch.empty(v.shape, dtype=v.dtype).pin_memory()) for n, v in outs.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for v in back.values() if v is not None)
+
+    def one():
+        for n, v in host.items():
+            if v is not None:
+                dev[n].copy_(v, non_blocking=True)
+        wkv.wkv_backward(dev["w"], dev["u"], dev["k"], dev["v"], dev["r"], dev["state"], dy=dev["dy"],
+                         dstate_out=dev["ds"], workspace=ws, **outs)
+        for n, v in back.items():
+            if v is not None:
+                v.copy_(outs[n], non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h}
+
+
+def cpu_baseline_backward(workload: str, budget_s: float, max_reps: int = 1000):
+    """The oracle's reverse mode as it stands, on this host's cores, over a
+    lane sample of the workload repeated for about `budget_s`."""
+    import oracle
+    from rwkv_wkv_recurrence_02_b200 import inputs as I
+    import numpy as np
+    wl = I.WORKLOADS[workload]
+    T, B, C = wl.chunk or wl.T, wl.B, wl.C
+    cap = max(1, int(1e7 // T))
+    csub = C if B * C <= cap else max(1, cap // B)
+    d = I.make_forward_inputs(wl, T=T, C=csub)
+    f = lambda x: None if x is None else x.float().numpy()
+    st = None if d["state"] is None else d["state"].double().numpy()
+    g = np.random.default_rng(0)
+    dy = g.normal(0, 1, (B, T, csub))
+    ds = g.normal(0, 1, (3, B, csub))
+    run = lambda: oracle.wkv_backward(f(d["w"]), f(d["u"]), f(d["k"]), f(d["v"]), f(d["r"]), st, dy, ds)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        run()
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= max_reps:
+            break
+    sec = time.perf_counter() - t0
+    sample = f"lane sample B={B}, T={T}, C={csub} of {C}" if csub < C else f"full step B={B}, T={T}, C={C}"
+    return {"value": B * T * csub * reps / sec, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{sample}, repeated {reps}x over {sec:.1f} s"}
 
 
 def cpu_baseline_sample(workload: str, budget_s: float, max_reps: int = 1000):
@@ -353,7 +475,7 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     wkv.lib()
-    case = make_case(args.workload, device, rank_seed(0, rank))
+    case = make_case(args.workload, device, rank_seed(0, rank), args.op)
     ws = wkv.Workspace(device)
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
@@ -381,21 +503,27 @@ def run_ours(args):
     if ws.buf is not None and ws.status() != 0:
         raise SystemExit("the GPU reported a cross-block wait timeout during the benchmark")
     value = whole_job_rate(case.elements, world, args.steps, sec)
-    per_launch = sec / args.steps / case.launches_per_step
+    # the roofline of a multi-kernel step (the backward) is taken over the whole
+    # step: its algorithmic bytes over the step's time, a lower bound on the
+    # dominant kernel's fraction
+    per_launch = sec / args.steps / (1 if isinstance(case, BackwardCase) else case.launches_per_step)
     peak, peak_kind = load_peaks()
     achieved = case.bytes / per_launch / 1e9
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if args.op == "backward" else METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "io_dtype": case.wl.dtype,
         "data": "synthetic (seeded; distributions of the workload definition)",
-        "config": config_of(case, args.workload, world),
+        "config": dict(config_of(case, args.workload, world), **({"op": "backward"} if args.op == "backward" else {})),
         "hbm_gbs": achieved, "hbm_pct_of_spec_8tbs": 100.0 * achieved / SPEC_HBM_GBS,
         "hbm_pct_of_measured": 100.0 * achieved / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "scope": ("whole step: checkpoint sweep + reverse walk + dw/du reduction"
+                               if isinstance(case, BackwardCase) else "the step's one kernel"),
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": case.bytes,
-                     "traffic": load_traffic(args.workload)},
+                     "traffic": load_traffic(args.workload + ("_backward" if args.op == "backward" else ""))},
         "gpu_launches": args.steps * case.launches_per_step,
         "clocks": clocks.summary(t0, t1),
     }
@@ -407,7 +535,8 @@ def run_ours(args):
                           "unit": UNIT, "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                           "steps": e["steps"], "path": "pinned host -> wkv_forward (C ABI) -> pinned host"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline_sample(args.workload, args.cpu_seconds)
+        out["cpu_baseline"] = (cpu_baseline_backward(args.workload, args.cpu_seconds) if args.op == "backward"
+                               else cpu_baseline_sample(args.workload, args.cpu_seconds))
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -430,29 +559,39 @@ def run_reference(args):
     if wl.layers:
         raise SystemExit("--impl reference times the forward workloads")
     T, B, C = (wl.chunk or wl.T), wl.B, wl.C
+    backward = args.op == "backward"
+
+    def call(d, n):
+        st = None if d["state"] is None else d["state"].double().numpy()
+        a = (f(d["w"]), f(d["u"]), f(d["k"]), f(d["v"]), f(d["r"]), st)
+        if not backward:
+            return lambda: oracle.wkv_forward(*a)
+        g = np.random.default_rng(1)
+        dy, ds = g.normal(0, 1, (1, T, n)), g.normal(0, 1, (3, 1, n))
+        return lambda: oracle.wkv_backward(*a, dy, ds)
+
     # calibrate: seconds per lane (all T tokens) with all cores busy
     cal = I.make_forward_inputs(wl, B=1, T=T, C=min(C, 256))
+    run = call(cal, min(C, 256))
     t0 = time.perf_counter()
-    oracle.wkv_forward(f(cal["w"]), f(cal["u"]), f(cal["k"]), f(cal["v"]), f(cal["r"]),
-                       None if cal["state"] is None else cal["state"].double().numpy())
+    run()
     per_lane = (time.perf_counter() - t0) / min(C, 256)
     lanes = int(max(1, min(B * C, budget / max(1, args.steps + args.warmup) / per_lane)))
     csub = max(1, min(C, lanes))
     d = I.make_forward_inputs(wl, B=1, T=T, C=csub)
-    st = None if d["state"] is None else d["state"].double().numpy()
-    args_np = (f(d["w"]), f(d["u"]), f(d["k"]), f(d["v"]), f(d["r"]), st)
+    run = call(d, csub)
     for _ in range(args.warmup):
-        oracle.wkv_forward(*args_np)
+        run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.wkv_forward(*args_np)
+        run()
     sec = time.perf_counter() - t0
     elems = T * csub
     value = elems * args.steps / sec
     sample = f"lane sample B=1, T={T}, C={csub} of the workload's B={B}, C={C} per step"
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
+        "metric": METRIC_BWD if backward else METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": args.workload, "B": B, "T": T, "C": C, "io_dtype": wl.dtype, "gate": wl.gate},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
@@ -470,6 +609,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="layer_1b5",
                    choices=["tiny", "layer_1b5", "layer_14b", "stream_1m", "decode"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--op", default="forward", choices=["forward", "backward"],
+                   help="forward (the headline) or the reverse mode on the same workload")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-budget-s", type=float, default=90.0)

@@ -802,19 +802,34 @@ BwdLayout bwd_layout(int64_t B, int64_t T, int64_t C) {
     return L;
 }
 
-template <typename IO, bool GATE, int S, int MINB>
-int launch_backward(const wkv::BwdArgs& a, int dtype, cudaStream_t st) {
+// Reverse walk: CTAs take equal shares of the lane-major (lane block, chunk)
+// order like the lane-resident forward kernel; grid = min(lane blocks,
+// resident capacity), with one reverse state handed between neighbours
+// through the workspace when a lane block is split.
+template <typename IO, bool GATE, int S, int MAXREG>
+int launch_backward(wkv::BwdArgs a, int dtype, void* workspace, cudaStream_t st) {
     using G = wkv::BwdGeometry<IO, GATE, kBwdW, kBwdLS, S>;
-    auto kern = wkv::lane_backward_kernel<IO, GATE, kBwdW, kBwdLS, S, MINB>;
-    static bool ready[kMaxDevices] = {false};
+    auto kern = wkv::lane_backward_kernel<IO, GATE, kBwdW, kBwdLS, S, MAXREG>;
+    static int capacity[kMaxDevices] = {0};
     int dev = 0;
     int rc = record_cuda(cudaGetDevice(&dev));
     if (rc != WKV_OK) return rc;
     if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
-    if (!ready[dev]) {
+    if (capacity[dev] == 0) {
         rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
         if (rc != WKV_OK) return rc;
-        ready[dev] = true;
+        int per_sm = 0;
+        rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+    }
+    const int64_t grid = a.nLB < capacity[dev] ? a.nLB : capacity[dev];
+    if (grid < a.nLB && a.nchunks > 1) {
+        a.hdr = reinterpret_cast<wkv::WsHeader*>(workspace);
+        a.incw = reinterpret_cast<wkv::Word*>(static_cast<char*>(workspace) + 256);
+    } else {
+        a.hdr = nullptr;
+        a.incw = nullptr;
     }
     CUtensorMap tk, tv, tdy, tr;
     if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
@@ -827,7 +842,7 @@ int launch_backward(const wkv::BwdArgs& a, int dtype, cudaStream_t st) {
         tr = tk;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(a.nLB));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(G::THREADS);
     cfg.dynamicSmemBytes = G::SMEM;
     cfg.stream = st;
@@ -845,11 +860,16 @@ int run_backward(const wkv::BwdArgs& b, wkv::ChunkArgs f, int dtype, void* ws, s
     constexpr int SF = sizeof(IO) == 4 ? 2 : 3;
     int rc = launch_lane<IO, false, SF, true>(f, dtype, ws, ws_bytes, st);
     if (rc != WKV_OK) return rc;
-    // stages: three with one CTA per SM for fp32, two with two CTAs for bf16
+    rc = record_cuda(cudaMemsetAsync(b.part, 0, 2 * size_t(b.nLB) * 64 * sizeof(float), st));
+    if (rc != WKV_OK) return rc;
+    // fp32: three stages, one CTA (9 warps) per SM, up to 224 registers;
+    // bf16: two stages, two CTAs per SM, 112 registers
     if constexpr (sizeof(IO) == 4)
-        return b.r != nullptr ? launch_backward<IO, true, 3, 1>(b, dtype, st) : launch_backward<IO, false, 3, 1>(b, dtype, st);
+        return b.r != nullptr ? launch_backward<IO, true, 3, 224>(b, dtype, ws, st)
+                              : launch_backward<IO, false, 3, 224>(b, dtype, ws, st);
     else
-        return b.r != nullptr ? launch_backward<IO, true, 2, 2>(b, dtype, st) : launch_backward<IO, false, 2, 2>(b, dtype, st);
+        return b.r != nullptr ? launch_backward<IO, true, 2, 112>(b, dtype, ws, st)
+                              : launch_backward<IO, false, 2, 112>(b, dtype, ws, st);
 }
 
 }  // namespace

@@ -68,7 +68,9 @@ struct BwdArgs {
     void* dr;
     float* ds_in;
     const St* ckpt;     // [nchunks + 1][nLB][CB], see ChunkArgs::ckpt
-    float* part;        // [2][nLB][CB]: dw, du of each lane block
+    float* part;        // [2][nLB][CB]: dw, du of each lane block (zeroed by the caller)
+    WsHeader* hdr;      // null when every CTA owns whole lane blocks
+    Word* incw;         // [nLB][CB] reverse states handed between neighbouring CTAs
     int64_t B, T, C;
     int64_t nCB, nLB, nchunks;
     uint64_t wait_limit_ns;
@@ -128,8 +130,55 @@ __device__ __forceinline__ void bwd_update(St& s, float w2, float k2, float v) {
     }
 }
 
-template <typename IO, bool GATE, int W, int LS, int S, int MINB>
-__global__ void __launch_bounds__(BwdGeometry<IO, GATE, W, LS, S>::THREADS, MINB)
+__device__ __forceinline__ void finish_bwd_launch(const BwdArgs& A, uint32_t ctas) {
+    const uint32_t before = atomicAdd(&A.hdr->done, 1u);
+    if (before == ctas - 1u) {
+        A.hdr->done = 0u;
+        A.hdr->ticket = 0u;
+        __threadfence();
+        atomicAdd(&A.hdr->epoch, 1u);
+    }
+}
+
+// Reverse state handed over by the CTA that walked the later chunks of lane
+// block lb (one 16-byte word per channel; bounded wait, NaN on expiry).
+template <int V>
+__device__ __noinline__ void bwd_wait_carry(const BwdArgs& A, int64_t lb, uint32_t epoch, St* out) {
+    constexpr int CB = 32 * V;
+    const int lane = threadIdx.x & 31;
+    const Word* src = A.incw + lb * CB + lane * V;
+    const uint64_t t0 = global_ns();
+    unsigned sleep_ns = 32;
+    for (;;) {
+        Word wv[V];
+        bool mine = true;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            wv[j] = ld_word(src + j);
+            mine = mine && wv[j].tag == word_tag(epoch, kKindInc);
+        }
+        if (__all_sync(0xffffffffu, mine)) {
+#pragma unroll
+            for (int j = 0; j < V; ++j) out[j] = word_state(wv[j]);
+            return;
+        }
+        if (global_ns() - t0 > A.wait_limit_ns) {
+            if (lane == 0) {
+                atomicOr(&A.hdr->error, kErrTimeout);
+                atomicExch(&A.hdr->err_unit, static_cast<uint32_t>(lb));
+            }
+            const float nan = __int_as_float(0x7fc00000);
+#pragma unroll
+            for (int j = 0; j < V; ++j) out[j] = St{nan, nan, nan};
+            return;
+        }
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 256) sleep_ns <<= 1;
+    }
+}
+
+template <typename IO, bool GATE, int W, int LS, int S, int MAXREG>
+__global__ void __launch_bounds__(BwdGeometry<IO, GATE, W, LS, S>::THREADS) __maxnreg__(MAXREG)
 lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                      const __grid_constant__ CUtensorMap tdy, const __grid_constant__ CUtensorMap tr,
                      const BwdArgs A) {
@@ -144,11 +193,10 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
     __shared__ St s_fseg[W][V][32];     // forward summaries of the segments
     __shared__ St s_rseg[W][V][32];     // reverse summaries of the segments
     __shared__ St s_gcarry[2][V][32];   // reverse state at the end of a chunk, by chunk parity
-    // partial sums of dw, du after the last chunk, in the forward summaries' place
-    static_assert(sizeof(s_fseg) >= 2 * W * V * 32 * sizeof(float), "reduction buffer");
-    float(*s_red)[W][V][32] = reinterpret_cast<float(*)[W][V][32]>(&s_fseg[0][0][0]);
+    __shared__ float s_red[2][W][V][32];
+    __shared__ LaneRange s_range;       // this CTA's share of the lane-major chunk order
+    __shared__ uint32_t s_epoch;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t lb = blockIdx.x;
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tk);
         prefetch_tensormap(&tv);
@@ -157,6 +205,8 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
     }
     pdl_begin();
     if (threadIdx.x == 0) {
+        s_range.init(A.nLB, A.nchunks, blockIdx.x, gridDim.x);
+        s_epoch = A.hdr != nullptr ? ld_relaxed_u32(&A.hdr->epoch) : 0u;
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], W);
@@ -164,29 +214,38 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+    const LaneRange& R = s_range;
+    const uint32_t epoch = s_epoch;
     const int64_t nch = A.nchunks;
-    const int64_t bs = lb / A.nCB;
-    const int x0 = static_cast<int>((lb % A.nCB) * CB);
 
     if (warp == W) {
-        // ---------------- producer: chunks from the last to the first ----------------
+        // ---------------- producer: each item's chunks from the last to the first ----------------
         if (lane == 0) {
-            int64_t issued = 0;
-            for (int64_t it = 0; it < nch; ++it) {
-                const int s = static_cast<int>(it % S);
-                if (it >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(((it / S) - 1) & 1), A.wait_limit_ns))
-                    break;
-                const int64_t chunk = nch - 1 - it;
-                unsigned char* st = smem + s * G::STAGE;
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_expect_tx(&full[s], G::NARR * G::TILE + G::CKPT);
-                const int y = static_cast<int>(chunk * TT), z = static_cast<int>(bs);
-                tma_load_3d(st, &tk, x0, y, z, &full[s]);
-                tma_load_3d(st + G::TILE, &tv, x0, y, z, &full[s]);
-                tma_load_3d(st + 2 * G::TILE, &tdy, x0, y, z, &full[s]);
-                if (GATE) tma_load_3d(st + 3 * G::TILE, &tr, x0, y, z, &full[s]);
-                bulk_load(st + G::NARR * G::TILE, A.ckpt + (chunk * A.nLB + lb) * CB, G::CKPT, &full[s]);
-                ++issued;
+            int64_t it = 0, issued = 0;
+            bool stop = false;
+            for (int item = 0; item < R.count && !stop; ++item) {
+                int64_t lb, c0, c1;
+                bool to_prev, from_next;
+                R.item_back(item, lb, c0, c1, to_prev, from_next);
+                const int x0 = static_cast<int>((lb % A.nCB) * CB), z = static_cast<int>(lb / A.nCB);
+                for (int64_t chunk = c1 - 1; chunk >= c0; --chunk, ++it) {
+                    const int s = static_cast<int>(it % S);
+                    if (it >= S &&
+                        !mbar_wait(&empty[s], static_cast<uint32_t>(((it / S) - 1) & 1), A.wait_limit_ns)) {
+                        stop = true;
+                        break;
+                    }
+                    unsigned char* st = smem + s * G::STAGE;
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_expect_tx(&full[s], G::NARR * G::TILE + G::CKPT);
+                    const int y = static_cast<int>(chunk * TT);
+                    tma_load_3d(st, &tk, x0, y, z, &full[s]);
+                    tma_load_3d(st + G::TILE, &tv, x0, y, z, &full[s]);
+                    tma_load_3d(st + 2 * G::TILE, &tdy, x0, y, z, &full[s]);
+                    if (GATE) tma_load_3d(st + 3 * G::TILE, &tr, x0, y, z, &full[s]);
+                    bulk_load(st + G::NARR * G::TILE, A.ckpt + (chunk * A.nLB + lb) * CB, G::CKPT, &full[s]);
+                    ++issued;
+                }
             }
             // every copy issued lands before this warp (and so the CTA) exits
             for (int64_t q = issued > S ? issued - S : 0; q < issued; ++q)
@@ -196,211 +255,230 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
     }
 
     // ---------------- compute ----------------
-    const int64_t c = x0 + lane * V;
-    const bool cvalid = c < A.C;
-    float w2[V], u2[V], lam[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-        w2[j] = cvalid ? __ldg(A.w + c + j) * kLog2e : 1.f;
-        u2[j] = cvalid ? __ldg(A.u + c + j) * kLog2e : 0.f;
-        lam[j] = ex2(-w2[j]);
-    }
     const int64_t lanes = A.B * A.C;
-    // reverse state after the sequence: dL/d(a_T, b_T) of the returned state
-    if (warp == 0) {
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            St g0 = st_identity();
-            if (A.ds_out != nullptr && cvalid) {
-                const St fin = A.ckpt[(nch * A.nLB + lb) * CB + lane * V + j];
-                const int64_t li = bs * A.C + c + j;
-                g0 = St{-fin.p, A.ds_out[li], A.ds_out[lanes + li]};
-            }
-            s_gcarry[0][j][lane] = g0;
-        }
-    }
-    float dw_acc[V] = {0.f, 0.f}, du_acc[V] = {0.f, 0.f};
+    int64_t it = 0;
     bool ok = true;
-    for (int64_t it = 0; it < nch; ++it) {
-        const int s = static_cast<int>(it % S);
-        const int par = static_cast<int>(it & 1);
-        const int64_t chunk = nch - 1 - it;
-        const bool got = mbar_wait(&full[s], static_cast<uint32_t>((it / S) & 1), kCopyWaitNs);
-        const unsigned char* stage = smem + s * G::STAGE;
-        const int64_t t_seg = chunk * TT + warp * LS;
-        const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), A.T - t_seg)));
-        const unsigned char* srow = stage + warp * LS * G::ROW + lane * V * static_cast<int>(sizeof(IO));
-        auto row = [&](int arr, int i) -> F2 {
-            return raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + arr * G::TILE + i * G::ROW));
-        };
-        // ---- sweep 0: forward summary of the segment ----
-        St fs[V] = {st_identity(), st_identity()};
-        if (got) {
-#pragma unroll
-            for (int i = 0; i < LS; ++i) {
-                if (i < n) {
-                    const F2 kk = row(0, i), vv = row(1, i);
-                    bwd_update(fs[0], w2[0], f2lo(kk) * kLog2e, f2lo(vv));
-                    bwd_update(fs[1], w2[1], f2hi(kk) * kLog2e, f2hi(vv));
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < V; ++j) s_fseg[warp][j][lane] = fs[j];
-        }
-        if (!named_sync_and(1, W * 32, got)) {
-            ok = false;
-            break;
-        }
-        // entering forward state of the segment
-        const St* ck = reinterpret_cast<const St*>(stage + G::NARR * G::TILE) + lane * V;
-        St F[V] = {ck[0], ck[1]};
-        for (int sg = 0; sg < warp; ++sg) {
-            const int len = static_cast<int>(max(static_cast<int64_t>(0),
-                                                 min(static_cast<int64_t>(LS), A.T - (chunk * TT + sg * LS))));
-#pragma unroll
-            for (int j = 0; j < V; ++j) F[j] = st_combine(F[j], s_fseg[sg][j][lane], static_cast<float>(len) * w2[j]);
-        }
-        // ---- sweep A: outputs, c_t, dr, du, reverse summary ----
-        float co[LS][V], cn[LS][V], cd[LS][V];
-        St rs[V] = {st_identity(), st_identity()};
-        {
-            St S_[V] = {F[0], F[1]};
-            IO* drp = GATE ? static_cast<IO*>(A.dr) + (bs * A.T + t_seg) * A.C + c : nullptr;
-#pragma unroll
-            for (int i = 0; i < LS; ++i) {
-                if (i < n) {
-                    const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
-                    F2 rr = f2s(0.f);
-                    if (GATE) rr = row(3, i);
-                    float drv[V];
-#pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                        const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
-                        const float dyj = j == 0 ? f2lo(dd) : f2hi(dd);
-                        float wkv, inv, o, e2;
-                        bwd_out(S_[j], u2[j], k2, vj, wkv, inv, o, e2);
-                        float g = 1.f;
-                        if (GATE) {
-                            g = rcp(1.f + ex2(-(j == 0 ? f2lo(rr) : f2hi(rr)) * kLog2e));
-                            drv[j] = dyj * wkv * g * (1.f - g);
-                        }
-                        const float dn = g * dyj * inv;
-                        const float dd2 = -dn * wkv;
-                        du_acc[j] = fmaf(fmaf(dn, vj, dd2), e2, du_acc[j]);
-                        co[i][j] = -o;
-                        cn[i][j] = dn;
-                        cd[i][j] = dd2;
-                        rs[j] = st_combine(rs[j], St{-o - static_cast<float>(i) * w2[j], dn, dd2}, 0.f);
-                        bwd_update(S_[j], w2[j], k2, vj);
-                    }
-                    if (GATE && cvalid) Ld::store(drp, drv);
-                }
-                if (GATE) drp += A.C;
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < V; ++j) s_rseg[warp][j][lane] = rs[j];
-        named_sync(1, W * 32);
-        // ---- fold: reverse state at the end of this warp's segment ----
-        St gend[V] = {s_gcarry[par][0][lane], s_gcarry[par][1][lane]};
-        for (int sg = W - 1; sg > warp; --sg) {
-            const int len = static_cast<int>(max(static_cast<int64_t>(0),
-                                                 min(static_cast<int64_t>(LS), A.T - (chunk * TT + sg * LS))));
-#pragma unroll
-            for (int j = 0; j < V; ++j) gend[j] = st_combine(gend[j], s_rseg[sg][j][lane], static_cast<float>(len) * w2[j]);
-        }
-        // ---- sweep B: dk, dv from the reverse walk ----
-        {
-            St g[V] = {gend[0], gend[1]};
-            IO* dkp = static_cast<IO*>(A.dk) + (bs * A.T + t_seg) * A.C + c;
-            IO* dvp = static_cast<IO*>(A.dv) + (bs * A.T + t_seg) * A.C + c;
-#pragma unroll
-            for (int i = LS - 1; i >= 0; --i) {
-                if (i < n) {
-                    const F2 kk = row(0, i), vv = row(1, i);
-                    float dkv[V], dvv[V];
-#pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                        const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
-                        const float ek = ex2(g[j].p + k2);                 // e^{k_t} gN_{t+1} / A
-                        const float e2 = ex2(u2[j] + k2 + co[i][j]);     // e^{u+k_t} dnum_t / dn
-                        dvv[j] = fmaf(cn[i][j], e2, g[j].a * ek);
-                        dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), e2, fmaf(g[j].a, vj, g[j].b) * ek);
-                        const St gn = st_combine(g[j], St{co[i][j], cn[i][j], cd[i][j]}, w2[j]);
-                        // keep the reverse state after token t for sweep C
-                        co[i][j] = g[j].p;
-                        cn[i][j] = g[j].a;
-                        cd[i][j] = g[j].b;
-                        g[j] = gn;
-                    }
-                    if (cvalid) {
-                        Ld::store(dkp + i * A.C, dkv);
-                        Ld::store(dvp + i * A.C, dvv);
-                    }
-                }
-            }
-            if (warp == 0) {
-#pragma unroll
-                for (int j = 0; j < V; ++j) s_gcarry[par ^ 1][j][lane] = g[j];
-            }
-        }
-        // ---- sweep C: dw from the forward states and the reverse states ----
-        {
-            St S_[V] = {F[0], F[1]};
-#pragma unroll
-            for (int i = 0; i < LS; ++i) {
-                if (i < n) {
-                    const F2 kk = row(0, i), vv = row(1, i);
-#pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        const float z = fmaf(cn[i][j], S_[j].a, cd[i][j] * S_[j].b) * ex2(co[i][j] + S_[j].p);
-                        dw_acc[j] += z;
-                        bwd_update(S_[j], w2[j], (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e, j == 0 ? f2lo(vv) : f2hi(vv));
-                    }
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    // ---- per-lane-block partial sums of dw, du; gradient of the initial state ----
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-        s_red[0][warp][j][lane] = -lam[j] * dw_acc[j];
-        s_red[1][warp][j][lane] = du_acc[j];
-    }
-    named_sync(1, W * 32);
-    if (warp == 0) {
-        const int par = static_cast<int>(nch & 1);
+    for (int item = 0; item < R.count && ok; ++item) {
+        int64_t lb, c0, c1;
+        bool to_prev, from_next;
+        R.item_back(item, lb, c0, c1, to_prev, from_next);
+        const int64_t bs = lb / A.nCB;
+        const int64_t c = (lb % A.nCB) * CB + lane * V;
+        const bool cvalid = c < A.C;
+        float w2[V], u2[V], lam[V];
 #pragma unroll
         for (int j = 0; j < V; ++j) {
-            float sw = 0.f, su = 0.f;
-            for (int q = 0; q < W; ++q) {
-                sw += s_red[0][q][j][lane];
-                su += s_red[1][q][j][lane];
-            }
-            A.part[lb * CB + lane * V + j] = ok ? sw : __int_as_float(0x7fc00000);
-            A.part[(A.nLB + lb) * CB + lane * V + j] = ok ? su : __int_as_float(0x7fc00000);
-            if (A.ds_in != nullptr && cvalid) {
-                const int64_t li = bs * A.C + c + j;
-                const St g = s_gcarry[par][j][lane];
-                float a0 = 0.f, b0 = 0.f, p2 = kFreshP2;
-                if (A.s_in != nullptr) {
-                    a0 = A.s_in[li];
-                    b0 = A.s_in[lanes + li];
-                    p2 = A.s_in[2 * lanes + li] * kLog2e;
+            w2[j] = cvalid ? __ldg(A.w + c + j) * kLog2e : 1.f;
+            u2[j] = cvalid ? __ldg(A.u + c + j) * kLog2e : 0.f;
+            lam[j] = ex2(-w2[j]);
+        }
+        // reverse state after the item's last chunk
+        if (warp == 0) {
+            St g0[V] = {st_identity(), st_identity()};
+            if (from_next) {
+                bwd_wait_carry<V>(A, lb, epoch, g0);
+            } else if (A.ds_out != nullptr && cvalid) {
+                // the end of the sequence: dL/d(a_T, b_T) of the returned state
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    const St fin = A.ckpt[(nch * A.nLB + lb) * CB + lane * V + j];
+                    const int64_t li = bs * A.C + c + j;
+                    g0[j] = St{-fin.p, A.ds_out[li], A.ds_out[lanes + li]};
                 }
-                const float sc = ex2(g.p + p2);
-                const float ga = ok ? g.a * sc : __int_as_float(0x7fc00000);
-                const float gb = ok ? g.b * sc : __int_as_float(0x7fc00000);
-                A.ds_in[li] = ga;
-                A.ds_in[lanes + li] = gb;
-                A.ds_in[2 * lanes + li] = fmaf(a0, ga, b0 * gb);
+            }
+#pragma unroll
+            for (int j = 0; j < V; ++j) s_gcarry[it & 1][j][lane] = g0[j];
+        }
+        float dw_acc[V] = {0.f, 0.f}, du_acc[V] = {0.f, 0.f};
+        for (int64_t chunk = c1 - 1; chunk >= c0; --chunk, ++it) {
+            const int s = static_cast<int>(it % S);
+            const int par = static_cast<int>(it & 1);
+            const bool got = mbar_wait(&full[s], static_cast<uint32_t>((it / S) & 1), kCopyWaitNs);
+            const unsigned char* stage = smem + s * G::STAGE;
+            const int64_t t_seg = chunk * TT + warp * LS;
+            const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), A.T - t_seg)));
+            const unsigned char* srow = stage + warp * LS * G::ROW + lane * V * static_cast<int>(sizeof(IO));
+            auto row = [&](int arr, int i) -> F2 {
+                return raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + arr * G::TILE + i * G::ROW));
+            };
+            // ---- sweep 0: forward summary of the segment ----
+            St fs[V] = {st_identity(), st_identity()};
+            if (got) {
+#pragma unroll
+                for (int i = 0; i < LS; ++i) {
+                    if (i < n) {
+                        const F2 kk = row(0, i), vv = row(1, i);
+                        bwd_update(fs[0], w2[0], f2lo(kk) * kLog2e, f2lo(vv));
+                        bwd_update(fs[1], w2[1], f2hi(kk) * kLog2e, f2hi(vv));
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < V; ++j) s_fseg[warp][j][lane] = fs[j];
+            }
+            // a copy that did not land stops every compute warp together
+            if (!named_sync_and(1, W * 32, got)) {
+                if (threadIdx.x == 0 && A.hdr != nullptr) atomicOr(&A.hdr->error, kErrTimeout);
+                ok = false;
+                break;
+            }
+            // entering forward state of the segment
+            const St* ck = reinterpret_cast<const St*>(stage + G::NARR * G::TILE) + lane * V;
+            St F[V] = {ck[0], ck[1]};
+            for (int sg = 0; sg < warp; ++sg) {
+                const int len = static_cast<int>(max(static_cast<int64_t>(0),
+                                                     min(static_cast<int64_t>(LS), A.T - (chunk * TT + sg * LS))));
+#pragma unroll
+                for (int j = 0; j < V; ++j) F[j] = st_combine(F[j], s_fseg[sg][j][lane], static_cast<float>(len) * w2[j]);
+            }
+            // ---- sweep A: outputs, c_t, dr, du, reverse summary ----
+            float co[LS][V], cn[LS][V], cd[LS][V];
+            St rs[V] = {st_identity(), st_identity()};
+            {
+                St S_[V] = {F[0], F[1]};
+                IO* drp = GATE ? static_cast<IO*>(A.dr) + (bs * A.T + t_seg) * A.C + c : nullptr;
+#pragma unroll
+                for (int i = 0; i < LS; ++i) {
+                    if (i < n) {
+                        const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
+                        F2 rr = f2s(0.f);
+                        if (GATE) rr = row(3, i);
+                        float drv[V];
+#pragma unroll
+                        for (int j = 0; j < V; ++j) {
+                            const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                            const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                            const float dyj = j == 0 ? f2lo(dd) : f2hi(dd);
+                            float wkv, inv, o, e2;
+                            bwd_out(S_[j], u2[j], k2, vj, wkv, inv, o, e2);
+                            float g = 1.f;
+                            if (GATE) {
+                                g = rcp(1.f + ex2(-(j == 0 ? f2lo(rr) : f2hi(rr)) * kLog2e));
+                                drv[j] = dyj * wkv * g * (1.f - g);
+                            }
+                            const float dn = g * dyj * inv;
+                            const float dd2 = -dn * wkv;
+                            du_acc[j] = fmaf(fmaf(dn, vj, dd2), e2, du_acc[j]);
+                            co[i][j] = -o;
+                            cn[i][j] = dn;
+                            cd[i][j] = dd2;
+                            rs[j] = st_combine(rs[j], St{-o - static_cast<float>(i) * w2[j], dn, dd2}, 0.f);
+                            bwd_update(S_[j], w2[j], k2, vj);
+                        }
+                        if (GATE && cvalid) Ld::store(drp, drv);
+                    }
+                    if (GATE) drp += A.C;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < V; ++j) s_rseg[warp][j][lane] = rs[j];
+            named_sync(1, W * 32);
+            // ---- fold: reverse state at the end of this warp's segment ----
+            St gend[V] = {s_gcarry[par][0][lane], s_gcarry[par][1][lane]};
+            for (int sg = W - 1; sg > warp; --sg) {
+                const int len = static_cast<int>(max(static_cast<int64_t>(0),
+                                                     min(static_cast<int64_t>(LS), A.T - (chunk * TT + sg * LS))));
+#pragma unroll
+                for (int j = 0; j < V; ++j) gend[j] = st_combine(gend[j], s_rseg[sg][j][lane], static_cast<float>(len) * w2[j]);
+            }
+            // ---- sweep B: dk, dv from the reverse walk ----
+            {
+                St g[V] = {gend[0], gend[1]};
+                IO* dkp = static_cast<IO*>(A.dk) + (bs * A.T + t_seg) * A.C + c;
+                IO* dvp = static_cast<IO*>(A.dv) + (bs * A.T + t_seg) * A.C + c;
+#pragma unroll
+                for (int i = LS - 1; i >= 0; --i) {
+                    if (i < n) {
+                        const F2 kk = row(0, i), vv = row(1, i);
+                        float dkv[V], dvv[V];
+#pragma unroll
+                        for (int j = 0; j < V; ++j) {
+                            const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                            const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                            const float ek = ex2(g[j].p + k2);                 // e^{k_t} gN_{t+1} / A
+                            const float e2 = ex2(u2[j] + k2 + co[i][j]);     // e^{u+k_t} dnum_t / dn
+                            dvv[j] = fmaf(cn[i][j], e2, g[j].a * ek);
+                            dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), e2, fmaf(g[j].a, vj, g[j].b) * ek);
+                            const St gn = st_combine(g[j], St{co[i][j], cn[i][j], cd[i][j]}, w2[j]);
+                            // keep the reverse state after token t for sweep C
+                            co[i][j] = g[j].p;
+                            cn[i][j] = g[j].a;
+                            cd[i][j] = g[j].b;
+                            g[j] = gn;
+                        }
+                        if (cvalid) {
+                            Ld::store(dkp + i * A.C, dkv);
+                            Ld::store(dvp + i * A.C, dvv);
+                        }
+                    }
+                }
+                if (warp == 0) {
+#pragma unroll
+                    for (int j = 0; j < V; ++j) s_gcarry[par ^ 1][j][lane] = g[j];
+                    if (chunk == c0 && to_prev) publish<V>(A.incw + lb * CB, g, epoch, kKindInc, lane);
+                    if (chunk == 0 && A.ds_in != nullptr && cvalid) {
+                        // gradient of the initial state: dL/da0 = gN_0 e^{p0}, ...
+#pragma unroll
+                        for (int j = 0; j < V; ++j) {
+                            const int64_t li = bs * A.C + c + j;
+                            float a0 = 0.f, b0 = 0.f, p2 = kFreshP2;
+                            if (A.s_in != nullptr) {
+                                a0 = A.s_in[li];
+                                b0 = A.s_in[lanes + li];
+                                p2 = A.s_in[2 * lanes + li] * kLog2e;
+                            }
+                            const float sc = ex2(g[j].p + p2);
+                            const float ga = g[j].a * sc, gb = g[j].b * sc;
+                            A.ds_in[li] = ga;
+                            A.ds_in[lanes + li] = gb;
+                            A.ds_in[2 * lanes + li] = fmaf(a0, ga, b0 * gb);
+                        }
+                    }
+                }
+            }
+            // ---- sweep C: dw from the forward states and the reverse states ----
+            {
+                St S_[V] = {F[0], F[1]};
+#pragma unroll
+                for (int i = 0; i < LS; ++i) {
+                    if (i < n) {
+                        const F2 kk = row(0, i), vv = row(1, i);
+#pragma unroll
+                        for (int j = 0; j < V; ++j) {
+                            const float z = fmaf(cn[i][j], S_[j].a, cd[i][j] * S_[j].b) * ex2(co[i][j] + S_[j].p);
+                            dw_acc[j] += z;
+                            bwd_update(S_[j], w2[j], (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e,
+                                       j == 0 ? f2lo(vv) : f2hi(vv));
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        if (!ok) break;
+        // ---- this item's share of dw, du for its lane block ----
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            s_red[0][warp][j][lane] = -lam[j] * dw_acc[j];
+            s_red[1][warp][j][lane] = du_acc[j];
+        }
+        named_sync(1, W * 32);
+        if (warp == 0) {
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                float sw = 0.f, su = 0.f;
+                for (int q = 0; q < W; ++q) {
+                    sw += s_red[0][q][j][lane];
+                    su += s_red[1][q][j][lane];
+                }
+                // at most two items (a head and a tail) share a lane block,
+                // and two additions onto zero commute exactly
+                atomicAdd(A.part + lb * CB + lane * V + j, sw);
+                atomicAdd(A.part + (A.nLB + lb) * CB + lane * V + j, su);
             }
         }
     }
+    if (warp == 0 && lane == 0 && A.hdr != nullptr) finish_bwd_launch(A, gridDim.x);
 }
 
 // dw[c], du[c]: sums of the lane blocks' partials over the sequences.

@@ -93,6 +93,36 @@ struct LaneRange {
         c1 = nc;
         from_prev = true;
     }
+    // item i in the order of the reverse mode, which walks chunks from the
+    // last to the first: the tail of the first lane block (it starts from
+    // the end of the sequence; its reverse state at tail_begin goes to the
+    // previous CTA), then whole lane blocks, then the head of the last one
+    // (it starts from the reverse state the next CTA hands over).
+    __device__ __forceinline__ void item_back(int i, int64_t& lb, int64_t& c0, int64_t& c1, bool& to_prev,
+                                              bool& from_next) const {
+        to_prev = false;
+        from_next = false;
+        if (tail) {
+            if (i == 0) {
+                lb = lb_tail;
+                c0 = tail_begin;
+                c1 = nc;
+                to_prev = true;
+                return;
+            }
+            --i;
+        }
+        if (i < nfull) {
+            lb = f0 + i;
+            c0 = 0;
+            c1 = nc;
+            return;
+        }
+        lb = lb_head;
+        c0 = 0;
+        c1 = head_end;
+        from_next = true;
+    }
 };
 
 // State entering work item i (called by one warp, once per item): the

@@ -86,6 +86,11 @@ SHAPES = [
     (1, 4099, 64, torch.bfloat16, True, True, False),   # ragged last chunk, long
     (4, 333, 256, torch.float32, True, True, True),
     (300, 40, 64, torch.bfloat16, True, False, True),   # more lane blocks than CTA slots
+    # more lane blocks than CTA slots with several chunks each: CTAs take
+    # equal shares of the chunk order and hand one reverse state to the
+    # CTA before them
+    (5, 200, 3840, torch.float32, True, True, True),
+    (7, 130, 2728, torch.bfloat16, True, True, True),   # ragged channel block and last chunk
 ]
 
 
