@@ -90,6 +90,12 @@ struct BwdGeometry {
     static constexpr int THREADS = (W + 1) * 32;
 };
 
+// Fixed-scale fast path limits (base 2): the segment's keys plus |u| span at
+// most kBwdFastSpan, and the entering state, |u| and the carried reverse
+// state lie within kBwdFastState of the segment's scale.
+constexpr float kBwdFastSpan = 96.f;
+constexpr float kBwdFastState = 60.f;
+
 // Output of the current (undecayed) state and token, base 2: wkv, 1/den and
 // the scale o of num and den (num = num_hat 2^o), and e2 = 2^(u2+k2-o).
 // One ex2: exactly one of the two scale factors is 1.
@@ -143,10 +149,11 @@ __device__ __forceinline__ void finish_bwd_launch(const BwdArgs& A, uint32_t cta
 // Reverse state handed over by the CTA that walked the later chunks of lane
 // block lb (one 16-byte word per channel; bounded wait, NaN on expiry).
 template <int V>
-__device__ __noinline__ void bwd_wait_carry(const BwdArgs& A, int64_t lb, uint32_t epoch, St* out) {
+__device__ __noinline__ void bwd_wait_carry(const Word* incw, WsHeader* hdr, uint64_t limit_ns, int64_t lb,
+                                            uint32_t epoch, St* out) {
     constexpr int CB = 32 * V;
     const int lane = threadIdx.x & 31;
-    const Word* src = A.incw + lb * CB + lane * V;
+    const Word* src = incw + lb * CB + lane * V;
     const uint64_t t0 = global_ns();
     unsigned sleep_ns = 32;
     for (;;) {
@@ -162,10 +169,10 @@ __device__ __noinline__ void bwd_wait_carry(const BwdArgs& A, int64_t lb, uint32
             for (int j = 0; j < V; ++j) out[j] = word_state(wv[j]);
             return;
         }
-        if (global_ns() - t0 > A.wait_limit_ns) {
+        if (global_ns() - t0 > limit_ns) {
             if (lane == 0) {
-                atomicOr(&A.hdr->error, kErrTimeout);
-                atomicExch(&A.hdr->err_unit, static_cast<uint32_t>(lb));
+                atomicOr(&hdr->error, kErrTimeout);
+                atomicExch(&hdr->err_unit, static_cast<uint32_t>(lb));
             }
             const float nan = __int_as_float(0x7fc00000);
 #pragma unroll
@@ -276,7 +283,7 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
         if (warp == 0) {
             St g0[V] = {st_identity(), st_identity()};
             if (from_next) {
-                bwd_wait_carry<V>(A, lb, epoch, g0);
+                bwd_wait_carry<V>(A.incw, A.hdr, A.wait_limit_ns, lb, epoch, g0);
             } else if (A.ds_out != nullptr && cvalid) {
                 // the end of the sequence: dL/d(a_T, b_T) of the returned state
 #pragma unroll
@@ -301,15 +308,21 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
             auto row = [&](int arr, int i) -> F2 {
                 return raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + arr * G::TILE + i * G::ROW));
             };
-            // ---- sweep 0: forward summary of the segment ----
+            // ---- sweep 0: forward summary and key range of the segment ----
             St fs[V] = {st_identity(), st_identity()};
+            float kmax[V] = {-3.0e38f, -3.0e38f}, kmin[V] = {3.0e38f, 3.0e38f};
             if (got) {
 #pragma unroll
                 for (int i = 0; i < LS; ++i) {
                     if (i < n) {
                         const F2 kk = row(0, i), vv = row(1, i);
-                        bwd_update(fs[0], w2[0], f2lo(kk) * kLog2e, f2lo(vv));
-                        bwd_update(fs[1], w2[1], f2hi(kk) * kLog2e, f2hi(vv));
+                        const float k0 = f2lo(kk) * kLog2e, k1 = f2hi(kk) * kLog2e;
+                        kmax[0] = fmaxf(kmax[0], k0);
+                        kmin[0] = fminf(kmin[0], k0);
+                        kmax[1] = fmaxf(kmax[1], k1);
+                        kmin[1] = fminf(kmin[1], k1);
+                        bwd_update(fs[0], w2[0], k0, f2lo(vv));
+                        bwd_update(fs[1], w2[1], k1, f2hi(vv));
                     }
                 }
 #pragma unroll
@@ -330,43 +343,111 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
 #pragma unroll
                 for (int j = 0; j < V; ++j) F[j] = st_combine(F[j], s_fseg[sg][j][lane], static_cast<float>(len) * w2[j]);
             }
+            // Fixed-scale fast path of this lane's two channels: every weight of
+            // the segment is taken relative to R = max(largest key, entering
+            // exponent), so each token costs one ex2 and the recurrences are
+            // plain FMAs.  It needs the keys (with the bonus) to span at most
+            // 96 in base 2 and the entering state not to dwarf them; the exact
+            // per-token max form covers the rest.
+            float R[V], eu[V];
+            bool fastA = true;
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                R[j] = fmaxf(kmax[j], F[j].p);
+                eu[j] = ex2(u2[j]);
+                fastA = fastA && (kmax[j] - kmin[j] + fabsf(u2[j]) <= kBwdFastSpan) && (F[j].p - kmax[j] <= kBwdFastState) &&
+                        (fabsf(u2[j]) <= kBwdFastState);
+            }
             // ---- sweep A: outputs, c_t, dr, du, reverse summary ----
+            // registers per token: fast (2^(k-R), dnum 2^R, dden 2^R); exact
+            // (-o_t, dnum 2^o_t, dden 2^o_t)
             float co[LS][V], cn[LS][V], cd[LS][V];
-            St rs[V] = {st_identity(), st_identity()};
+            St rs[V];
             {
-                St S_[V] = {F[0], F[1]};
                 IO* drp = GATE ? static_cast<IO*>(A.dr) + (bs * A.T + t_seg) * A.C + c : nullptr;
+                if (fastA) {
+                    float nh[V], dh[V], pw[V], rn[V] = {0.f, 0.f}, rd[V] = {0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < LS; ++i) {
-                    if (i < n) {
-                        const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
-                        F2 rr = f2s(0.f);
-                        if (GATE) rr = row(3, i);
-                        float drv[V];
-#pragma unroll
-                        for (int j = 0; j < V; ++j) {
-                            const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                            const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
-                            const float dyj = j == 0 ? f2lo(dd) : f2hi(dd);
-                            float wkv, inv, o, e2;
-                            bwd_out(S_[j], u2[j], k2, vj, wkv, inv, o, e2);
-                            float g = 1.f;
-                            if (GATE) {
-                                g = rcp(1.f + ex2(-(j == 0 ? f2lo(rr) : f2hi(rr)) * kLog2e));
-                                drv[j] = dyj * wkv * g * (1.f - g);
-                            }
-                            const float dn = g * dyj * inv;
-                            const float dd2 = -dn * wkv;
-                            du_acc[j] = fmaf(fmaf(dn, vj, dd2), e2, du_acc[j]);
-                            co[i][j] = -o;
-                            cn[i][j] = dn;
-                            cd[i][j] = dd2;
-                            rs[j] = st_combine(rs[j], St{-o - static_cast<float>(i) * w2[j], dn, dd2}, 0.f);
-                            bwd_update(S_[j], w2[j], k2, vj);
-                        }
-                        if (GATE && cvalid) Ld::store(drp, drv);
+                    for (int j = 0; j < V; ++j) {
+                        const float s0 = ex2(F[j].p - R[j]);
+                        nh[j] = F[j].a * s0;
+                        dh[j] = F[j].b * s0;
+                        pw[j] = 1.f;
                     }
-                    if (GATE) drp += A.C;
+#pragma unroll
+                    for (int i = 0; i < LS; ++i) {
+                        if (i < n) {
+                            const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
+                            F2 rr = f2s(0.f);
+                            if (GATE) rr = row(3, i);
+                            float drv[V];
+#pragma unroll
+                            for (int j = 0; j < V; ++j) {
+                                const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                                const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                                const float dyj = j == 0 ? f2lo(dd) : f2hi(dd);
+                                const float ek = ex2(k2 - R[j]);
+                                const float eek = eu[j] * ek;
+                                const float inv = rcp(dh[j] + eek);
+                                const float wkv = fmaf(eek, vj, nh[j]) * inv;
+                                float g = 1.f;
+                                if (GATE) {
+                                    g = rcp(1.f + ex2(-(j == 0 ? f2lo(rr) : f2hi(rr)) * kLog2e));
+                                    drv[j] = dyj * wkv * g * (1.f - g);
+                                }
+                                const float dn = g * dyj * inv;
+                                const float dd2 = -dn * wkv;
+                                du_acc[j] = fmaf(fmaf(dn, vj, dd2), eek, du_acc[j]);
+                                co[i][j] = ek;
+                                cn[i][j] = dn;
+                                cd[i][j] = dd2;
+                                rn[j] = fmaf(pw[j], dn, rn[j]);
+                                rd[j] = fmaf(pw[j], dd2, rd[j]);
+                                pw[j] *= lam[j];
+                                nh[j] = fmaf(lam[j], nh[j], ek * vj);
+                                dh[j] = fmaf(lam[j], dh[j], ek);
+                            }
+                            if (GATE && cvalid) Ld::store(drp, drv);
+                        }
+                        if (GATE) drp += A.C;
+                    }
+#pragma unroll
+                    for (int j = 0; j < V; ++j) rs[j] = St{-R[j], rn[j], rd[j]};
+                } else {
+                    St S_[V] = {F[0], F[1]};
+                    rs[0] = rs[1] = st_identity();
+#pragma unroll
+                    for (int i = 0; i < LS; ++i) {
+                        if (i < n) {
+                            const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
+                            F2 rr = f2s(0.f);
+                            if (GATE) rr = row(3, i);
+                            float drv[V];
+#pragma unroll
+                            for (int j = 0; j < V; ++j) {
+                                const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                                const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                                const float dyj = j == 0 ? f2lo(dd) : f2hi(dd);
+                                float wkv, inv, o, e2;
+                                bwd_out(S_[j], u2[j], k2, vj, wkv, inv, o, e2);
+                                float g = 1.f;
+                                if (GATE) {
+                                    g = rcp(1.f + ex2(-(j == 0 ? f2lo(rr) : f2hi(rr)) * kLog2e));
+                                    drv[j] = dyj * wkv * g * (1.f - g);
+                                }
+                                const float dn = g * dyj * inv;
+                                const float dd2 = -dn * wkv;
+                                du_acc[j] = fmaf(fmaf(dn, vj, dd2), e2, du_acc[j]);
+                                co[i][j] = -o;
+                                cn[i][j] = dn;
+                                cd[i][j] = dd2;
+                                rs[j] = st_combine(rs[j], St{-o - static_cast<float>(i) * w2[j], dn, dd2}, 0.f);
+                                bwd_update(S_[j], w2[j], k2, vj);
+                            }
+                            if (GATE && cvalid) Ld::store(drp, drv);
+                        }
+                        if (GATE) drp += A.C;
+                    }
                 }
             }
 #pragma unroll
@@ -380,41 +461,87 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
 #pragma unroll
                 for (int j = 0; j < V; ++j) gend[j] = st_combine(gend[j], s_rseg[sg][j][lane], static_cast<float>(len) * w2[j]);
             }
+            // the fast reverse walk also needs the carried reverse state in range at scale 2^-R
+            bool fastB = fastA;
+#pragma unroll
+            for (int j = 0; j < V; ++j) fastB = fastB && (gend[j].p + R[j] <= kBwdFastState);
             // ---- sweep B: dk, dv from the reverse walk ----
             {
-                St g[V] = {gend[0], gend[1]};
+                St g0[V];
                 IO* dkp = static_cast<IO*>(A.dk) + (bs * A.T + t_seg) * A.C + c;
                 IO* dvp = static_cast<IO*>(A.dv) + (bs * A.T + t_seg) * A.C + c;
+                if (fastB) {
+                    float gN[V], gD[V];
 #pragma unroll
-                for (int i = LS - 1; i >= 0; --i) {
-                    if (i < n) {
-                        const F2 kk = row(0, i), vv = row(1, i);
-                        float dkv[V], dvv[V];
+                    for (int j = 0; j < V; ++j) {
+                        const float sc = ex2(gend[j].p + R[j]);
+                        gN[j] = gend[j].a * sc;
+                        gD[j] = gend[j].b * sc;
+                    }
 #pragma unroll
-                        for (int j = 0; j < V; ++j) {
-                            const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                            const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
-                            const float ek = ex2(g[j].p + k2);                 // e^{k_t} gN_{t+1} / A
-                            const float e2 = ex2(u2[j] + k2 + co[i][j]);     // e^{u+k_t} dnum_t / dn
-                            dvv[j] = fmaf(cn[i][j], e2, g[j].a * ek);
-                            dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), e2, fmaf(g[j].a, vj, g[j].b) * ek);
-                            const St gn = st_combine(g[j], St{co[i][j], cn[i][j], cd[i][j]}, w2[j]);
-                            // keep the reverse state after token t for sweep C
-                            co[i][j] = g[j].p;
-                            cn[i][j] = g[j].a;
-                            cd[i][j] = g[j].b;
-                            g[j] = gn;
-                        }
-                        if (cvalid) {
-                            Ld::store(dkp + i * A.C, dkv);
-                            Ld::store(dvp + i * A.C, dvv);
+                    for (int i = LS - 1; i >= 0; --i) {
+                        if (i < n) {
+                            const F2 vv = row(1, i);
+                            float dkv[V], dvv[V];
+#pragma unroll
+                            for (int j = 0; j < V; ++j) {
+                                const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                                const float ek = co[i][j], eek = eu[j] * ek;
+                                dvv[j] = fmaf(cn[i][j], eek, gN[j] * ek);
+                                dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), eek, fmaf(gN[j], vj, gD[j]) * ek);
+                                const float nN = fmaf(lam[j], gN[j], cn[i][j]);
+                                const float nD = fmaf(lam[j], gD[j], cd[i][j]);
+                                // keep the reverse state after token t for sweep C
+                                cn[i][j] = gN[j];
+                                cd[i][j] = gD[j];
+                                gN[j] = nN;
+                                gD[j] = nD;
+                            }
+                            if (cvalid) {
+                                Ld::store(dkp + i * A.C, dkv);
+                                Ld::store(dvp + i * A.C, dvv);
+                            }
                         }
                     }
+#pragma unroll
+                    for (int j = 0; j < V; ++j) g0[j] = St{-R[j], gN[j], gD[j]};
+                } else {
+                    St g[V] = {gend[0], gend[1]};
+#pragma unroll
+                    for (int i = LS - 1; i >= 0; --i) {
+                        if (i < n) {
+                            const F2 kk = row(0, i), vv = row(1, i);
+                            float dkv[V], dvv[V];
+#pragma unroll
+                            for (int j = 0; j < V; ++j) {
+                                const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                                const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                                // c_t as a max-form state, whichever way sweep A kept it
+                                const float cx = fastA ? -R[j] : co[i][j];
+                                const float e2 = fastA ? eu[j] * co[i][j] : ex2(u2[j] + k2 + cx);
+                                const float ek = ex2(g[j].p + k2);                 // e^{k_t} gN_{t+1} / A
+                                dvv[j] = fmaf(cn[i][j], e2, g[j].a * ek);
+                                dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), e2, fmaf(g[j].a, vj, g[j].b) * ek);
+                                const St gn = st_combine(g[j], St{cx, cn[i][j], cd[i][j]}, w2[j]);
+                                // keep the reverse state after token t for sweep C
+                                co[i][j] = g[j].p;
+                                cn[i][j] = g[j].a;
+                                cd[i][j] = g[j].b;
+                                g[j] = gn;
+                            }
+                            if (cvalid) {
+                                Ld::store(dkp + i * A.C, dkv);
+                                Ld::store(dvp + i * A.C, dvv);
+                            }
+                        }
+                    }
+                    g0[0] = g[0];
+                    g0[1] = g[1];
                 }
                 if (warp == 0) {
 #pragma unroll
-                    for (int j = 0; j < V; ++j) s_gcarry[par ^ 1][j][lane] = g[j];
-                    if (chunk == c0 && to_prev) publish<V>(A.incw + lb * CB, g, epoch, kKindInc, lane);
+                    for (int j = 0; j < V; ++j) s_gcarry[par ^ 1][j][lane] = g0[j];
+                    if (chunk == c0 && to_prev) publish<V>(A.incw + lb * CB, g0, epoch, kKindInc, lane);
                     if (chunk == 0 && A.ds_in != nullptr && cvalid) {
                         // gradient of the initial state: dL/da0 = gN_0 e^{p0}, ...
 #pragma unroll
@@ -426,8 +553,8 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
                                 b0 = A.s_in[lanes + li];
                                 p2 = A.s_in[2 * lanes + li] * kLog2e;
                             }
-                            const float sc = ex2(g[j].p + p2);
-                            const float ga = g[j].a * sc, gb = g[j].b * sc;
+                            const float sc = ex2(g0[j].p + p2);
+                            const float ga = g0[j].a * sc, gb = g0[j].b * sc;
                             A.ds_in[li] = ga;
                             A.ds_in[lanes + li] = gb;
                             A.ds_in[2 * lanes + li] = fmaf(a0, ga, b0 * gb);
@@ -436,7 +563,28 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
                 }
             }
             // ---- sweep C: dw from the forward states and the reverse states ----
-            {
+            if (fastB) {
+                float nh[V], dh[V];
+#pragma unroll
+                for (int j = 0; j < V; ++j) {
+                    const float s0 = ex2(F[j].p - R[j]);
+                    nh[j] = F[j].a * s0;
+                    dh[j] = F[j].b * s0;
+                }
+#pragma unroll
+                for (int i = 0; i < LS; ++i) {
+                    if (i < n) {
+                        const F2 vv = row(1, i);
+#pragma unroll
+                        for (int j = 0; j < V; ++j) {
+                            dw_acc[j] = fmaf(cn[i][j], nh[j], fmaf(cd[i][j], dh[j], dw_acc[j]));
+                            const float ek = co[i][j];
+                            nh[j] = fmaf(lam[j], nh[j], ek * (j == 0 ? f2lo(vv) : f2hi(vv)));
+                            dh[j] = fmaf(lam[j], dh[j], ek);
+                        }
+                    }
+                }
+            } else {
                 St S_[V] = {F[0], F[1]};
 #pragma unroll
                 for (int i = 0; i < LS; ++i) {

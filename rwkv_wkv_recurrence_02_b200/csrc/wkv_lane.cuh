@@ -128,28 +128,31 @@ struct LaneRange {
 // State entering work item i (called by one warp, once per item): the
 // sequence's initial state, or the state the previous CTA handed over
 // (waited for with a time bound; NaN and a recorded error on expiry).
+// The call's arguments come as values (not the argument block by reference),
+// so the kernel's arguments stay in the constant bank.
 template <int V>
-__device__ __noinline__ void lane_entry_state(const ChunkArgs& A, const LaneRange& R, int i, uint32_t epoch,
-                                              St* out) {
+__device__ __noinline__ void lane_entry_state(const float* s_in, int64_t B, int64_t C, int64_t nCB,
+                                              const Word* incw, WsHeader* hdr, uint64_t limit_ns,
+                                              const LaneRange& R, int i, uint32_t epoch, St* out) {
     constexpr int CB = 32 * V;
     const int lane = threadIdx.x & 31;
-    const int64_t lanes = A.B * A.C;
+    const int64_t lanes = B * C;
     int64_t lb, c0, c1;
     bool from_prev, to_next;
     R.item(i, lb, c0, c1, from_prev, to_next);
-    const int64_t cb = (lb % A.nCB) * CB + lane * V;
+    const int64_t cb = (lb % nCB) * CB + lane * V;
     if (!from_prev) {
 #pragma unroll
         for (int j = 0; j < V; ++j) {
             out[j] = st_identity();
-            if (A.s_in != nullptr && cb + j < A.C) {
-                const int64_t li = (lb / A.nCB) * A.C + cb + j;
-                out[j] = St{A.s_in[2 * lanes + li] * kLog2e, A.s_in[li], A.s_in[lanes + li]};
+            if (s_in != nullptr && cb + j < C) {
+                const int64_t li = (lb / nCB) * C + cb + j;
+                out[j] = St{s_in[2 * lanes + li] * kLog2e, s_in[li], s_in[lanes + li]};
             }
         }
         return;
     }
-    const Word* src = A.incw + lb * CB + lane * V;
+    const Word* src = incw + lb * CB + lane * V;
     const uint64_t t0 = global_ns();
     unsigned sleep_ns = 32;
     for (;;) {
@@ -165,8 +168,11 @@ __device__ __noinline__ void lane_entry_state(const ChunkArgs& A, const LaneRang
             for (int j = 0; j < V; ++j) out[j] = word_state(wv[j]);
             return;
         }
-        if (global_ns() - t0 > A.wait_limit_ns) {
-            if (lane == 0) record_timeout(A, lb);
+        if (global_ns() - t0 > limit_ns) {
+            if (lane == 0) {
+                atomicOr(&hdr->error, kErrTimeout);
+                atomicExch(&hdr->err_unit, static_cast<uint32_t>(lb));
+            }
             const float nan = __int_as_float(0x7fc00000);
 #pragma unroll
             for (int j = 0; j < V; ++j) out[j] = St{nan, nan, nan};
@@ -267,7 +273,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     bool ok = true;
     if (warp == W - 1 && R.count > 0) {
         St x0[V];
-        lane_entry_state<V>(A, R, 0, epoch, x0);
+        lane_entry_state<V>(A.s_in, A.B, A.C, A.nCB, A.incw, A.hdr, A.wait_limit_ns, R, 0, epoch, x0);
 #pragma unroll
         for (int j = 0; j < V; ++j) s_carry[0][j][lane] = x0[j];
     }
@@ -355,7 +361,9 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
                             A.s_out[2 * lanes + li] = nx[j].p * kLn2;
                         }
                     }
-                    if (item + 1 < R.count) lane_entry_state<V>(A, R, item + 1, epoch, nx);
+                    if (item + 1 < R.count)
+                        lane_entry_state<V>(A.s_in, A.B, A.C, A.nCB, A.incw, A.hdr, A.wait_limit_ns, R, item + 1,
+                                            epoch, nx);
                 }
 #pragma unroll
                 for (int j = 0; j < V; ++j) s_carry[par ^ 1][j][lane] = nx[j];

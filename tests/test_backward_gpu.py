@@ -109,6 +109,21 @@ def test_backward_extreme_keys():
     check(d, run(d))
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_mixed_paths(dtype):
+    """Sparse +-50 outliers among N(0, 1) keys: within one launch some
+    segments take the fixed-scale fast path and others the exact one, and
+    reverse states cross between them."""
+    B, T, C = 3, 700, 128
+    d = gen(B, T, C, dtype, True, True, True, seed=21)
+    g = torch.Generator(device="cpu").manual_seed(4)
+    k = torch.randn(B, T, C, generator=g)
+    hit = torch.rand(B, T, C, generator=g) < 0.01
+    k = torch.where(hit, torch.where(torch.rand(B, T, C, generator=g) < 0.5, -50.0, 50.0), k)
+    d["k"] = k.to(dtype).to(DEV).contiguous()
+    check(d, run(d))
+
+
 def test_backward_chunked_equals_one_pass():
     """dstate_in of the later chunk, fed as dstate_out of the earlier one,
     reproduces one backward pass; dw and du add up."""
