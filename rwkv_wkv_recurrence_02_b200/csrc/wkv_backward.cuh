@@ -359,60 +359,53 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
                         (fabsf(u2[j]) <= kBwdFastState);
             }
             // ---- sweep A: outputs, c_t, dr, du, reverse summary ----
-            // registers per token: fast (2^(k-R), dnum 2^R, dden 2^R); exact
-            // (-o_t, dnum 2^o_t, dden 2^o_t)
-            float co[LS][V], cn[LS][V], cd[LS][V];
+            // registers per token, the lane's two channels packed: fast
+            // (2^(k-R), dnum 2^R, dden 2^R); exact (-o_t, dnum 2^o_t, dden 2^o_t)
+            F2 co[LS], cn[LS], cd[LS];
             St rs[V];
+            const F2 L2 = f2s(kLog2e), ONE = f2s(1.f), MONE = f2s(-1.f);
+            const F2 LAM = f2(lam[0], lam[1]), EU = f2(eu[0], eu[1]), NR = f2(-R[0], -R[1]);
             {
                 IO* drp = GATE ? static_cast<IO*>(A.dr) + (bs * A.T + t_seg) * A.C + c : nullptr;
                 if (fastA) {
-                    float nh[V], dh[V], pw[V], rn[V] = {0.f, 0.f}, rd[V] = {0.f, 0.f};
-#pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        const float s0 = ex2(F[j].p - R[j]);
-                        nh[j] = F[j].a * s0;
-                        dh[j] = F[j].b * s0;
-                        pw[j] = 1.f;
-                    }
+                    const float s00 = ex2(F[0].p - R[0]), s01 = ex2(F[1].p - R[1]);
+                    F2 nh = f2(F[0].a * s00, F[1].a * s01), dh = f2(F[0].b * s00, F[1].b * s01);
+                    F2 pw = ONE, rn = f2s(0.f), rd = f2s(0.f), dus = f2s(0.f);
 #pragma unroll
                     for (int i = 0; i < LS; ++i) {
                         if (i < n) {
-                            const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
-                            F2 rr = f2s(0.f);
-                            if (GATE) rr = row(3, i);
-                            float drv[V];
-#pragma unroll
-                            for (int j = 0; j < V; ++j) {
-                                const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                                const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
-                                const float dyj = j == 0 ? f2lo(dd) : f2hi(dd);
-                                const float ek = ex2(k2 - R[j]);
-                                const float eek = eu[j] * ek;
-                                const float inv = rcp(dh[j] + eek);
-                                const float wkv = fmaf(eek, vj, nh[j]) * inv;
-                                float g = 1.f;
-                                if (GATE) {
-                                    g = rcp(1.f + ex2(-(j == 0 ? f2lo(rr) : f2hi(rr)) * kLog2e));
-                                    drv[j] = dyj * wkv * g * (1.f - g);
+                            const F2 vv = row(1, i), dd = row(2, i);
+                            const F2 ek = ex2x2(fma2(row(0, i), L2, NR));
+                            const F2 eek = mul2(EU, ek);
+                            const F2 inv = rcpx2(add2(dh, eek));
+                            const F2 wkv = mul2(fma2(eek, vv, nh), inv);
+                            F2 dn = mul2(dd, inv);
+                            if (GATE) {
+                                const F2 g = rcpx2(add2(ONE, ex2x2(mul2(row(3, i), f2s(-kLog2e)))));
+                                dn = mul2(dn, g);
+                                if (cvalid) {
+                                    const F2 dr2 = mul2(mul2(dd, wkv), mul2(g, fma2(g, MONE, ONE)));
+                                    const float drv[V] = {f2lo(dr2), f2hi(dr2)};
+                                    Ld::store(drp, drv);
                                 }
-                                const float dn = g * dyj * inv;
-                                const float dd2 = -dn * wkv;
-                                du_acc[j] = fmaf(fmaf(dn, vj, dd2), eek, du_acc[j]);
-                                co[i][j] = ek;
-                                cn[i][j] = dn;
-                                cd[i][j] = dd2;
-                                rn[j] = fmaf(pw[j], dn, rn[j]);
-                                rd[j] = fmaf(pw[j], dd2, rd[j]);
-                                pw[j] *= lam[j];
-                                nh[j] = fmaf(lam[j], nh[j], ek * vj);
-                                dh[j] = fmaf(lam[j], dh[j], ek);
                             }
-                            if (GATE && cvalid) Ld::store(drp, drv);
+                            const F2 dd2 = mul2(mul2(dn, wkv), MONE);
+                            dus = fma2(fma2(dn, vv, dd2), eek, dus);
+                            co[i] = ek;
+                            cn[i] = dn;
+                            cd[i] = dd2;
+                            rn = fma2(pw, dn, rn);
+                            rd = fma2(pw, dd2, rd);
+                            pw = mul2(pw, LAM);
+                            nh = fma2(LAM, nh, mul2(ek, vv));
+                            dh = fma2(LAM, dh, ek);
                         }
                         if (GATE) drp += A.C;
                     }
-#pragma unroll
-                    for (int j = 0; j < V; ++j) rs[j] = St{-R[j], rn[j], rd[j]};
+                    du_acc[0] += f2lo(dus);
+                    du_acc[1] += f2hi(dus);
+                    rs[0] = St{-R[0], f2lo(rn), f2lo(rd)};
+                    rs[1] = St{-R[1], f2hi(rn), f2hi(rd)};
                 } else {
                     St S_[V] = {F[0], F[1]};
                     rs[0] = rs[1] = st_identity();
@@ -422,7 +415,7 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
                             const F2 kk = row(0, i), vv = row(1, i), dd = row(2, i);
                             F2 rr = f2s(0.f);
                             if (GATE) rr = row(3, i);
-                            float drv[V];
+                            float drv[V], to[V], tn[V], td[V];
 #pragma unroll
                             for (int j = 0; j < V; ++j) {
                                 const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
@@ -438,12 +431,15 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
                                 const float dn = g * dyj * inv;
                                 const float dd2 = -dn * wkv;
                                 du_acc[j] = fmaf(fmaf(dn, vj, dd2), e2, du_acc[j]);
-                                co[i][j] = -o;
-                                cn[i][j] = dn;
-                                cd[i][j] = dd2;
+                                to[j] = -o;
+                                tn[j] = dn;
+                                td[j] = dd2;
                                 rs[j] = st_combine(rs[j], St{-o - static_cast<float>(i) * w2[j], dn, dd2}, 0.f);
                                 bwd_update(S_[j], w2[j], k2, vj);
                             }
+                            co[i] = f2(to[0], to[1]);
+                            cn[i] = f2(tn[0], tn[1]);
+                            cd[i] = f2(td[0], td[1]);
                             if (GATE && cvalid) Ld::store(drp, drv);
                         }
                         if (GATE) drp += A.C;
@@ -471,64 +467,61 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
                 IO* dkp = static_cast<IO*>(A.dk) + (bs * A.T + t_seg) * A.C + c;
                 IO* dvp = static_cast<IO*>(A.dv) + (bs * A.T + t_seg) * A.C + c;
                 if (fastB) {
-                    float gN[V], gD[V];
-#pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        const float sc = ex2(gend[j].p + R[j]);
-                        gN[j] = gend[j].a * sc;
-                        gD[j] = gend[j].b * sc;
-                    }
+                    const float sc0 = ex2(gend[0].p + R[0]), sc1 = ex2(gend[1].p + R[1]);
+                    F2 gN = f2(gend[0].a * sc0, gend[1].a * sc1), gD = f2(gend[0].b * sc0, gend[1].b * sc1);
 #pragma unroll
                     for (int i = LS - 1; i >= 0; --i) {
                         if (i < n) {
                             const F2 vv = row(1, i);
-                            float dkv[V], dvv[V];
-#pragma unroll
-                            for (int j = 0; j < V; ++j) {
-                                const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
-                                const float ek = co[i][j], eek = eu[j] * ek;
-                                dvv[j] = fmaf(cn[i][j], eek, gN[j] * ek);
-                                dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), eek, fmaf(gN[j], vj, gD[j]) * ek);
-                                const float nN = fmaf(lam[j], gN[j], cn[i][j]);
-                                const float nD = fmaf(lam[j], gD[j], cd[i][j]);
-                                // keep the reverse state after token t for sweep C
-                                cn[i][j] = gN[j];
-                                cd[i][j] = gD[j];
-                                gN[j] = nN;
-                                gD[j] = nD;
-                            }
+                            const F2 ek = co[i], eek = mul2(EU, ek);
+                            const F2 dv2 = fma2(cn[i], eek, mul2(gN, ek));
+                            const F2 dk2 = fma2(fma2(cn[i], vv, cd[i]), eek, mul2(fma2(gN, vv, gD), ek));
+                            const F2 nN = fma2(LAM, gN, cn[i]);
+                            const F2 nD = fma2(LAM, gD, cd[i]);
+                            // keep the reverse state after token t for sweep C
+                            cn[i] = gN;
+                            cd[i] = gD;
+                            gN = nN;
+                            gD = nD;
                             if (cvalid) {
+                                const float dkv[V] = {f2lo(dk2), f2hi(dk2)}, dvv[V] = {f2lo(dv2), f2hi(dv2)};
                                 Ld::store(dkp + i * A.C, dkv);
                                 Ld::store(dvp + i * A.C, dvv);
                             }
                         }
                     }
-#pragma unroll
-                    for (int j = 0; j < V; ++j) g0[j] = St{-R[j], gN[j], gD[j]};
+                    g0[0] = St{-R[0], f2lo(gN), f2lo(gD)};
+                    g0[1] = St{-R[1], f2hi(gN), f2hi(gD)};
                 } else {
                     St g[V] = {gend[0], gend[1]};
 #pragma unroll
                     for (int i = LS - 1; i >= 0; --i) {
                         if (i < n) {
                             const F2 kk = row(0, i), vv = row(1, i);
-                            float dkv[V], dvv[V];
+                            float dkv[V], dvv[V], to[V], tn[V], td[V];
 #pragma unroll
                             for (int j = 0; j < V; ++j) {
                                 const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
                                 const float vj = j == 0 ? f2lo(vv) : f2hi(vv);
+                                const float coj = j == 0 ? f2lo(co[i]) : f2hi(co[i]);
+                                const float cnj = j == 0 ? f2lo(cn[i]) : f2hi(cn[i]);
+                                const float cdj = j == 0 ? f2lo(cd[i]) : f2hi(cd[i]);
                                 // c_t as a max-form state, whichever way sweep A kept it
-                                const float cx = fastA ? -R[j] : co[i][j];
-                                const float e2 = fastA ? eu[j] * co[i][j] : ex2(u2[j] + k2 + cx);
+                                const float cx = fastA ? -R[j] : coj;
+                                const float e2 = fastA ? eu[j] * coj : ex2(u2[j] + k2 + cx);
                                 const float ek = ex2(g[j].p + k2);                 // e^{k_t} gN_{t+1} / A
-                                dvv[j] = fmaf(cn[i][j], e2, g[j].a * ek);
-                                dkv[j] = fmaf(fmaf(cn[i][j], vj, cd[i][j]), e2, fmaf(g[j].a, vj, g[j].b) * ek);
-                                const St gn = st_combine(g[j], St{cx, cn[i][j], cd[i][j]}, w2[j]);
+                                dvv[j] = fmaf(cnj, e2, g[j].a * ek);
+                                dkv[j] = fmaf(fmaf(cnj, vj, cdj), e2, fmaf(g[j].a, vj, g[j].b) * ek);
+                                const St gn = st_combine(g[j], St{cx, cnj, cdj}, w2[j]);
                                 // keep the reverse state after token t for sweep C
-                                co[i][j] = g[j].p;
-                                cn[i][j] = g[j].a;
-                                cd[i][j] = g[j].b;
+                                to[j] = g[j].p;
+                                tn[j] = g[j].a;
+                                td[j] = g[j].b;
                                 g[j] = gn;
                             }
+                            co[i] = f2(to[0], to[1]);
+                            cn[i] = f2(tn[0], tn[1]);
+                            cd[i] = f2(td[0], td[1]);
                             if (cvalid) {
                                 Ld::store(dkp + i * A.C, dkv);
                                 Ld::store(dvp + i * A.C, dvv);
@@ -564,26 +557,18 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
             }
             // ---- sweep C: dw from the forward states and the reverse states ----
             if (fastB) {
-                float nh[V], dh[V];
-#pragma unroll
-                for (int j = 0; j < V; ++j) {
-                    const float s0 = ex2(F[j].p - R[j]);
-                    nh[j] = F[j].a * s0;
-                    dh[j] = F[j].b * s0;
-                }
+                const float s00 = ex2(F[0].p - R[0]), s01 = ex2(F[1].p - R[1]);
+                F2 nh = f2(F[0].a * s00, F[1].a * s01), dh = f2(F[0].b * s00, F[1].b * s01), dws = f2s(0.f);
 #pragma unroll
                 for (int i = 0; i < LS; ++i) {
                     if (i < n) {
-                        const F2 vv = row(1, i);
-#pragma unroll
-                        for (int j = 0; j < V; ++j) {
-                            dw_acc[j] = fmaf(cn[i][j], nh[j], fmaf(cd[i][j], dh[j], dw_acc[j]));
-                            const float ek = co[i][j];
-                            nh[j] = fmaf(lam[j], nh[j], ek * (j == 0 ? f2lo(vv) : f2hi(vv)));
-                            dh[j] = fmaf(lam[j], dh[j], ek);
-                        }
+                        dws = fma2(cn[i], nh, fma2(cd[i], dh, dws));
+                        nh = fma2(LAM, nh, mul2(co[i], row(1, i)));
+                        dh = fma2(LAM, dh, co[i]);
                     }
                 }
+                dw_acc[0] += f2lo(dws);
+                dw_acc[1] += f2hi(dws);
             } else {
                 St S_[V] = {F[0], F[1]};
 #pragma unroll
@@ -592,7 +577,10 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
                         const F2 kk = row(0, i), vv = row(1, i);
 #pragma unroll
                         for (int j = 0; j < V; ++j) {
-                            const float z = fmaf(cn[i][j], S_[j].a, cd[i][j] * S_[j].b) * ex2(co[i][j] + S_[j].p);
+                            const float coj = j == 0 ? f2lo(co[i]) : f2hi(co[i]);
+                            const float cnj = j == 0 ? f2lo(cn[i]) : f2hi(cn[i]);
+                            const float cdj = j == 0 ? f2lo(cd[i]) : f2hi(cd[i]);
+                            const float z = fmaf(cnj, S_[j].a, cdj * S_[j].b) * ex2(coj + S_[j].p);
                             dw_acc[j] += z;
                             bwd_update(S_[j], w2[j], (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e,
                                        j == 0 ? f2lo(vv) : f2hi(vv));
