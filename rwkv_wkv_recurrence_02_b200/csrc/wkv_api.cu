@@ -266,7 +266,9 @@ int launch_tma(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
         int per_sm = 0;
         rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
         if (rc != WKV_OK) return rc;
-        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+        // a configuration that fits no SM is an error, not one CTA per SM
+        if (per_sm <= 0) return record_cuda(cudaErrorLaunchOutOfResources);
+        capacity[dev] = per_sm * sm_count();
     }
     CUtensorMap tk, tv, tr;
     if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
@@ -299,7 +301,9 @@ int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
         int per_sm = 0;
         rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
         if (rc != WKV_OK) return rc;
-        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+        // a configuration that fits no SM is an error, not one CTA per SM
+        if (per_sm <= 0) return record_cuda(cudaErrorLaunchOutOfResources);
+        capacity[dev] = per_sm * sm_count();
     }
     CUtensorMap tk, tv, tr;
     if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
@@ -346,7 +350,9 @@ int launch_part(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
         int per_sm = 0;
         rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
         if (rc != WKV_OK) return rc;
-        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+        // a configuration that fits no SM is an error, not one CTA per SM
+        if (per_sm <= 0) return record_cuda(cudaErrorLaunchOutOfResources);
+        capacity[dev] = per_sm * sm_count();
     }
     const ChunkGeom g = chunk_geom(a.B, a.T, a.C, 2, G::PT);
     a.nCB = g.nCB;
@@ -821,7 +827,9 @@ int launch_backward(wkv::BwdArgs a, int dtype, void* workspace, cudaStream_t st)
         int per_sm = 0;
         rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
         if (rc != WKV_OK) return rc;
-        capacity[dev] = (per_sm > 0 ? per_sm : 1) * sm_count();
+        // a configuration that fits no SM is an error, not one CTA per SM
+        if (per_sm <= 0) return record_cuda(cudaErrorLaunchOutOfResources);
+        capacity[dev] = per_sm * sm_count();
     }
     const int64_t grid = a.nLB < capacity[dev] ? a.nLB : capacity[dev];
     if (grid < a.nLB && a.nchunks > 1) {
@@ -862,14 +870,13 @@ int run_backward(const wkv::BwdArgs& b, wkv::ChunkArgs f, int dtype, void* ws, s
     if (rc != WKV_OK) return rc;
     rc = record_cuda(cudaMemsetAsync(b.part, 0, 2 * size_t(b.nLB) * 64 * sizeof(float), st));
     if (rc != WKV_OK) return rc;
-    // fp32: three stages, one CTA (9 warps) per SM, up to 224 registers;
-    // bf16: two stages, two CTAs per SM, 112 registers
-    if constexpr (sizeof(IO) == 4)
-        return b.r != nullptr ? launch_backward<IO, true, 3, 224>(b, dtype, ws, st)
-                              : launch_backward<IO, false, 3, 224>(b, dtype, ws, st);
-    else
-        return b.r != nullptr ? launch_backward<IO, true, 2, 112>(b, dtype, ws, st)
-                              : launch_backward<IO, false, 2, 112>(b, dtype, ws, st);
+    // three stages, one CTA (9 warps) per SM.  Registers: each of the SM's 4
+    // sub-partitions holds 16K, and one of them carries 3 of the 9 warps, so
+    // at most 168 per thread.  Two CTAs per SM would cap registers at 112,
+    // and the spills cost more than the second CTA gains (measured on the
+    // 14B-shaped layer: 1715 vs 1348 us).
+    return b.r != nullptr ? launch_backward<IO, true, 3, 168>(b, dtype, ws, st)
+                          : launch_backward<IO, false, 3, 168>(b, dtype, ws, st);
 }
 
 }  // namespace

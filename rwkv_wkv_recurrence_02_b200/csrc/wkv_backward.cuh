@@ -263,6 +263,10 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
 
     // ---------------- compute ----------------
     const int64_t lanes = A.B * A.C;
+    // the sizes the forward kernels' segment pass reads
+    ChunkArgs ca{};
+    ca.T = A.T;
+    ca.C = A.C;
     int64_t it = 0;
     bool ok = true;
     for (int item = 0; item < R.count && ok; ++item) {
@@ -272,11 +276,13 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
         const int64_t bs = lb / A.nCB;
         const int64_t c = (lb % A.nCB) * CB + lane * V;
         const bool cvalid = c < A.C;
-        float w2[V], u2[V], lam[V];
+        float w2[V], u2[V], lam[V], wv[V], uv[V];
 #pragma unroll
         for (int j = 0; j < V; ++j) {
-            w2[j] = cvalid ? __ldg(A.w + c + j) * kLog2e : 1.f;
-            u2[j] = cvalid ? __ldg(A.u + c + j) * kLog2e : 0.f;
+            wv[j] = cvalid ? __ldg(A.w + c + j) : 1.f;
+            uv[j] = cvalid ? __ldg(A.u + c + j) : 0.f;
+            w2[j] = cvalid ? wv[j] * kLog2e : 1.f;
+            u2[j] = cvalid ? uv[j] * kLog2e : 0.f;
             lam[j] = ex2(-w2[j]);
         }
         // reverse state after the item's last chunk
@@ -308,21 +314,21 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
             auto row = [&](int arr, int i) -> F2 {
                 return raw_pair<IO>(*reinterpret_cast<const Raw*>(srow + arr * G::TILE + i * G::ROW));
             };
-            // ---- sweep 0: forward summary and key range of the segment ----
+            // ---- sweep 0: forward summary and key range of the segment (the
+            // forward kernels' pass 0/1: fixed-scale fast path, exact fallback) ----
             St fs[V] = {st_identity(), st_identity()};
             float kmax[V] = {-3.0e38f, -3.0e38f}, kmin[V] = {3.0e38f, 3.0e38f};
             if (got) {
+                SegCtx<V, LS> cx;
+                cx.cvalid = cvalid;
+                set_params<V, LS>(cx, wv, uv);
+                if ((chunk + 1) * TT <= A.T) seg_pass01<IO, V, false, W, LS, true, false, false>(ca, chunk, bs, c, stage, cx, fs);
+                else seg_pass01<IO, V, false, W, LS, false, false, false>(ca, chunk, bs, c, stage, cx, fs);
+                if (n > 0) {
 #pragma unroll
-                for (int i = 0; i < LS; ++i) {
-                    if (i < n) {
-                        const F2 kk = row(0, i), vv = row(1, i);
-                        const float k0 = f2lo(kk) * kLog2e, k1 = f2hi(kk) * kLog2e;
-                        kmax[0] = fmaxf(kmax[0], k0);
-                        kmin[0] = fminf(kmin[0], k0);
-                        kmax[1] = fmaxf(kmax[1], k1);
-                        kmin[1] = fminf(kmin[1], k1);
-                        bwd_update(fs[0], w2[0], k0, f2lo(vv));
-                        bwd_update(fs[1], w2[1], k1, f2hi(vv));
+                    for (int j = 0; j < V; ++j) {
+                        kmax[j] = cx.kmax[j];
+                        kmin[j] = cx.kmin[j];
                     }
                 }
 #pragma unroll
