@@ -14,7 +14,6 @@
 
 #include "../../include/wkv.h"
 #include "wkv_chunk.cuh"
-#include "wkv_chunk_ws.cuh"
 #include "wkv_lane.cuh"
 #include "wkv_part.cuh"
 #include "wkv_backward.cuh"
@@ -29,15 +28,13 @@ constexpr int64_t kMaxElems = int64_t(1) << 62;
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
 
-// Chunked-kernel geometry: W compute warps per CTA, LS tokens per warp
-// segment, TT = W * LS tokens per chunk.  The register-load kernel uses
-// kW warps; the warp-specialised TMA kernel kWsW compute warps and a ring of
-// kWsStages stages.  The workspace is sized for the smaller chunk.
+// Register-load look-back kernel: W compute warps per CTA, LS tokens per warp
+// segment, TT = W * LS = 64 tokens per chunk.  The workspace is sized for the
+// smallest unit any kernel publishes words for (64 tokens here and in the
+// part kernel).
 constexpr int kW = 8;
 constexpr int kLS = 8;
-constexpr int kWsW = 4;
-constexpr int kWsStages = 4;
-constexpr int kMinTT = (kW < kWsW ? kW : kWsW) * kLS;
+constexpr int kMinTT = kW * kLS;
 // Lane-resident kernel: compute warps and tokens per warp segment (64-token
 // chunks).
 constexpr int kLaneW = 4;
@@ -212,18 +209,15 @@ bool tma_eligible(int V, int dtype, int64_t B, int64_t T, int64_t C, const void*
 }
 
 // Kernel choice: 0 = automatic; the environment variable WKV_FORWARD_KERNEL
-// (seq | chunk | tma | lookback | part | lane) forces one, for ablation
-// measurements: chunk = register-load look-back kernel, lookback = TMA
-// look-back kernel, part = part kernel, lane = lane-resident kernel, each
-// even where another would run.
+// (seq | chunk | part | lane) forces one, for ablation measurements:
+// chunk = register-load look-back kernel, part = part kernel, lane =
+// lane-resident kernel, each even where another would run.
 int forced_kernel() {
     static int f = []() {
         const char* e = std::getenv("WKV_FORWARD_KERNEL");
         if (e == nullptr) return 0;
         if (std::strcmp(e, "seq") == 0) return 1;
         if (std::strcmp(e, "chunk") == 0) return 2;
-        if (std::strcmp(e, "tma") == 0) return 3;
-        if (std::strcmp(e, "lookback") == 0) return 4;
         if (std::strcmp(e, "part") == 0) return 5;
         if (std::strcmp(e, "lane") == 0) return 6;
         return 0;
@@ -249,39 +243,6 @@ int launch_pdl(void (*kern)(P...), int64_t grid, int threads, uint32_t smem, cud
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return record_cuda(cudaLaunchKernelEx(&cfg, kern, tk, tv, tr, a));
-}
-
-template <typename IO, bool GATE, int STAGES>
-int launch_tma(const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
-    using G = wkv::WsGeometry<IO, 2, GATE, kWsW, kLS, STAGES>;
-    auto kern = wkv::chunk_ws_kernel<IO, 2, GATE, kWsW, kLS, STAGES>;
-    static int capacity[kMaxDevices] = {0};
-    int dev = 0;
-    int rc = record_cuda(cudaGetDevice(&dev));
-    if (rc != WKV_OK) return rc;
-    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
-    if (capacity[dev] == 0) {
-        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
-        if (rc != WKV_OK) return rc;
-        int per_sm = 0;
-        rc = record_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, G::THREADS, G::SMEM));
-        if (rc != WKV_OK) return rc;
-        // a configuration that fits no SM is an error, not one CTA per SM
-        if (per_sm <= 0) return record_cuda(cudaErrorLaunchOutOfResources);
-        capacity[dev] = per_sm * sm_count();
-    }
-    CUtensorMap tk, tv, tr;
-    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
-        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT))
-        return WKV_ERR_CUDA;
-    if (GATE) {
-        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT)) return WKV_ERR_CUDA;
-    } else {
-        tr = tv;
-    }
-    const int64_t grid = a.units < capacity[dev] ? a.units : capacity[dev];
-    kern<<<static_cast<unsigned>(grid), G::THREADS, G::SMEM, st>>>(tk, tv, tr, a);
-    return check_launch();
 }
 
 // Lane-resident kernel: each CTA owns whole lane blocks; grid = min(lane
@@ -407,12 +368,6 @@ int dispatch_lane(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_
     constexpr int S = sizeof(IO) == 4 ? 2 : 3;
     return gate ? launch_lane<IO, true, S>(a, dtype, ws, ws_bytes, st)
                 : launch_lane<IO, false, S>(a, dtype, ws, ws_bytes, st);
-}
-
-template <typename IO>
-int dispatch_tma(bool gate, const wkv::ChunkArgs& a, int dtype, cudaStream_t st) {
-    constexpr int S = kWsStages;
-    return gate ? launch_tma<IO, true, S>(a, dtype, st) : launch_tma<IO, false, S>(a, dtype, st);
 }
 
 template <typename IO, int V>
@@ -567,8 +522,7 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
                        ? dispatch_part<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
                        : dispatch_part<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
         }
-        const bool lane_resident = tma && force != 4;
-        if (lane_resident) {
+        if (tma) {
             const ChunkGeom g = chunk_geom(B, T, C, 2, kLaneW * kLaneLS);
             a.nCB = g.nCB;
             a.nLB = g.nLB;
@@ -578,7 +532,7 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
                        ? dispatch_lane<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
                        : dispatch_lane<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
         }
-        const ChunkGeom g = chunk_geom(B, T, C, V, (tma ? kWsW : kW) * kLS);
+        const ChunkGeom g = chunk_geom(B, T, C, V, kW * kLS);
         a.nCB = g.nCB;
         a.nLB = g.nLB;
         a.nchunks = g.nchunks;
@@ -593,10 +547,6 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
             a.hdr = reinterpret_cast<wkv::WsHeader*>(ws);
             a.aggw = reinterpret_cast<wkv::Word*>(ws + g.aggw_off);
             a.incw = reinterpret_cast<wkv::Word*>(ws + g.incw_off);
-        }
-        if (tma) {
-            return dtype == WKV_F32 ? dispatch_tma<float>(r != nullptr, a, dtype, stream)
-                                    : dispatch_tma<__nv_bfloat16>(r != nullptr, a, dtype, stream);
         }
     }
     if (seq && B * (C / V) > int64_t(0x7fffffff) * 256) return WKV_ERR_SHAPE;

@@ -20,7 +20,7 @@
 // compute warps release a stage with an mbarrier the producer waits on.
 #pragma once
 
-#include "wkv_chunk_ws.cuh"
+#include "wkv_segment.cuh"
 
 namespace wkv {
 

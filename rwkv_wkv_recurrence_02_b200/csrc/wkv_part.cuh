@@ -29,7 +29,7 @@
 // parts with a fixed stride instead.
 #pragma once
 
-#include "wkv_chunk_ws.cuh"
+#include "wkv_segment.cuh"
 
 namespace wkv {
 
