@@ -1,9 +1,11 @@
 """A cross-block wait that runs out is reported, not hung: with the wait limit
-forced to 1 ns (environment knob read once per process) the look-back waits of
-a 300-chunk launch expire before their predecessors publish.  The kernel must
-record WKV_ERR_TIMEOUT in the workspace and write NaN for the affected
-outputs, and the workspace must work again after a reset.  Runs in a child
-process so the knob does not leak into other tests."""
+forced to 1 ns (environment knob read once per process), the look-back waits
+of the kernels whose CTAs wait on one another expire before their
+predecessors publish.  The kernel must record WKV_ERR_TIMEOUT in the workspace and write
+NaN for the affected outputs, and the workspace must work again after a
+reset.  Waits for a CTA's own TMA copies keep their fixed limit, so no copy is
+left in flight.  Each case runs in a child process so the knob does not leak
+into other tests."""
 import os
 import subprocess
 import sys
@@ -12,12 +14,13 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-CHILD = r"""
+FORWARD = r"""
 import sys, torch
 sys.path.insert(0, %r)
 import rwkv_wkv_recurrence_02_b200 as wkv
 from rwkv_wkv_recurrence_02_b200 import inputs as I
-wl = I.Workload("t", 1, 64 * 300, 64, "f32", False, -3.0, 1.0, 1.0, 1.0, False, seed=5)
+B, T, C = %d, %d, %d
+wl = I.Workload("t", B, T, C, "f32", False, -3.0, 1.0, 1.0, 1.0, False, seed=5)
 d = I.make_forward_inputs(wl, device="cuda")
 ws = wkv.Workspace()
 y, s = wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], workspace=ws)
@@ -27,11 +30,27 @@ ws.reset()
 print("AFTER_RESET", ws.status())
 """
 
+# The two look-back kernels: parts and chunks of one lane block run in
+# different CTAs at the same time, so a part waits for the ones before it.
+# The lane-resident forward and the reverse walk hand one state between
+# neighbouring CTAs, but a CTA publishes its word from its first work item and
+# reads its neighbour's only in its last, so that word is there by then and a
+# 1 ns limit cannot expire it; its wait is the same bounded loop.
+CASES = [
+    # name, script, forced kernel, (B, T, C)
+    ("register-load look-back", FORWARD, "chunk", (1, 64 * 300, 64)),
+    ("part kernel look-back", FORWARD, "part", (1, 64 * 300, 64)),
+]
+
 
 @pytest.mark.gpu
-def test_expired_wait_is_reported():
-    env = dict(os.environ, WKV_WAIT_LIMIT_NS="1", WKV_FORWARD_KERNEL="chunk")
-    r = subprocess.run([sys.executable, "-c", CHILD % ROOT], env=env, capture_output=True, text=True, timeout=300)
+@pytest.mark.parametrize("name,script,kernel,shape", CASES, ids=[c[0] for c in CASES])
+def test_expired_wait_is_reported(name, script, kernel, shape):
+    env = dict(os.environ, WKV_WAIT_LIMIT_NS="1")
+    if kernel is not None:
+        env["WKV_FORWARD_KERNEL"] = kernel
+    r = subprocess.run([sys.executable, "-c", script % ((ROOT,) + shape)], env=env, capture_output=True, text=True,
+                       timeout=300)
     assert r.returncode == 0, r.stderr
     out = dict(zip(r.stdout.split()[::2], r.stdout.split()[1::2]))
     assert out["STATUS"] == "-7"           # WKV_ERR_TIMEOUT
