@@ -212,8 +212,9 @@ size_t wkv_forward_noalloc_scratch_bytes(int64_t B, int64_t T, int64_t C, int dt
  *                             256-byte aligned, zeroed once by
  *                             wkv_workspace_init() before its first use (a
  *                             wkv_forward workspace of that size serves too).
- * Requirements of this version: every array 16-byte aligned and C a multiple
- * of 4 (WKV_ERR_ALIGN otherwise).  No output may overlap an input or another
+ * Requirements of this version: every array 16-byte aligned and rows of a
+ * multiple of 16 bytes, i.e. C a multiple of 4 for fp32 and of 8 for bf16
+ * (WKV_ERR_ALIGN otherwise).  No output may overlap an input or another
  * output (WKV_ERR_ALIAS).  T == 0: dw = du = 0 and dstate_in passes
  * dstate_out through.  Asynchronous on `stream` like every call.
  */
