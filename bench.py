@@ -284,9 +284,19 @@ class BackwardCase:
                          workspace=ws, **self.out[i % 2])
 
 
+def workload(name):
+    """A workload by name.  `stream_1m_single` is the streaming workload's
+    whole 1M-token sequence in one call instead of 1024-token chunks."""
+    import dataclasses
+    from rwkv_wkv_recurrence_02_b200 import inputs as I
+    if name == "stream_1m_single":
+        return dataclasses.replace(I.WORKLOADS["stream_1m"], name=name, chunk=0)
+    return I.WORKLOADS[name]
+
+
 def make_case(name, device, seed_base, op="forward"):
     from rwkv_wkv_recurrence_02_b200 import inputs as I
-    wl = I.WORKLOADS[name]
+    wl = workload(name)
     if op == "backward":
         if wl.layers:
             raise SystemExit("--op backward takes the forward workloads (the decode step has no reverse mode)")
@@ -370,13 +380,13 @@ def e2e_measure_backward(case, wkv, ws, steps, warmup, stream):
     return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h}
 
 
-def cpu_baseline_backward(workload: str, budget_s: float, max_reps: int = 1000):
+def cpu_baseline_backward(name: str, budget_s: float, max_reps: int = 1000):
     """The oracle's reverse mode as it stands, on this host's cores, over a
     lane sample of the workload repeated for about `budget_s`."""
     import oracle
     from rwkv_wkv_recurrence_02_b200 import inputs as I
     import numpy as np
-    wl = I.WORKLOADS[workload]
+    wl = workload(name)
     T, B, C = wl.chunk or wl.T, wl.B, wl.C
     cap = max(1, int(1e7 // T))
     csub = C if B * C <= cap else max(1, cap // B)
@@ -400,13 +410,13 @@ def cpu_baseline_backward(workload: str, budget_s: float, max_reps: int = 1000):
             "sample": f"{sample}, repeated {reps}x over {sec:.1f} s"}
 
 
-def cpu_baseline_sample(workload: str, budget_s: float, max_reps: int = 1000):
+def cpu_baseline_sample(name: str, budget_s: float, max_reps: int = 1000):
     """Time the oracle as it stands on this host's cores: whole steps of the
     workload (or a lane sample of one) repeated for about `budget_s`."""
     import numpy as np
     import oracle
     from rwkv_wkv_recurrence_02_b200 import inputs as I
-    wl = I.WORKLOADS[workload]
+    wl = workload(name)
     if wl.layers:
         B, C = wl.B, wl.C
         w, u = I.make_params(wl, layers=wl.layers)
@@ -553,7 +563,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = I.WORKLOADS[args.workload]
+    wl = workload(args.workload)
     budget = args.ref_budget_s
     f = lambda x: None if x is None else x.float().numpy()
     if wl.layers:
@@ -607,7 +617,7 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=3000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--workload", default="layer_1b5",
-                   choices=["tiny", "layer_1b5", "layer_14b", "stream_1m", "decode"])
+                   choices=["tiny", "layer_1b5", "layer_14b", "stream_1m", "stream_1m_single", "decode"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--op", default="forward", choices=["forward", "backward"],
                    help="forward (the headline) or the reverse mode on the same workload")
