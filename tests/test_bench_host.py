@@ -33,6 +33,25 @@ def test_algorithmic_bytes_bf16_and_decode():
     assert bench.algorithmic_bytes(dec, 256, 1, 4096, layers=24) == lanes * 8 + lanes * 24 + 24 * 4096 * 8
 
 
+def test_algorithmic_bytes_backward():
+    wl = I.WORKLOADS["layer_1b5"]
+    n = 8 * 1024 * 2048
+    # k, v, dy, r read + dk, dv, dr written (4 B each); state read, dL/d(a, b)
+    # of the returned state read, dL/d(state) written; w, u read, dw, du written
+    assert bench.algorithmic_bytes_backward(wl, 8, 1024, 2048) == n * 28 + 8 * 2048 * (12 + 8 + 12) + 2048 * 16
+    st = I.WORKLOADS["layer_14b"]       # bf16, gated, no initial state
+    assert bench.algorithmic_bytes_backward(st, 4, 8192, 5120) == 4 * 8192 * 5120 * 14 + 4 * 5120 * 20 + 5120 * 16
+
+
+def test_single_call_stream_workload():
+    wl = bench.workload("stream_1m_single")
+    base = I.WORKLOADS["stream_1m"]
+    assert wl.chunk == 0 and wl.T == base.T == 1 << 20
+    assert (wl.B, wl.C, wl.dtype, wl.gate, wl.seed) == (base.B, base.C, base.dtype, base.gate, base.seed)
+    assert bench.algorithmic_bytes(wl, 1, wl.T, wl.C) == wl.T * 4096 * 6 + 4096 * 12 + 4096 * 8
+    assert bench.parse_args(["--workload", "stream_1m_single", "--op", "backward"]).op == "backward"
+
+
 def test_rates_and_seeds():
     assert bench.whole_job_rate(100, 4, 10, 2.0) == 2000.0
     assert len({bench.rank_seed(0, r) for r in range(8)}) == 8
