@@ -21,6 +21,7 @@ data path), the time is the max over ranks and the value is the total.
 lane sample per step (rank 0 only).
 """
 import argparse
+import math
 import hashlib
 import json
 import os
@@ -215,6 +216,8 @@ class ForwardCase:
         self.elements = self.B * self.T * self.C
         self.bytes = algorithmic_bytes(wl, self.B, self.T, self.C)
         self.launches_per_step = 1
+        self.roofline_per_step = False
+        self.period = nsets
 
     def step(self, i, wkv, ws):
         d = self.sets[i % len(self.sets)]
@@ -227,9 +230,10 @@ class ForwardCase:
 
 
 class DecodeCase:
-    """Decode: one wkv_step over all layers per step, inputs from the ring."""
+    """Decode: one wkv_step over all layers per step, inputs from the ring; or,
+    per_layer, one wkv_step per layer (L = 1 each)."""
 
-    def __init__(self, wl, device, seed_base):
+    def __init__(self, wl, device, seed_base, per_layer=False):
         import torch
         from rwkv_wkv_recurrence_02_b200 import inputs as I
         self.wl, self.I = wl, I
@@ -239,13 +243,23 @@ class DecodeCase:
         self.y = torch.empty((wl.layers, wl.B, wl.C), dtype=wl.torch_dtype, device=device)
         self.elements = wl.layers * wl.B * wl.C
         self.bytes = algorithmic_bytes(wl, wl.B, 1, wl.C, layers=wl.layers)
-        self.launches_per_step = 1
+        self.per_layer = per_layer
+        self.launches_per_step = wl.layers if per_layer else 1
+        self.roofline_per_step = per_layer
+        # steps whose inputs coincide: the ring start advances by `layers` mod `ring`
+        self.period = wl.ring // math.gcd(wl.layers, wl.ring)
 
     def step(self, i, wkv, ws):
         a = self.I.decode_ring_start(self.wl, i)
         L = self.wl.layers
-        wkv.wkv_step(self.w, self.u, self.k[a:a + L], self.v[a:a + L], self.state,
-                     None if self.r is None else self.r[a:a + L], y=self.y)
+        if not self.per_layer:
+            wkv.wkv_step(self.w, self.u, self.k[a:a + L], self.v[a:a + L], self.state,
+                         None if self.r is None else self.r[a:a + L], y=self.y)
+            return
+        for l in range(L):
+            sl = slice(l, l + 1)
+            wkv.wkv_step(self.w[sl], self.u[sl], self.k[a + l:a + l + 1], self.v[a + l:a + l + 1], self.state[sl],
+                         None if self.r is None else self.r[a + l:a + l + 1], y=self.y[sl])
 
 
 class BackwardCase:
@@ -277,6 +291,8 @@ class BackwardCase:
         self.elements = self.B * T * self.C
         self.bytes = algorithmic_bytes_backward(wl, self.B, T, self.C)
         self.launches_per_step = 3   # checkpoint sweep, reverse walk, dw/du reduction
+        self.roofline_per_step = True
+        self.period = len(self.sets) * 2 // math.gcd(len(self.sets), 2)
 
     def step(self, i, wkv, ws):
         d = self.sets[i % len(self.sets)]
@@ -294,7 +310,7 @@ def workload(name):
     return I.WORKLOADS[name]
 
 
-def make_case(name, device, seed_base, op="forward"):
+def make_case(name, device, seed_base, op="forward", per_layer=False):
     from rwkv_wkv_recurrence_02_b200 import inputs as I
     wl = workload(name)
     if op == "backward":
@@ -302,7 +318,7 @@ def make_case(name, device, seed_base, op="forward"):
             raise SystemExit("--op backward takes the forward workloads (the decode step has no reverse mode)")
         return BackwardCase(wl, device, seed_base)
     if wl.layers:
-        return DecodeCase(wl, device, seed_base)
+        return DecodeCase(wl, device, seed_base, per_layer)
     return ForwardCase(wl, device, seed_base)
 
 
@@ -312,8 +328,8 @@ def e2e_measure(case, wkv, ws, steps, warmup, stream):
     import torch
     if isinstance(case, BackwardCase):
         return e2e_measure_backward(case, wkv, ws, steps, warmup, stream)
-    if not isinstance(case, ForwardCase):
-        return None
+    if isinstance(case, DecodeCase):
+        return e2e_measure_decode(case, wkv, steps, warmup, stream)
     d = case.sets[0]
     host = {k: (None if v is None else v.to("cpu").pin_memory()) for k, v in d.items()}
     y_host = torch.empty(case.y[0].shape, dtype=case.y[0].dtype).pin_memory()
@@ -342,6 +358,46 @@ def e2e_measure(case, wkv, ws, steps, warmup, stream):
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) / 1e3
     return {"seconds": sec, "steps": steps, "h2d": h2d, "d2h": d2h}
+
+
+def e2e_measure_decode(case, wkv, steps, warmup, stream):
+    """Decode through the public API with host buffers: each step copies the
+    token's k, v (and r) for every layer from pinned host memory, runs the
+    step in the bench's form, and reads y of every layer back."""
+    import torch
+    L = case.wl.layers
+    a = case.I.decode_ring_start(case.wl, 0)
+    host = [None if t is None else t[a:a + L].to("cpu").pin_memory() for t in (case.k, case.v, case.r)]
+    dev = [None if t is None else torch.empty_like(t, device=case.k.device) for t in host]
+    y_host = torch.empty(case.y.shape, dtype=case.y.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host if t is not None)
+    d2h = y_host.numel() * y_host.element_size()
+
+    def one():
+        for dv, hv in zip(dev, host):
+            if hv is not None:
+                dv.copy_(hv, non_blocking=True)
+        k, v, r = dev
+        if case.per_layer:
+            for l in range(L):
+                sl = slice(l, l + 1)
+                wkv.wkv_step(case.w[sl], case.u[sl], k[sl], v[sl], case.state[sl],
+                             None if r is None else r[sl], y=case.y[sl])
+        else:
+            wkv.wkv_step(case.w, case.u, k, v, case.state, r, y=case.y)
+        y_host.copy_(case.y, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h,
+            "path": "pinned host -> wkv_step (C ABI) -> pinned host"}
 
 
 def e2e_measure_backward(case, wkv, ws, steps, warmup, stream):
@@ -377,7 +433,8 @@ def e2e_measure_backward(case, wkv, ws, steps, warmup, stream):
         one()
     e1.record(stream)
     torch.cuda.synchronize()
-    return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h}
+    return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h,
+            "path": "pinned host -> wkv_backward (C ABI) -> pinned host"}
 
 
 def cpu_baseline_backward(name: str, budget_s: float, max_reps: int = 1000):
@@ -485,12 +542,24 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     wkv.lib()
-    case = make_case(args.workload, device, rank_seed(0, rank), args.op)
+    case = make_case(args.workload, device, rank_seed(0, rank), args.op, args.decode_per_layer)
     ws = wkv.Workspace(device)
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
         case.step(i, wkv, ws)
     torch.cuda.synchronize()
+    graphs = None
+    if args.graph:
+        # one CUDA graph per distinct step (inputs rotate with period case.period)
+        graphs = []
+        for p in range(case.period):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                case.step(args.warmup + p, wkv, ws)
+            graphs.append(g)
+        for p in range(case.period):
+            graphs[p].replay()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = ClockSampler(local).start()
@@ -502,7 +571,10 @@ def run_ours(args):
     t0 = time.time()
     e0.record(stream)
     for i in range(args.steps):
-        case.step(args.warmup + i, wkv, ws)
+        if graphs is not None:
+            graphs[i % len(graphs)].replay()
+        else:
+            case.step(args.warmup + i, wkv, ws)
     e1.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
@@ -516,7 +588,7 @@ def run_ours(args):
     # the roofline of a multi-kernel step (the backward) is taken over the whole
     # step: its algorithmic bytes over the step's time, a lower bound on the
     # dominant kernel's fraction
-    per_launch = sec / args.steps / (1 if isinstance(case, BackwardCase) else case.launches_per_step)
+    per_launch = sec / args.steps / (1 if case.roofline_per_step else case.launches_per_step)
     peak, peak_kind = load_peaks()
     achieved = case.bytes / per_launch / 1e9
     out = {
@@ -525,12 +597,15 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "io_dtype": case.wl.dtype,
         "data": "synthetic (seeded; distributions of the workload definition)",
-        "config": dict(config_of(case, args.workload, world), **({"op": "backward"} if args.op == "backward" else {})),
+        "config": dict(config_of(case, args.workload, world), **({"op": "backward"} if args.op == "backward" else {}),
+                       **({"graph": f"{len(graphs)} captured steps replayed"} if graphs is not None else {}),
+                       **({"decode_form": "one wkv_step per layer (L = 1)"} if args.decode_per_layer else {})),
         "hbm_gbs": achieved, "hbm_pct_of_spec_8tbs": 100.0 * achieved / SPEC_HBM_GBS,
         "hbm_pct_of_measured": 100.0 * achieved / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "scope": ("whole step: checkpoint sweep + reverse walk + dw/du reduction"
-                               if isinstance(case, BackwardCase) else "the step's one kernel"),
+                               if isinstance(case, BackwardCase) else
+                               "whole step: one launch per layer" if case.roofline_per_step else "the step's one kernel"),
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": case.bytes,
                      "traffic": load_traffic(args.workload + ("_backward" if args.op == "backward" else ""))},
@@ -543,7 +618,7 @@ def run_ours(args):
             out["e2e"] = {"value": whole_job_rate(case.elements, world, e["steps"],
                                                   max_over_ranks(e["seconds"], dist if world > 1 else None)),
                           "unit": UNIT, "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
-                          "steps": e["steps"], "path": "pinned host -> wkv_forward (C ABI) -> pinned host"}
+                          "steps": e["steps"], "path": e.get("path", "pinned host -> wkv_forward (C ABI) -> pinned host")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = (cpu_baseline_backward(args.workload, args.cpu_seconds) if args.op == "backward"
                                else cpu_baseline_sample(args.workload, args.cpu_seconds))
@@ -619,6 +694,10 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="layer_1b5",
                    choices=["tiny", "layer_1b5", "layer_14b", "stream_1m", "stream_1m_single", "decode"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--graph", action="store_true",
+                   help="replay each step from a captured CUDA graph instead of launching it")
+    p.add_argument("--decode-per-layer", action="store_true",
+                   help="decode: one wkv_step per layer (L = 1) instead of one call over all layers")
     p.add_argument("--op", default="forward", choices=["forward", "backward"],
                    help="forward (the headline) or the reverse mode on the same workload")
     p.add_argument("--e2e-steps", type=int, default=20)

@@ -116,3 +116,67 @@ def test_reference_arm_prints_one_line():
     assert out["impl"] == "reference" and out["unit"] == "elements/s" and out["value"] > 0
     assert out["cpu_baseline"]["kind"] == "oracle" and out["e2e"]["h2d_bytes_per_step"] == 0
     assert out["config"]["workload"] == "layer_1b5"
+
+
+def test_decode_forms_and_graph_period():
+    """The per-layer decode form issues one L = 1 call per layer on the same rows
+    as the one-call form, and steps one graph period apart read the same rows."""
+    import dataclasses
+    wl = dataclasses.replace(I.WORKLOADS["decode"], B=2, C=8)
+
+    class Rec:
+        def __init__(self):
+            self.calls = []
+
+        def wkv_step(self, w, u, k, v, state, r, y):
+            self.calls.append((w.shape[0], k.data_ptr(), state.data_ptr(), y.data_ptr()))
+
+    one = bench.DecodeCase(wl, "cpu", 0)
+    per = bench.DecodeCase(wl, "cpu", 0, per_layer=True)
+    assert one.launches_per_step == 1 and per.launches_per_step == wl.layers
+    assert one.period == per.period == 8
+    for i in range(3 * one.period):
+        assert I.decode_ring_start(wl, i) == I.decode_ring_start(wl, i + one.period)
+        a, b = Rec(), Rec()
+        one.step(i, a, None)
+        per.step(i, b, None)
+        assert len(a.calls) == 1 and a.calls[0][0] == wl.layers
+        assert len(b.calls) == wl.layers and all(c[0] == 1 for c in b.calls)
+        row = one.k[0].numel() * one.k.element_size()
+        assert a.calls[0][1] - one.k.data_ptr() == b.calls[0][1] - per.k.data_ptr()
+        assert [c[1] - per.k.data_ptr() for c in b.calls] == [(I.decode_ring_start(wl, i) + l) * row
+                                                              for l in range(wl.layers)]
+
+
+def test_decode_e2e_bytes():
+    """The decode end-to-end leg copies k, v, r of every layer in and y out."""
+    import dataclasses
+    import torch
+    wl = dataclasses.replace(I.WORKLOADS["decode"], B=2, C=8)
+    case = bench.DecodeCase(wl, "cpu", 0, per_layer=True)
+    calls = []
+
+    class Rec:
+        def wkv_step(self, w, u, k, v, state, r, y):
+            calls.append(k.shape[0])
+
+    class Ev:
+        def __init__(self, **kw):
+            pass
+
+        def record(self, stream):
+            pass
+
+        def elapsed_time(self, other):
+            return 1.0
+
+    orig_pin, orig_ev, orig_sync = torch.Tensor.pin_memory, torch.cuda.Event, torch.cuda.synchronize
+    torch.Tensor.pin_memory, torch.cuda.Event, torch.cuda.synchronize = (lambda t: t), Ev, (lambda: None)
+    try:
+        e = bench.e2e_measure(case, Rec(), None, 3, 1, None)
+    finally:
+        torch.Tensor.pin_memory, torch.cuda.Event, torch.cuda.synchronize = orig_pin, orig_ev, orig_sync
+    el = torch.tensor([], dtype=wl.torch_dtype).element_size()
+    assert e["h2d"] == 3 * wl.layers * wl.B * wl.C * el
+    assert e["d2h"] == wl.layers * wl.B * wl.C * el
+    assert calls == [1] * (wl.layers * 4) and "wkv_step" in e["path"]
