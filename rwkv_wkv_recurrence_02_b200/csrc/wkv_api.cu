@@ -386,14 +386,23 @@ void dispatch_forward(bool gate, bool seq, const wkv::ChunkArgs& a, int64_t grid
 }
 
 template <typename IO, int V, bool GATE>
-void launch_step(int64_t L, int64_t B, int64_t C, const float* w, const float* u, const void* k,
+int launch_step(int64_t L, int64_t B, int64_t C, const float* w, const float* u, const void* k,
                  const void* v, const void* r, float* state, void* y, cudaStream_t st) {
     const int64_t total = L * B * (C / V);
     const int threads = 256;
     const int64_t blocks = (total + threads - 1) / threads;
-    wkv::step_kernel<IO, V, GATE><<<static_cast<unsigned>(blocks), threads, 0, st>>>(
-        L, B, C, w, u, static_cast<const IO*>(k), static_cast<const IO*>(v),
-        static_cast<const IO*>(r), state, static_cast<IO*>(y));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(threads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return record_cuda(cudaLaunchKernelEx(&cfg, wkv::step_kernel<IO, V, GATE>, L, B, C, w, u,
+                                          static_cast<const IO*>(k), static_cast<const IO*>(v),
+                                          static_cast<const IO*>(r), state, static_cast<IO*>(y)));
 }
 
 }  // namespace
@@ -587,15 +596,13 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype, const float* w, const f
 #define WKV_STEP(IO_, V_)                                                                  \
     (g ? launch_step<IO_, V_, true>(L, B, C, w, u, k, v, r, state, y, stream)              \
        : launch_step<IO_, V_, false>(L, B, C, w, u, k, v, r, state, y, stream))
-    if (dtype == WKV_F32) {
-        if (V == 2) WKV_STEP(float, 2);
-        else WKV_STEP(float, 1);
-    } else {
-        if (V == 2) WKV_STEP(__nv_bfloat16, 2);
-        else WKV_STEP(__nv_bfloat16, 1);
-    }
+    int rc;
+    if (dtype == WKV_F32)
+        rc = V == 2 ? WKV_STEP(float, 2) : WKV_STEP(float, 1);
+    else
+        rc = V == 2 ? WKV_STEP(__nv_bfloat16, 2) : WKV_STEP(__nv_bfloat16, 1);
 #undef WKV_STEP
-    return check_launch();
+    return rc != WKV_OK ? rc : check_launch();
 }
 
 // ---------------------------------------------------------------------------

@@ -624,17 +624,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     return mbar_wait_slow(bar, parity, limit_ns);
 }
 
-// Programmatic dependent launch: let the next kernel of the stream be
-// scheduled as this one's CTAs retire, then wait until the previous kernel
-// of the stream has finished and its writes are visible.  Nothing before
-// this may read or write global memory (kernel parameters, tensor maps
-// included, are not global memory).  Without the launch attribute both are
-// no-ops.
-__device__ __forceinline__ void pdl_begin() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -188,6 +188,17 @@ __device__ __forceinline__ F2 add2(F2 a, F2 b) {
 __device__ __forceinline__ F2 ex2x2(F2 x) { return f2(ex2(f2lo(x)), ex2(f2hi(x))); }
 __device__ __forceinline__ F2 rcpx2(F2 x) { return f2(rcp(f2lo(x)), rcp(f2hi(x))); }
 
+// Programmatic dependent launch: let the next kernel of the stream be
+// scheduled as this one's CTAs retire, then wait until the previous kernel
+// of the stream has finished and its writes are visible.  Nothing before
+// this may read or write global memory (kernel parameters, tensor maps
+// included, are not global memory).  Without the launch attribute both are
+// no-ops.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // 1 + e^-r, the denominator factor of sigmoid(r) = 1 / (1 + e^-r).
 __device__ __forceinline__ float gate_den(float r) { return 1.f + ex2(-r * kLog2e); }
 

@@ -3,7 +3,9 @@
 // RNN mode of "二重性：Transformerモード vs RNNモード": the same token update
 // as the forward kernels, applied once, with the state streamed from and back
 // to HBM in place.  A thread owns V consecutive channels of one (layer, batch)
-// row; a warp's accesses to every array are contiguous.
+// row; a warp's accesses to every array are contiguous.  Launched as a
+// programmatic dependent of the stream's previous kernel, so that a chain of
+// small calls (one per layer) overlaps each launch with the previous drain.
 #pragma once
 
 #include "wkv_common.cuh"
@@ -20,6 +22,7 @@ step_kernel(int64_t L, int64_t B, int64_t C, const float* __restrict__ w,
     const int64_t cg = C / V;
     const int64_t total = L * B * cg;
     const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    pdl_begin();
     if (g >= total) return;
     const int64_t row = g / cg;          // (l, b)
     const int64_t c = (g % cg) * V;
