@@ -80,13 +80,18 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
 // caller has set them in cx already).  CACHE: keep the per-token
 // exponentials of the fast path in cx.kf for pass 2 (else pass 2 recomputes
 // them from the keys in the stage, and kf is dead after pass 1).
+// EXACT_Q: form every candidate exponent of pass 0 from one product,
+// k2_i - (n-1-i) w2, instead of running sums of w2; the running sums round
+// once per token, which long segments (32 tokens) with a fast decay make
+// visible in q.
 //
 // Pass 0 works on raw keys: the key range (max, min) and the segment's
 // running-max exponent q = max_i (k2_i + i w2) - (n-1) w2, which equals the
 // recurrence p <- max(p - w2, k2) over the segment.  Pass 1 (fast path)
 // scales every token by the largest key: one ex2 per token, whose argument
 // fuses the base-2 conversion.
-template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool PARAMS_IN_STAGE = true, bool CACHE = true>
+template <typename IO, int V, bool GATE, int W, int LS, bool FULL, bool PARAMS_IN_STAGE = true, bool CACHE = true,
+          bool EXACT_Q = false>
 __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, int64_t b, int64_t c,
                                            const unsigned char* stage, SegCtx<V, LS>& cx, St* seg) {
     constexpr int CB = 32 * V;
@@ -106,6 +111,7 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, in
     const F2 W2 = f2(cx.w2[0], cx.w2[1]);
 
     // ---- pass 0 ----
+    const float nm1 = static_cast<float>(cx.nvalid - 1);
     float kx0 = -3.0e38f, kx1 = -3.0e38f, kn0 = 3.0e38f, kn1 = 3.0e38f;
     float qa0 = -3.0e38f, qa1 = -3.0e38f;
     F2 iw = f2s(0.f);
@@ -121,16 +127,22 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, in
             kx1 = max3(kx1, f2hi(ka), f2hi(kb));
             kn0 = min3(kn0, f2lo(ka), f2lo(kb));
             kn1 = min3(kn1, f2hi(ka), f2hi(kb));
-            const F2 qa = fma2(ka, L2, iw);
-            iw = add2(iw, W2);
-            const F2 qb = two ? fma2(kb, L2, iw) : qa;
-            iw = add2(iw, W2);
+            F2 qa, qb;
+            if constexpr (EXACT_Q) {
+                const float oa = static_cast<float>(i) - nm1, ob = oa + 1.f;
+                qa = fma2(ka, L2, f2(oa * cx.w2[0], oa * cx.w2[1]));
+                qb = two ? fma2(kb, L2, f2(ob * cx.w2[0], ob * cx.w2[1])) : qa;
+            } else {
+                qa = fma2(ka, L2, iw);
+                iw = add2(iw, W2);
+                qb = two ? fma2(kb, L2, iw) : qa;
+                iw = add2(iw, W2);
+            }
             qa0 = max3(qa0, f2lo(qa), f2lo(qb));
             qa1 = max3(qa1, f2hi(qa), f2hi(qb));
         }
     }
-    const float nm1 = static_cast<float>(cx.nvalid - 1);
-    const float q[2] = {qa0 - nm1 * cx.w2[0], qa1 - nm1 * cx.w2[1]};
+    const float q[2] = {EXACT_Q ? qa0 : qa0 - nm1 * cx.w2[0], EXACT_Q ? qa1 : qa1 - nm1 * cx.w2[1]};
     cx.kmax[0] = kx0 * kLog2e;
     cx.kmax[1] = kx1 * kLog2e;
     cx.kmin[0] = kn0 * kLog2e;
@@ -159,9 +171,15 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, in
         seg[0] = St{q[0], f2lo(n) * sc0, f2lo(db) * sc0};
         seg[1] = St{q[1], f2hi(n) * sc1, f2hi(db) * sc1};
     } else {
-        // keys too spread for one reference: the exact running-max recurrence
+        // keys too spread for one reference: the exact running-max
+        // recurrence, its exponent held as pb - m w2 (see lane_token_pm)
+        float pb[V], m[V];
 #pragma unroll
-        for (int j = 0; j < V; ++j) seg[j] = st_identity();
+        for (int j = 0; j < V; ++j) {
+            seg[j] = st_identity();
+            pb[j] = seg[j].p;
+            m[j] = 0.f;
+        }
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < cx.nvalid) {
@@ -170,22 +188,61 @@ __device__ __forceinline__ void seg_pass01(const ChunkArgs& A, int64_t chunk, in
                 for (int j = 0; j < V; ++j) {
                     const float k2 = (j == 0 ? f2lo(cx.kf[i]) : f2hi(cx.kf[i])) * kLog2e;
                     const float v1 = j == 0 ? f2lo(vv) : f2hi(vv);
-                    const float pd = seg[j].p - cx.w2[j];
+                    const float pd = fmaf(-(m[j] + 1.f), cx.w2[j], pb[j]);
                     const float d2 = pd - k2;
                     const float e = ex2(-fabsf(d2));
                     if (d2 >= 0.f) {
                         seg[j].a = fmaf(e, v1, seg[j].a);
                         seg[j].b += e;
-                        seg[j].p = pd;
+                        m[j] += 1.f;
                     } else {
                         seg[j].a = fmaf(e, seg[j].a, v1);
                         seg[j].b = fmaf(e, seg[j].b, 1.f);
-                        seg[j].p = k2;
+                        pb[j] = k2;
+                        m[j] = 0.f;
                     }
                 }
             }
         }
+#pragma unroll
+        for (int j = 0; j < V; ++j) seg[j].p = fmaf(-m[j], cx.w2[j], pb[j]);
     }
+}
+
+// One token of the exact recurrence (as lane_token, base 2) with the
+// running-max exponent held as pb - m w: pb is the last new maximum, m the
+// decay steps since.  Each token forms its exponents from pb with one
+// rounding; p <- p - w would round once per token, and at exponents near the
+// largest keys (|p| ~ 70 for keys of 50) that error accumulates along the
+// segment into the relative weights of old and new terms.
+__device__ __forceinline__ float lane_token_pm(float& a, float& b, float& pb, float& m, float w, float u, float k,
+                                               float v, float gate_den) {
+    const float p = fmaf(-m, w, pb);
+    const float d1 = p - (u + k);
+    const float e1 = ex2(-fabsf(d1));
+    float num, den;
+    if (d1 >= 0.f) {
+        num = fmaf(e1, v, a);
+        den = b + e1;
+    } else {
+        num = fmaf(e1, a, v);
+        den = fmaf(e1, b, 1.f);
+    }
+    const float y = num * rcp(den * gate_den);
+    const float pd = fmaf(-(m + 1.f), w, pb);
+    const float d2 = pd - k;
+    const float e2 = ex2(-fabsf(d2));
+    if (d2 >= 0.f) {
+        a = fmaf(e2, v, a);
+        b = b + e2;
+        m += 1.f;
+    } else {
+        a = fmaf(e2, a, v);
+        b = fmaf(e2, b, 1.f);
+        pb = k;
+        m = 0.f;
+    }
+    return y;
 }
 // Pass 2 of one warp's segment: outputs from the segment's start state st.
 // Fast path: every term rescaled to R = max(kmax, p) and the cached
@@ -251,6 +308,12 @@ __device__ __forceinline__ void seg_pass2(const ChunkArgs& A, const unsigned cha
             yp += C;
         }
     } else {
+        float pb[V], m[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            pb[j] = st[j].p;
+            m[j] = 0.f;
+        }
 #pragma unroll
         for (int i = 0; i < LS; ++i) {
             if (FULL || i < cx.nvalid) {
@@ -263,13 +326,15 @@ __device__ __forceinline__ void seg_pass2(const ChunkArgs& A, const unsigned cha
                 for (int j = 0; j < V; ++j) {
                     const float gd = GATE ? gate_den(j == 0 ? f2lo(rv) : f2hi(rv)) : 1.f;
                     const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                    out[j] = lane_token(st[j].a, st[j].b, st[j].p, cx.w2[j], cx.u2[j], k2,
-                                        j == 0 ? f2lo(vv) : f2hi(vv), gd, 1.f);
+                    out[j] = lane_token_pm(st[j].a, st[j].b, pb[j], m[j], cx.w2[j], cx.u2[j], k2,
+                                           j == 0 ? f2lo(vv) : f2hi(vv), gd);
                 }
                 Ld::store(yp, out);
             }
             yp += C;
         }
+#pragma unroll
+        for (int j = 0; j < V; ++j) st[j].p = fmaf(-m[j], cx.w2[j], pb[j]);
     }
 }
 
