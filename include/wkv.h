@@ -94,6 +94,14 @@ typedef enum {
  *                later call with any shape.  May be NULL when the required
  *                size is 0.  Calls sharing a workspace must be ordered on the
  *                GPU (same stream, or synchronised); they race otherwise.
+ *                NULL (or too small) is also accepted when every sequence
+ *                fits one cluster of parts: 17 <= T <= 1024, C a multiple of
+ *                4 (of 8 for bfloat16), k, v, r, w, u, state_in 16-byte
+ *                aligned, y and state_out aligned to two elements.  Such a
+ *                call runs the cluster kernel, which needs no scratch (thread
+ *                block clusters of ceil(T/128) CTAs that combine their parts'
+ *                summaries in distributed shared memory).  Any other call
+ *                without an adequate workspace returns WKV_ERR_WORKSPACE.
  *   stream       CUDA stream of the launch.
  */
 int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype,
@@ -152,7 +160,9 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype,
  *
  *   - Limit: problems whose scratch need (wkv_forward_noalloc_scratch_bytes)
  *     exceeds WKV_NOALLOC_SCRATCH_BYTES are rejected with WKV_ERR_SCRATCH
- *     before anything runs.  Sequences of at most 64 tokens need none.
+ *     before anything runs.  Sequences of at most 64 tokens need none, and
+ *     neither do calls that fit the cluster kernel (described under
+ *     wkv_forward's workspace): those share no array and need no ordering.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before capturing a stream into a graph.
@@ -171,7 +181,9 @@ int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype,
                         const float* state_in, void* y, float* state_out,
                         cudaStream_t stream);
 
-/* Scratch bytes wkv_forward_noalloc would use for these sizes (0: none). */
+/* Scratch bytes wkv_forward_noalloc would use for these sizes (0: none); an
+ * upper bound: calls that take the cluster kernel (see wkv_forward's
+ * workspace) use none and are not subject to WKV_NOALLOC_SCRATCH_BYTES. */
 size_t wkv_forward_noalloc_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype);
 
 /*

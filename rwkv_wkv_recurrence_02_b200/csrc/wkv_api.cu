@@ -16,6 +16,7 @@
 #include "wkv_chunk.cuh"
 #include "wkv_lane.cuh"
 #include "wkv_part.cuh"
+#include "wkv_cluster.cuh"
 #include "wkv_backward.cuh"
 #include "wkv_seq.cuh"
 #include "wkv_step.cuh"
@@ -49,6 +50,14 @@ constexpr int kPartMinBlocks = 4;
 // exponentials in registers for pass 2
 constexpr int kPartWin = 1;
 constexpr bool kPartCache = true;
+// Cluster kernel: 4 compute warps x 32-token segments (128-token parts), at
+// most 8 parts (a portable cluster) per sequence, four CTAs per SM.  It runs
+// instead of the part kernel when every sequence fits one cluster.
+constexpr int kClusterW = 4;
+constexpr int kClusterLS = 32;
+constexpr int kClusterPT = kClusterW * kClusterLS;
+constexpr int kClusterMax = 8;
+constexpr int kClusterMinBlocks = 4;
 // Sequences at most this long take the sequential kernel.
 constexpr int64_t kSeqMaxT = 16;
 // Limit of every wait on another CTA's result: 1 s, or WKV_WAIT_LIMIT_NS (read
@@ -208,10 +217,22 @@ bool tma_eligible(int V, int dtype, int64_t B, int64_t T, int64_t C, const void*
     return encode_fn() != nullptr;
 }
 
+// The cluster kernel takes the call: TMA-eligible, vectorisable, and every
+// sequence within one cluster of parts.
+bool fits_cluster(int dtype, int64_t B, int64_t T, int64_t C, const void* k, const void* v, const void* r,
+                  const float* w, const float* u, const float* s_in, const void* y, const float* s_out) {
+    if (T <= kSeqMaxT || (T + kClusterPT - 1) / kClusterPT > kClusterMax) return false;
+    if (C % 2 != 0 || !aligned(y, 2 * elem_bytes(dtype)) || (s_out && !aligned(s_out, 8))) return false;
+    const int64_t nLB = B * ((C + 63) / 64);
+    if (nLB * ((T + kClusterPT - 1) / kClusterPT) > 0x7fffffffLL) return false;
+    return tma_eligible(2, dtype, B, T, C, k, v, r, w, u, s_in);
+}
+
 // Kernel choice: 0 = automatic; the environment variable WKV_FORWARD_KERNEL
-// (seq | chunk | part | lane) forces one, for ablation measurements:
-// chunk = register-load look-back kernel, part = part kernel, lane =
-// lane-resident kernel, each even where another would run.
+// (seq | chunk | part | lane | cluster) forces one, for ablation
+// measurements: chunk = register-load look-back kernel, part = part kernel,
+// lane = lane-resident kernel, each even where another would run; cluster =
+// cluster kernel wherever every sequence fits one cluster.
 int forced_kernel() {
     static int f = []() {
         const char* e = std::getenv("WKV_FORWARD_KERNEL");
@@ -220,6 +241,7 @@ int forced_kernel() {
         if (std::strcmp(e, "chunk") == 0) return 2;
         if (std::strcmp(e, "part") == 0) return 5;
         if (std::strcmp(e, "lane") == 0) return 6;
+        if (std::strcmp(e, "cluster") == 0) return 7;
         return 0;
     }();
     return f;
@@ -345,6 +367,66 @@ int launch_part(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
     }
     const int64_t grid = a.units < capacity[dev] ? a.units : capacity[dev];
     return launch_pdl(kern, grid, G::THREADS, G::SMEM, st, tk, tv, tr, a);
+}
+
+// Cluster kernel: one cluster of ceil(T / PT) CTAs per lane block, one CTA
+// per part; needs no workspace (a workspace given only receives a failed
+// copy's error flag).
+template <typename IO, bool GATE>
+int launch_cluster(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+    using G = wkv::PartGeometry<IO, 2, GATE, kClusterW, kClusterLS, 1>;
+    auto kern = wkv::cluster_forward_kernel<IO, 2, GATE, kClusterW, kClusterLS, kClusterMinBlocks>;
+    static bool ready[kMaxDevices] = {false};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (!ready[dev]) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        ready[dev] = true;
+    }
+    const ChunkGeom g = chunk_geom(a.B, a.T, a.C, 2, G::PT);
+    if (g.nchunks < 1 || g.nchunks > kClusterMax || g.units > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    a.nCB = g.nCB;
+    a.nLB = g.nLB;
+    a.nchunks = g.nchunks;
+    a.units = g.units;
+    a.hdr = workspace != nullptr && aligned(workspace, 256) && workspace_bytes >= sizeof(wkv::WsHeader)
+                ? reinterpret_cast<wkv::WsHeader*>(workspace)
+                : nullptr;
+    a.aggw = nullptr;
+    a.incw = nullptr;
+    CUtensorMap tk, tv, tr;
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::PT) ||
+        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::PT))
+        return WKV_ERR_CUDA;
+    if (GATE) {
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
+    } else {
+        tr = tv;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(g.units));
+    cfg.blockDim = dim3(G::THREADS);
+    cfg.dynamicSmemBytes = G::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(g.nchunks);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tk, tv, tr, a));
+}
+
+template <typename IO>
+int dispatch_cluster(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
+    return gate ? launch_cluster<IO, true>(a, dtype, ws, ws_bytes, st)
+                : launch_cluster<IO, false>(a, dtype, ws, ws_bytes, st);
 }
 
 // Part buffers per CTA: as many as fit beside kPartMinBlocks CTAs per SM
@@ -524,6 +606,17 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
         const int64_t nLB = B * ((C + 63) / 64);
         const int64_t nparts = nLB * ((T + kPartW * kPartLS - 1) / (kPartW * kPartLS));
         const bool part_ok = tma && nparts < (int64_t(1) << 31);
+        // Every sequence within one cluster of parts: the cluster kernel needs
+        // no workspace, so it serves calls that bring none (wkv_forward_noalloc
+        // among them).  With a workspace the part kernel runs instead, which
+        // measured a little faster on the streaming chunk.
+        const bool cluster_ok = part_ok && (T + kClusterPT - 1) / kClusterPT <= kClusterMax;
+        const bool ws_ok = workspace != nullptr && workspace_bytes >= wkv_forward_workspace_bytes(B, T, C, dtype);
+        if (cluster_ok && (force == 7 || (force == 0 && !ws_ok))) {
+            return dtype == WKV_F32
+                       ? dispatch_cluster<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
+                       : dispatch_cluster<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
+        }
         const bool part = part_ok && (force == 5 || (force == 0 && nLB < sm_count()));
         if (part) {
             a.nLB = nLB;
@@ -665,6 +758,10 @@ int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype, const float*
     if (B == 0 || C == 0 || T <= kSeqMaxT) {
         // nothing to do, or a sequence short enough for the kernel that needs
         // no scratch: the regular entry point does exactly that
+        return wkv_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, nullptr, 0, stream);
+    }
+    if (fits_cluster(dtype, B, T, C, k, v, r, w, u, state_in, y, state_out) && forced_kernel() == 0) {
+        // the cluster kernel needs no scratch: no shared array, no clearing
         return wkv_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, nullptr, 0, stream);
     }
     if (!w || !u || !k || !v || !y) return WKV_ERR_NULLPTR;

@@ -107,6 +107,7 @@ PART = [
     (1, 128, 64, torch.bfloat16, False, True),
     (1, 129, 128, torch.float32, True, False),
     (2, 1000, 72, torch.bfloat16, True, True),     # ragged channel block and last part
+    (1, 1025, 64, torch.float32, True, True),
     (1, 5000, 256, torch.float32, False, True),    # many parts per lane block
     (2, 2000, 4096, torch.bfloat16, True, False),  # more parts than CTA slots: claimed in ticket order
     (3, 777, 1000, torch.bfloat16, False, True),
@@ -118,6 +119,49 @@ def test_part_shapes(B, T, C, dtype, gate, state):
     d = gen_case(B, T, C, dtype, gate, state, seed=B * 13 + T + C)
     y, s = run_forward(d)
     check_forward(d, y, s)
+
+
+# Calls without a workspace whose sequences fit one cluster (at most 1024
+# tokens): the cluster kernel, one cluster of ceil(T / 128) CTAs per lane
+# block whose parts exchange their summaries through distributed shared
+# memory.  wkv_forward_noalloc brings no workspace.
+CLUSTER = [
+    # B, T, C, dtype, gate, state
+    (1, 17, 64, torch.float32, True, True),        # a cluster of one CTA, shorter than a part
+    (1, 64, 64, torch.bfloat16, False, True),
+    (1, 128, 64, torch.bfloat16, False, True),     # exactly one part
+    (1, 129, 128, torch.float32, True, False),     # one token in the second part
+    (1, 65, 128, torch.float32, True, True),
+    (2, 1000, 72, torch.bfloat16, True, True),     # eight parts, ragged channel block and last part
+    (3, 777, 1000, torch.bfloat16, False, True),
+    (1, 896, 200, torch.bfloat16, True, True),     # seven parts, ragged channel block
+    (1, 1024, 4096, torch.bfloat16, False, True),  # the streaming workload's chunk shape
+    (2, 1024, 2048, torch.float32, True, True),    # fp32 gated: two CTAs per SM, more CTAs than slots
+]
+
+
+@pytest.mark.parametrize("B,T,C,dtype,gate,state", CLUSTER)
+def test_cluster_shapes(B, T, C, dtype, gate, state):
+    d = gen_case(B, T, C, dtype, gate, state, seed=B * 17 + T + C)
+    y = torch.empty_like(d["k"])
+    s = torch.empty((3, B, C), dtype=torch.float32, device=DEV)
+    wkv.wkv_forward_noalloc(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"], y=y, state_out=s)
+    torch.cuda.synchronize()
+    check_forward(d, y, s)
+
+
+def test_cluster_chain_in_place_equals_one_call():
+    """Chunks of one sequence through the cluster kernel, the state carried in
+    place (state_out == state_in), against the oracle over the whole sequence."""
+    d = gen_case(1, 4 * 1000, 256, torch.bfloat16, True, True, seed=4242)
+    state = d["state"].clone()
+    y = torch.empty_like(d["k"])
+    for i in range(4):
+        sl = slice(i * 1000, (i + 1) * 1000)
+        wkv.wkv_forward_noalloc(d["w"], d["u"], d["k"][:, sl], d["v"][:, sl], d["r"][:, sl], state, y=y[:, sl],
+                                state_out=state)
+    torch.cuda.synchronize()
+    check_forward(d, y, state)
 
 
 def test_tiny_workload_against_brute_force():
