@@ -33,6 +33,7 @@ def lib():
         L.oracle_wkv_summary.argtypes = [d, i64, p, p, p]
         L.oracle_wkv_combine.argtypes = [d, d, d, d, d, d, d, i64, p]
         L.oracle_wkv_backward.argtypes = [i64, i64, i64, p, p, p, p, p, p, p, p, p, p, p, p, p, p, i32]
+        L.oracle_token_shift.argtypes = [i64, i64, i64, i64, p, p, p, p, p]
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -128,6 +129,24 @@ def wkv_backward(w, u, k, v, r=None, state_in=None, dy=None, dstate_out=None, nt
                               _ptr(dy), _ptr(dstate_out), _ptr(dk), _ptr(dv), _ptr(dr), _ptr(dw), _ptr(du),
                               _ptr(ds), int(nthreads))
     return dk, dv, dr, dw, du, ds
+
+
+def token_shift(x, mu, x_prev=None):
+    """Token shift: x (B, T, C), mu (nmix, C), x_prev (B, C) or None (zeros).
+    Returns (out (nmix, B, T, C), x_last (B, C)) as float64, where
+    out[m, b, t] = mu[m] * x[b, t] + (1 - mu[m]) * x[b, t - 1] and x[b, -1] is
+    x_prev[b]; x_last is the input the next call mixes its first token with."""
+    x, mu, x_prev = _f32(x), _f32(mu), _f32(x_prev)
+    if x.ndim != 3 or mu.ndim != 2:
+        raise ValueError("x must be (B, T, C) and mu (nmix, C)")
+    B, T, C = x.shape
+    nmix = mu.shape[0]
+    if mu.shape[1] != C or (x_prev is not None and x_prev.shape != (B, C)):
+        raise ValueError("shape mismatch")
+    out = np.empty((nmix, B, T, C), np.float64)
+    last = np.empty((B, C), np.float64)
+    lib().oracle_token_shift(B, T, C, nmix, _ptr(x), _ptr(mu), _ptr(x_prev), _ptr(out), _ptr(last))
+    return out, last
 
 
 def fresh_state(B, C):

@@ -13,7 +13,9 @@
  *     bookkeeping, new max = max(previous max - w, k);
  *   - "並列学習の定式化" (parallel training formulation): the order "output
  *     from the current (undecayed) state, then decay and add";
- * and the block diagram in "高レベル構造" (out_t = sigmoid(r_t) * wkv_t).
+ * and the block diagram in "高レベル構造" (out_t = sigmoid(r_t) * wkv_t);
+ * the token shift that precedes the projections follows "トークンシフト：秘密
+ * の要素" (mixing each input with the previous token's).
  *
  * Conventions shared by every function (all arrays row-major):
  *   k, v, r, y : (B, T, C), channel fastest.   r may be NULL (no gate).
@@ -359,5 +361,39 @@ void oracle_wkv_backward(int64_t B, int64_t T, int64_t C,
         du[c] = du_c;
         free(Nt);
         free(Dt);
+    }
+}
+
+/*
+ * Token shift ("トークンシフト：秘密の要素"): before its R, K, V projections
+ * every sub-layer mixes each token's input with the previous token's,
+ *     x'_t = mu * x_t + (1 - mu) * x_{t-1},
+ * with one learned interpolation weight mu per channel.  nmix mixes (one row
+ * of mu each, e.g. one per projection) of the same input.
+ *
+ *   x      : (B, T, C)
+ *   mu     : (nmix, C)
+ *   x_prev : (B, C), the input of the token before x[:, 0, :] (carried from
+ *            an earlier chunk or decode step), or NULL for a fresh sequence,
+ *            whose first token mixes with zeros.
+ *   out    : (nmix, B, T, C)
+ *   x_last : (B, C) or NULL, receives the input the next call mixes its first
+ *            token with: x[:, T-1, :], or x_prev (zeros) when T == 0.
+ */
+void oracle_token_shift(int64_t B, int64_t T, int64_t C, int64_t nmix, const float* x, const float* mu,
+                        const float* x_prev, double* out, double* x_last) {
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t c = 0; c < C; ++c) {
+            double prev = x_prev ? (double)x_prev[b * C + c] : 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                const double cur = (double)x[(b * T + t) * C + c];
+                for (int64_t m = 0; m < nmix; ++m) {
+                    const double mc = (double)mu[m * C + c];
+                    out[((m * B + b) * T + t) * C + c] = mc * cur + (1.0 - mc) * prev;
+                }
+                prev = cur;
+            }
+            if (x_last) x_last[b * C + c] = prev;
+        }
     }
 }
