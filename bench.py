@@ -36,6 +36,8 @@ if ROOT not in sys.path:
 
 METRIC = "WKV elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
 METRIC_BWD = "WKV backward elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
+METRIC_SHIFT = "token shift elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
+SHIFT_MIXES = 3   # RWKV-4 time mixing: one mix each for K, V and R
 UNIT = "elements/s"
 SPEC_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
@@ -83,6 +85,14 @@ def algorithmic_bytes_backward(wl, B, T, C) -> int:
     io = n * eb * ((narr + 1) + narr)
     state = B * C * (12 * (1 if wl.random_state or wl.chunk else 0) + 8 + 12)
     return io + state + C * 16
+
+
+def algorithmic_bytes_shift(wl, B, T, C, nmix=SHIFT_MIXES) -> int:
+    """Bytes one token-shift call must move at minimum: x read once, nmix
+    output rows written per input row, the carried previous token read and
+    the next one written, mu read."""
+    eb = wl.elem_bytes
+    return B * T * C * eb * (1 + nmix) + 2 * B * C * eb + nmix * C * 4
 
 
 def max_over_ranks(value: float, dist=None) -> float:
@@ -300,6 +310,40 @@ class BackwardCase:
                          workspace=ws, **self.out[i % 2])
 
 
+class TokenShiftCase:
+    """Token shift on a workload's shape (decode: one token of one layer):
+    x of the workload's dtype, SHIFT_MIXES mixes, the previous token carried;
+    inputs rotate over sets larger than L2, outputs preallocated."""
+
+    def __init__(self, wl, device, seed_base):
+        import torch
+        self.wl = wl
+        T = 1 if wl.layers else (wl.chunk or wl.T)
+        self.B, self.T, self.C = wl.B, T, wl.C
+        one = algorithmic_bytes_shift(wl, self.B, T, self.C)
+        nsets = 2
+        while nsets * one < 2 * L2_BYTES:
+            nsets += 1
+        self.sets = []
+        for i in range(nsets):
+            g = torch.Generator(device="cpu").manual_seed(7000 + seed_base + i)
+            self.sets.append({"x": torch.randn(self.B, T, self.C, generator=g).to(wl.torch_dtype).to(device),
+                              "mu": torch.rand(SHIFT_MIXES, self.C, generator=g).to(device),
+                              "xp": torch.randn(self.B, self.C, generator=g).to(wl.torch_dtype).to(device)})
+        self.out = [torch.empty((SHIFT_MIXES, self.B, T, self.C), dtype=wl.torch_dtype, device=device)
+                    for _ in range(2)]
+        self.last = [torch.empty((self.B, self.C), dtype=wl.torch_dtype, device=device) for _ in range(2)]
+        self.elements = self.B * T * self.C
+        self.bytes = one
+        self.launches_per_step = 1
+        self.roofline_per_step = False
+        self.period = nsets * 2 // math.gcd(nsets, 2)
+
+    def step(self, i, wkv, ws):
+        d = self.sets[i % len(self.sets)]
+        wkv.wkv_token_shift(d["x"], d["mu"], d["xp"], out=self.out[i % 2], x_last=self.last[i % 2])
+
+
 def workload(name):
     """A workload by name.  `stream_1m_single` is the streaming workload's
     whole 1M-token sequence in one call instead of 1024-token chunks."""
@@ -313,6 +357,8 @@ def workload(name):
 def make_case(name, device, seed_base, op="forward", per_layer=False):
     from rwkv_wkv_recurrence_02_b200 import inputs as I
     wl = workload(name)
+    if op == "token_shift":
+        return TokenShiftCase(wl, device, seed_base)
     if op == "backward":
         if wl.layers:
             raise SystemExit("--op backward takes the forward workloads (the decode step has no reverse mode)")
@@ -330,6 +376,8 @@ def e2e_measure(case, wkv, ws, steps, warmup, stream):
         return e2e_measure_backward(case, wkv, ws, steps, warmup, stream)
     if isinstance(case, DecodeCase):
         return e2e_measure_decode(case, wkv, steps, warmup, stream)
+    if isinstance(case, TokenShiftCase):
+        return e2e_measure_shift(case, wkv, steps, warmup, stream)
     d = case.sets[0]
     host = {k: (None if v is None else v.to("cpu").pin_memory()) for k, v in d.items()}
     y_host = torch.empty(case.y[0].shape, dtype=case.y[0].dtype).pin_memory()
@@ -398,6 +446,64 @@ def e2e_measure_decode(case, wkv, steps, warmup, stream):
     torch.cuda.synchronize()
     return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h,
             "path": "pinned host -> wkv_step (C ABI) -> pinned host"}
+
+
+def e2e_measure_shift(case, wkv, steps, warmup, stream):
+    """Token shift through the public API with host buffers: x and the
+    previous token in from pinned host memory, every mix and x_last out."""
+    import torch
+    d = case.sets[0]
+    host = {n: d[n].to("cpu").pin_memory() for n in ("x", "mu", "xp")}
+    dev = {n: torch.empty_like(v, device=d["x"].device) for n, v in host.items()}
+    out_h = torch.empty(case.out[0].shape, dtype=case.out[0].dtype).pin_memory()
+    last_h = torch.empty(case.last[0].shape, dtype=case.last[0].dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size() + last_h.numel() * last_h.element_size()
+
+    def one():
+        for n, v in host.items():
+            dev[n].copy_(v, non_blocking=True)
+        wkv.wkv_token_shift(dev["x"], dev["mu"], dev["xp"], out=case.out[0], x_last=case.last[0])
+        out_h.copy_(case.out[0], non_blocking=True)
+        last_h.copy_(case.last[0], non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h,
+            "path": "pinned host -> wkv_token_shift (C ABI) -> pinned host"}
+
+
+def cpu_baseline_shift(name: str, budget_s: float, max_reps: int = 1000):
+    """The oracle's token shift as it stands, on this host, over a channel
+    sample of one call repeated for about `budget_s`."""
+    import numpy as np
+    import oracle
+    wl = workload(name)
+    T = 1 if wl.layers else (wl.chunk or wl.T)
+    B, C = wl.B, wl.C
+    csub = max(1, min(C, int(2e7 // (B * T))))
+    g = np.random.default_rng(3)
+    x = g.standard_normal((B, T, csub)).astype(np.float32)
+    mu = g.uniform(0, 1, (SHIFT_MIXES, csub)).astype(np.float32)
+    xp = g.standard_normal((B, csub)).astype(np.float32)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.token_shift(x, mu, xp)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= max_reps:
+            break
+    sec = time.perf_counter() - t0
+    sample = f"B={B}, T={T}, C={csub} of {C}, {SHIFT_MIXES} mixes"
+    return {"value": B * T * csub * reps / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{sample}, repeated {reps}x over {sec:.1f} s"}
 
 
 def e2e_measure_backward(case, wkv, ws, steps, warmup, stream):
@@ -526,6 +632,15 @@ def config_of(case, workload, world):
     return cfg
 
 
+def shift_config(case):
+    """Config keys of the token shift: its mixes, and for the decode workload
+    that one step is one layer's token."""
+    cfg = {"nmix": SHIFT_MIXES, "x_prev": "carried"}
+    if case.wl.layers:
+        cfg.update({"T": 1, "layers": 1, "decode": "one layer's token per step"})
+    return cfg
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -592,12 +707,13 @@ def run_ours(args):
     peak, peak_kind = load_peaks()
     achieved = case.bytes / per_launch / 1e9
     out = {
-        "metric": METRIC_BWD if args.op == "backward" else METRIC, "value": value, "unit": UNIT,
-        "n_gpus": world, "steps": args.steps,
+        "metric": {"backward": METRIC_BWD, "token_shift": METRIC_SHIFT}.get(args.op, METRIC), "value": value,
+        "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "io_dtype": case.wl.dtype,
         "data": "synthetic (seeded; distributions of the workload definition)",
-        "config": dict(config_of(case, args.workload, world), **({"op": "backward"} if args.op == "backward" else {}),
+        "config": dict(config_of(case, args.workload, world), **({"op": args.op} if args.op != "forward" else {}),
+                       **(shift_config(case) if args.op == "token_shift" else {}),
                        **({"graph": f"{len(graphs)} captured steps replayed"} if graphs is not None else {}),
                        **({"decode_form": "one wkv_step per layer (L = 1)"} if args.decode_per_layer else {})),
         "hbm_gbs": achieved, "hbm_pct_of_spec_8tbs": 100.0 * achieved / SPEC_HBM_GBS,
@@ -608,7 +724,7 @@ def run_ours(args):
                                "whole step: one launch per layer" if case.roofline_per_step else "the step's one kernel"),
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": case.bytes,
-                     "traffic": load_traffic(args.workload + ("_backward" if args.op == "backward" else ""))},
+                     "traffic": load_traffic(args.workload + ("" if args.op == "forward" else "_" + args.op))},
         "gpu_launches": args.steps * case.launches_per_step,
         "clocks": clocks.summary(t0, t1),
     }
@@ -620,8 +736,8 @@ def run_ours(args):
                           "unit": UNIT, "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                           "steps": e["steps"], "path": e.get("path", "pinned host -> wkv_forward (C ABI) -> pinned host")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = (cpu_baseline_backward(args.workload, args.cpu_seconds) if args.op == "backward"
-                               else cpu_baseline_sample(args.workload, args.cpu_seconds))
+        out["cpu_baseline"] = {"backward": cpu_baseline_backward, "token_shift": cpu_baseline_shift}.get(
+            args.op, cpu_baseline_sample)(args.workload, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -641,6 +757,8 @@ def run_reference(args):
     wl = workload(args.workload)
     budget = args.ref_budget_s
     f = lambda x: None if x is None else x.float().numpy()
+    if args.op == "token_shift":
+        return run_reference_shift(args, wl)
     if wl.layers:
         raise SystemExit("--impl reference times the forward workloads")
     T, B, C = (wl.chunk or wl.T), wl.B, wl.C
@@ -686,6 +804,45 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_reference_shift(args, wl):
+    """The oracle's token shift on a channel sample of the workload's call,
+    sized so that every step takes a bounded share of the budget."""
+    import numpy as np
+    import oracle
+    T = 1 if wl.layers else (wl.chunk or wl.T)
+    B, C = wl.B, wl.C
+    g = np.random.default_rng(3)
+    per_step = args.ref_budget_s / max(1, args.steps + args.warmup)
+    cal = 64
+    xc = g.standard_normal((B, T, cal)).astype(np.float32)
+    muc = g.uniform(0, 1, (SHIFT_MIXES, cal)).astype(np.float32)
+    t0 = time.perf_counter()
+    oracle.token_shift(xc, muc, None)
+    per_chan = (time.perf_counter() - t0) / cal
+    csub = int(max(1, min(C, per_step / max(per_chan, 1e-12))))
+    x = g.standard_normal((B, T, csub)).astype(np.float32)
+    mu = g.uniform(0, 1, (SHIFT_MIXES, csub)).astype(np.float32)
+    xp = g.standard_normal((B, csub)).astype(np.float32)
+    for _ in range(args.warmup):
+        oracle.token_shift(x, mu, xp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.token_shift(x, mu, xp)
+    sec = time.perf_counter() - t0
+    value = B * T * csub * args.steps / sec
+    sample = f"channel sample B={B}, T={T}, C={csub} of {C}, {SHIFT_MIXES} mixes per step"
+    out = {
+        "metric": METRIC_SHIFT, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "B": B, "T": T, "C": C, "io_dtype": wl.dtype, "op": "token_shift",
+                   "nmix": SHIFT_MIXES},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
@@ -698,8 +855,8 @@ def parse_args(argv=None):
                    help="replay each step from a captured CUDA graph instead of launching it")
     p.add_argument("--decode-per-layer", action="store_true",
                    help="decode: one wkv_step per layer (L = 1) instead of one call over all layers")
-    p.add_argument("--op", default="forward", choices=["forward", "backward"],
-                   help="forward (the headline) or the reverse mode on the same workload")
+    p.add_argument("--op", default="forward", choices=["forward", "backward", "token_shift"],
+                   help="forward (the headline), the reverse mode, or the token shift on the workload's shape")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-budget-s", type=float, default=90.0)

@@ -250,6 +250,41 @@ const char* wkv_last_cuda_error(void);
 /* ABI version of this header: 1. */
 int wkv_abi_version(void);
 
+/*
+ * wkv_token_shift -- the token shift that precedes the R, K, V projections of
+ * every sub-layer (the article's section "トークンシフト：秘密の要素"): each
+ * token's input mixed with the previous token's,
+ *     out[m, b, t, c] = mu[m, c] * x[b, t, c] + (1 - mu[m, c]) * x[b, t-1, c],
+ * with one learned weight per channel, for nmix mixes of one input (RWKV-4's
+ * time mixing takes three: for K, V and R).  x[b, -1, :] is x_prev[b, :], the
+ * input carried from the previous chunk or decode step; a fresh sequence
+ * (x_prev NULL) mixes its first token with zeros.  Decode is T = 1.
+ *
+ *   B, T, C      sizes, each >= 0.  B == 0 or C == 0: nothing to do.
+ *                T == 0: out untouched, x_last = x_prev (zeros if NULL).
+ *   dtype        wkv_dtype of x, x_prev, out, x_last.
+ *   nmix         number of mixes, 1..8.
+ *   x            (B,T,C) device array, required.
+ *   mu           (nmix, C) float32 device array, required.
+ *   x_prev       (B,C) device array, or NULL for zeros.
+ *   out          (nmix,B,T,C) device array, written; must not overlap any
+ *                other argument.  Computed in float32 as mu*x_t +
+ *                (1-mu)*x_{t-1} and rounded once to dtype.
+ *   x_last       (B,C) device array or NULL: receives x[:, T-1, :], the
+ *                x_prev of the next call.  May be the same pointer as x_prev
+ *                (in-place update); other overlaps are WKV_ERR_ALIAS.
+ *   stream       CUDA stream of the launch.
+ *
+ * Returns WKV_OK or an error before launching: WKV_ERR_SHAPE (negative size,
+ * nmix outside 1..8, nmix*B*T*C beyond 2^62), WKV_ERR_NULLPTR, WKV_ERR_DTYPE,
+ * WKV_ERR_ALIGN (a pointer not aligned to its element type), WKV_ERR_ALIAS,
+ * WKV_ERR_CUDA.  16-byte aligned arrays with C a multiple of 4 (float32) or
+ * 8 (bfloat16) take 16-byte accesses; any other layout runs element-wise.
+ */
+int wkv_token_shift(int64_t B, int64_t T, int64_t C, int dtype, int nmix,
+                    const void* x, const float* mu, const void* x_prev,
+                    void* out, void* x_last, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,7 +32,8 @@ STATUS = {
 # the functions include/wkv.h declares
 EXPORTS = ("wkv_forward", "wkv_forward_workspace_bytes", "wkv_workspace_init", "wkv_workspace_status",
            "wkv_step", "wkv_forward_noalloc", "wkv_forward_noalloc_scratch_bytes", "wkv_backward",
-           "wkv_backward_workspace_bytes", "wkv_strerror", "wkv_last_cuda_error", "wkv_abi_version")
+           "wkv_backward_workspace_bytes", "wkv_token_shift", "wkv_strerror", "wkv_last_cuda_error",
+           "wkv_abi_version")
 
 _lib = None
 _lock = threading.Lock()
@@ -71,6 +72,8 @@ def lib():
         L.wkv_workspace_status.restype = i32
         L.wkv_step.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.wkv_step.restype = i32
+        L.wkv_token_shift.argtypes = [i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.wkv_token_shift.restype = i32
         L.wkv_forward_noalloc.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.wkv_forward_noalloc.restype = i32
         L.wkv_forward_noalloc_scratch_bytes.argtypes = [i64, i64, i64, i32]
@@ -296,6 +299,35 @@ def wkv_backward(w, u, k, v, r=None, state_in=None, *, dy, dstate_out=None, dk=N
                               _ptr(dy), _ptr(dstate_out), _ptr(dk), _ptr(dv), _ptr(dr), _ptr(dw), _ptr(du),
                               _ptr(dstate_in), ws_ptr, ws_bytes, sp), "wkv_backward")
     return dk, dv, dr, dw, du, dstate_in
+
+
+def wkv_token_shift(x, mu, x_prev=None, *, out=None, x_last=None, want_last=True, stream=None):
+    """Token shift: x (B, T, C) float32 or bfloat16, mu (nmix, C) float32,
+    x_prev (B, C) of x's dtype or None (zeros).  Returns (out, x_last) with
+    out[m, b, t] = mu[m] * x[b, t] + (1 - mu[m]) * x[b, t - 1] (nmix, B, T, C)
+    and x_last = x[:, T - 1] (B, C), the next call's x_prev; x_last may be
+    x_prev for an in-place update."""
+    torch = _torch()
+    if x.dim() != 3 or mu.dim() != 2:
+        raise ValueError("x must be (B, T, C) and mu (nmix, C)")
+    B, T, C = x.shape
+    nmix = mu.shape[0]
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("wkv_token_shift runs on CUDA tensors only")
+    code = _dtype_code(x)
+    _need(x, "x", (B, T, C), x.dtype, dev)
+    _need(mu, "mu", (nmix, C), torch.float32, dev)
+    _need(x_prev, "x_prev", (B, C), x.dtype, dev)
+    if out is None:
+        out = torch.empty((nmix, B, T, C), dtype=x.dtype, device=dev)
+    _need(out, "out", (nmix, B, T, C), x.dtype, dev)
+    if x_last is None and want_last:
+        x_last = torch.empty((B, C), dtype=x.dtype, device=dev)
+    _need(x_last, "x_last", (B, C), x.dtype, dev)
+    _check(lib().wkv_token_shift(B, T, C, code, nmix, _ptr(x), _ptr(mu), _ptr(x_prev), _ptr(out), _ptr(x_last),
+                                 _stream_ptr(stream, dev)), "wkv_token_shift")
+    return out, x_last
 
 
 def wkv_step(w, u, k, v, state, r=None, *, y=None, stream=None):

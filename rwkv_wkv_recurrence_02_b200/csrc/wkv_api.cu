@@ -20,6 +20,7 @@
 #include "wkv_backward.cuh"
 #include "wkv_seq.cuh"
 #include "wkv_step.cuh"
+#include "wkv_shift.cuh"
 
 namespace {
 
@@ -487,6 +488,30 @@ int launch_step(int64_t L, int64_t B, int64_t C, const float* w, const float* u,
                                           static_cast<const IO*>(r), state, static_cast<IO*>(y)));
 }
 
+// Token shift: one thread per (sequence, kShiftTS tokens, V channels).
+constexpr int kShiftTS = 8;
+
+template <typename IO, int V>
+int launch_shift(int64_t B, int64_t T, int64_t C, int nmix, const void* x, const float* mu, const void* x_prev,
+                 void* out, void* x_last, cudaStream_t st) {
+    const int64_t units = B * ((T + kShiftTS - 1) / kShiftTS) * (C / V);
+    const int threads = 256;
+    const int64_t blocks = (units + threads - 1) / threads;
+    if (blocks > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(threads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return record_cuda(cudaLaunchKernelEx(&cfg, wkv::token_shift_kernel<IO, V, kShiftTS>, B, T, C, nmix,
+                                          static_cast<const IO*>(x), mu, static_cast<const IO*>(x_prev),
+                                          static_cast<IO*>(out), static_cast<IO*>(x_last)));
+}
+
 }  // namespace
 
 extern "C" {
@@ -695,6 +720,43 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype, const float* w, const f
     else
         rc = V == 2 ? WKV_STEP(__nv_bfloat16, 2) : WKV_STEP(__nv_bfloat16, 1);
 #undef WKV_STEP
+    return rc != WKV_OK ? rc : check_launch();
+}
+
+int wkv_token_shift(int64_t B, int64_t T, int64_t C, int dtype, int nmix, const void* x, const float* mu,
+                    const void* x_prev, void* out, void* x_last, cudaStream_t stream) {
+    if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n) || nmix < 1 || nmix > wkv::kShiftMaxMix || n > kMaxElems / nmix) return WKV_ERR_SHAPE;
+    if (B == 0 || C == 0) return WKV_OK;
+    const size_t eb = elem_bytes(dtype);
+    const size_t lane_bytes = size_t(B) * C * eb, io_bytes = size_t(n) * eb;
+    const size_t out_bytes = io_bytes * nmix, mu_bytes = size_t(nmix) * C * 4;
+    if (!aligned(x, eb) || !aligned(mu, 4) || !aligned(out, eb) || !aligned(x_prev, eb) || !aligned(x_last, eb))
+        return WKV_ERR_ALIGN;
+    if (x_last && x_prev && x_last != x_prev && overlaps(x_last, lane_bytes, x_prev, lane_bytes))
+        return WKV_ERR_ALIAS;
+    if (T == 0) {
+        if (x_last == nullptr || x_last == x_prev) return WKV_OK;
+        if (x_prev == nullptr) return record_cuda(cudaMemsetAsync(x_last, 0, lane_bytes, stream));
+        return record_cuda(cudaMemcpyAsync(x_last, x_prev, lane_bytes, cudaMemcpyDeviceToDevice, stream));
+    }
+    if (!x || !mu || !out) return WKV_ERR_NULLPTR;
+    if (overlaps(out, out_bytes, x, io_bytes) || overlaps(out, out_bytes, mu, mu_bytes) ||
+        overlaps(out, out_bytes, x_prev, lane_bytes) || overlaps(out, out_bytes, x_last, lane_bytes))
+        return WKV_ERR_ALIAS;
+    if (overlaps(x_last, lane_bytes, x, io_bytes) || overlaps(x_last, lane_bytes, mu, mu_bytes)) return WKV_ERR_ALIAS;
+    // 16-byte accesses when every array and row allows them
+    const int64_t vw = static_cast<int64_t>(16 / eb);
+    const bool vec = C % vw == 0 && aligned(x, 16) && aligned(mu, 16) && aligned(out, 16) &&
+                     (x_prev == nullptr || aligned(x_prev, 16)) && (x_last == nullptr || aligned(x_last, 16));
+    int rc;
+    if (dtype == WKV_F32)
+        rc = vec ? launch_shift<float, 4>(B, T, C, nmix, x, mu, x_prev, out, x_last, stream)
+                 : launch_shift<float, 1>(B, T, C, nmix, x, mu, x_prev, out, x_last, stream);
+    else
+        rc = vec ? launch_shift<__nv_bfloat16, 8>(B, T, C, nmix, x, mu, x_prev, out, x_last, stream)
+                 : launch_shift<__nv_bfloat16, 1>(B, T, C, nmix, x, mu, x_prev, out, x_last, stream);
     return rc != WKV_OK ? rc : check_launch();
 }
 

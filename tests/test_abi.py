@@ -184,3 +184,25 @@ def test_backward_validation(L):
     assert bwd(L, ws=None) == WORKSPACE
     assert bwd(L, ws_bytes=L.wkv_backward_workspace_bytes(2, 100, 64, F32) - 1) == WORKSPACE
     assert bwd(L, ws=BASE + (7 << 30) + 16) == ALIGN
+
+
+def test_token_shift_validation(L):
+    ts = L.wkv_token_shift
+    x, mu, xp, out, xl = BASE, BASE + (1 << 36), BASE + (2 << 36), BASE + (3 << 36), BASE + (4 << 36)
+    assert ts(2, 8, 64, 7, 3, x, mu, xp, out, xl, None) == DTYPE
+    assert ts(-1, 8, 64, F32, 3, x, mu, xp, out, xl, None) == SHAPE
+    assert ts(2, 8, 64, F32, 0, x, mu, xp, out, xl, None) == SHAPE          # nmix 1..8
+    assert ts(2, 8, 64, F32, 9, x, mu, xp, out, xl, None) == SHAPE
+    assert ts(1 << 30, 1 << 30, 8, F32, 1, x, mu, xp, out, xl, None) == SHAPE
+    assert ts(0, 8, 64, F32, 3, None, None, None, None, None, None) == OK    # nothing to do
+    assert ts(2, 8, 64, F32, 3, None, mu, xp, out, xl, None) == NULLPTR
+    assert ts(2, 8, 64, F32, 3, x, None, xp, out, xl, None) == NULLPTR
+    assert ts(2, 8, 64, F32, 3, x, mu, xp, None, xl, None) == NULLPTR
+    assert ts(2, 8, 64, F32, 3, x + 2, mu, xp, out, xl, None) == ALIGN
+    assert ts(2, 8, 64, BF16, 3, x, mu + 2, xp, out, xl, None) == ALIGN
+    assert ts(2, 8, 64, BF16, 3, x, mu, xp + 1, out, xl, None) == ALIGN
+    assert ts(2, 8, 64, F32, 3, x, mu, xp, x + 64, xl, None) == ALIAS           # out over x
+    assert ts(2, 8, 64, F32, 3, x, mu, xp, out, out + 4096, None) == ALIAS      # x_last inside out
+    assert ts(2, 8, 64, F32, 3, x, mu, xp, out, x, None) == ALIAS               # x_last over x
+    assert ts(2, 8, 64, F32, 3, x, mu, xp, out, xp + 4, None) == ALIAS          # x_last partly over x_prev
+    assert ts(2, 8, 64, F32, 3, x, mu, xp, xp, xl, None) == ALIAS               # out over x_prev

@@ -180,3 +180,21 @@ def test_decode_e2e_bytes():
     assert e["h2d"] == 3 * wl.layers * wl.B * wl.C * el
     assert e["d2h"] == wl.layers * wl.B * wl.C * el
     assert calls == [1] * (wl.layers * 4) and "wkv_step" in e["path"]
+
+
+def test_token_shift_bytes_and_reference_arm(capsys):
+    """Token-shift byte accounting, and its reference arm (the oracle on a
+    channel sample) prints one line with the op's metric."""
+    wl = I.WORKLOADS["layer_14b"]
+    n = 4 * 8192 * 5120
+    assert bench.algorithmic_bytes_shift(wl, 4, 8192, 5120) == n * 2 * 4 + 2 * 4 * 5120 * 2 + 3 * 5120 * 4
+    bench.main(["--impl", "reference", "--op", "token_shift", "--workload", "decode", "--steps", "3",
+                "--warmup", "3", "--ref-budget-s", "2"])
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC_SHIFT and line["value"] > 0
+    assert line["config"]["T"] == 1 and line["config"]["op"] == "token_shift"
+
+
+def test_token_shift_cpu_baseline_is_bounded():
+    r = bench.cpu_baseline_shift("layer_1b5", 0.5)
+    assert r["value"] > 0 and r["kind"] == "oracle" and "mixes" in r["sample"]
