@@ -67,6 +67,23 @@ def test_traffic_record_invalidated_by_source_change(tmp_path, monkeypatch):
     assert bench.load_traffic("layer_1b5") == 123
 
 
+def test_traffic_hash_scopes(tmp_path, monkeypatch):
+    """A WKV kernel's record does not depend on the token-shift-only sources;
+    the token shift's record depends on every source."""
+    csrc = tmp_path / "csrc"
+    csrc.mkdir()
+    (csrc / "wkv_api.cu").write_text("api")
+    (csrc / "wkv_lane.cuh").write_text("lane")
+    (csrc / "wkv_shift.cuh").write_text("shift v1")
+    monkeypatch.setattr(bench, "CSRC", str(csrc))
+    wkv1, ts1 = bench.kernel_source_hash("lane_forward"), bench.kernel_source_hash("token_shift")
+    (csrc / "wkv_shift.cuh").write_text("shift v2")
+    assert bench.kernel_source_hash("lane_forward") == wkv1
+    assert bench.kernel_source_hash("token_shift") != ts1
+    (csrc / "wkv_lane.cuh").write_text("lane v2")
+    assert bench.kernel_source_hash("lane_forward") != wkv1
+
+
 def _rank_main(rank, world, port, q):
     import torch.distributed as dist
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
