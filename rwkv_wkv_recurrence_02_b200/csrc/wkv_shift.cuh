@@ -5,7 +5,10 @@
 // A thread owns V consecutive channels (16 bytes of one row) of one sequence
 // over TS consecutive tokens: it reads the row before its first token once
 // (x_prev for the first tokens of the sequence), keeps the previous row in
-// registers, and writes nmix output rows per token.  Units run channel group
+// registers, and writes nmix output rows per token.  A whole unit issues its
+// TS row loads before using the first (6% faster than loading each row when
+// it is needed, on the 14B layer shape); a partial unit at the end of a
+// sequence loads row by row.  Units run channel group
 // fastest, so a warp's accesses to every array are contiguous.  The thread
 // that owns a sequence's first tokens also writes x_last, after reading
 // x_prev, so x_last may be x_prev itself.
@@ -21,15 +24,22 @@ template <typename IO, int V>
 struct ShiftVec;
 
 // load: read-only path (x, mu); load_rw: plain load (x_prev, which this
-// kernel may overwrite as x_last)
+// kernel may overwrite as x_last); load_raw + widen_raw: a read-only load
+// kept packed in registers and widened when it is used
 template <>
 struct ShiftVec<float, 1> {
+    using Raw = float;
+    static __device__ __forceinline__ Raw load_raw(const float* p) { return __ldg(p); }
+    static __device__ __forceinline__ void widen_raw(Raw v, float* o) { o[0] = v; }
     static __device__ __forceinline__ void load(const float* p, float* o) { o[0] = __ldg(p); }
     static __device__ __forceinline__ void load_rw(const float* p, float* o) { o[0] = *p; }
     static __device__ __forceinline__ void store(float* p, const float* o) { *p = o[0]; }
 };
 template <>
 struct ShiftVec<float, 4> {
+    using Raw = float4;
+    static __device__ __forceinline__ Raw load_raw(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+    static __device__ __forceinline__ void widen_raw(Raw v, float* o) { o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w; }
     static __device__ __forceinline__ void load(const float* p, float* o) {
         const float4 v = __ldg(reinterpret_cast<const float4*>(p));
         o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w;
@@ -44,12 +54,18 @@ struct ShiftVec<float, 4> {
 };
 template <>
 struct ShiftVec<__nv_bfloat16, 1> {
+    using Raw = __nv_bfloat16;
+    static __device__ __forceinline__ Raw load_raw(const __nv_bfloat16* p) { return __ldg(p); }
+    static __device__ __forceinline__ void widen_raw(Raw v, float* o) { o[0] = __bfloat162float(v); }
     static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* o) { o[0] = __bfloat162float(__ldg(p)); }
     static __device__ __forceinline__ void load_rw(const __nv_bfloat16* p, float* o) { o[0] = __bfloat162float(*p); }
     static __device__ __forceinline__ void store(__nv_bfloat16* p, const float* o) { *p = __float2bfloat16_rn(o[0]); }
 };
 template <>
 struct ShiftVec<__nv_bfloat16, 8> {
+    using Raw = uint4;
+    static __device__ __forceinline__ Raw load_raw(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+    static __device__ __forceinline__ void widen_raw(Raw v, float* o) { widen(v, o); }
     static __device__ __forceinline__ void widen(uint4 v, float* o) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -104,6 +120,31 @@ token_shift_kernel(int64_t B, int64_t T, int64_t C, int nmix, const IO* __restri
         for (int j = 0; j < V; ++j) prev[j] = 0.f;
     }
     const int64_t plane = B * T * C;
+    if (t1 - t0 == TS) {
+        // a whole unit: all TS rows in flight before the first is used
+        typename ShiftVec<IO, V>::Raw raw[TS];
+#pragma unroll
+        for (int i = 0; i < TS; ++i) raw[i] = ShiftVec<IO, V>::load_raw(x + (b * T + t0 + i) * C + c);
+#pragma unroll
+        for (int i = 0; i < TS; ++i) {
+            float cur[V];
+            ShiftVec<IO, V>::widen_raw(raw[i], cur);
+#pragma unroll
+            for (int m = 0; m < kShiftMaxMix; ++m) {
+                if (m < nmix) {
+                    // mu of the unit's channels (L1-resident after the first token)
+                    float mm[V], o[V];
+                    ShiftVec<float, V == 8 ? 4 : V>::load(mu + m * C + c, mm);
+                    if constexpr (V == 8) ShiftVec<float, 4>::load(mu + m * C + c + 4, mm + 4);
+#pragma unroll
+                    for (int j = 0; j < V; ++j) o[j] = fmaf(mm[j], cur[j], (1.f - mm[j]) * prev[j]);
+                    ShiftVec<IO, V>::store(out + m * plane + (b * T + t0 + i) * C + c, o);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < V; ++j) prev[j] = cur[j];
+        }
+    } else
     for (int64_t t = t0; t < t1; ++t) {
         float cur[V];
         ShiftVec<IO, V>::load(x + (b * T + t) * C + c, cur);
