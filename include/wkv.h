@@ -161,8 +161,11 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype,
  *   - Limit: problems whose scratch need (wkv_forward_noalloc_scratch_bytes)
  *     exceeds WKV_NOALLOC_SCRATCH_BYTES are rejected with WKV_ERR_SCRATCH
  *     before anything runs.  Sequences of at most 64 tokens need none, and
- *     neither do calls that fit the cluster kernel (described under
- *     wkv_forward's workspace): those share no array and need no ordering.
+ *     neither do TMA-eligible calls of at most 1024 tokens, which run the
+ *     cluster kernel (described under wkv_forward's workspace): those share
+ *     no array and need no ordering.  (A wkv_forward call with a NULL
+ *     workspace takes the cluster kernel from 17 tokens on, also where the
+ *     required size is 0.)
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before capturing a stream into a graph.

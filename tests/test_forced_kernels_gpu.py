@@ -3,6 +3,8 @@ forces one kernel (environment knob read once per process), runs a list of
 shapes through wkv_forward and saves the results; this process compares them
 with the oracle on the same seeded inputs.
 
+- part: short sequences of few lane blocks, which take the cluster kernel
+  when the call brings no workspace (at most 64 tokens need none);
 - cluster: many lane blocks (more clusters than fit the GPU at once), which
   with a workspace take the lane-resident kernel.
 """
@@ -35,6 +37,15 @@ torch.save(res, out)
 """
 
 FORCED = {
+    "part": [
+        # B, T, C, dtype, gate, state
+        (1, 17, 64, "float32", True, True),
+        (1, 64, 64, "bfloat16", False, True),
+        (1, 65, 128, "float32", True, False),
+        (1, 129, 128, "float32", True, False),
+        (2, 1000, 72, "bfloat16", True, True),
+        (3, 777, 1000, "bfloat16", False, True),
+    ],
     "cluster": [
         (40, 130, 256, "bfloat16", True, False),     # 160 lane blocks
         (160, 64, 64, "float32", False, True),

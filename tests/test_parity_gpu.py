@@ -98,7 +98,10 @@ def test_lane_resident_shapes(B, T, C, dtype, gate, state):
 
 
 # Fewer 64-channel blocks than SMs: the part kernel cuts every sequence into
-# 64-token parts that find their entering state by look-back.
+# 64-token parts that find their entering state by look-back.  (Calls of at
+# most 64 tokens need no workspace, so the binding brings none and they take
+# the cluster kernel; tests/test_forced_kernels_gpu.py forces the part kernel
+# on short sequences.)
 PART = [
     # B, T, C, dtype, gate, state
     (1, 17, 64, torch.float32, True, True),        # a single part, shorter than a part
@@ -121,14 +124,14 @@ def test_part_shapes(B, T, C, dtype, gate, state):
     check_forward(d, y, s)
 
 
-# Calls without a workspace whose sequences fit one cluster (at most 1024
+# Calls without a workspace whose sequences fit one cluster (17 to 1024
 # tokens): the cluster kernel, one cluster of ceil(T / 128) CTAs per lane
 # block whose parts exchange their summaries through distributed shared
 # memory.  wkv_forward_noalloc brings no workspace.
 CLUSTER = [
     # B, T, C, dtype, gate, state
-    (1, 17, 64, torch.float32, True, True),        # a cluster of one CTA, shorter than a part
-    (1, 64, 64, torch.bfloat16, False, True),
+    (1, 100, 64, torch.float32, True, True),       # a cluster of one CTA, shorter than a part
+    (1, 66, 64, torch.bfloat16, False, True),
     (1, 128, 64, torch.bfloat16, False, True),     # exactly one part
     (1, 129, 128, torch.float32, True, False),     # one token in the second part
     (1, 65, 128, torch.float32, True, True),
