@@ -149,7 +149,7 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype,
  * memory: code running where cudaMalloc is unavailable or forbidden (a
  * plug-in inside a host application that owns every allocation, a runtime
  * that hands out only pre-registered buffers, or a pre-recorded launch
- * sequence that must not touch the allocator).  The paper has no counterpart
+ * sequence that must not touch the allocator).  The article has no counterpart
  * to this entry point; it only changes where the scratch memory comes from.
  *
  * Same arguments and results as wkv_forward, without the workspace.  The

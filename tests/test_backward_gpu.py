@@ -3,7 +3,7 @@ reverse mode, on identical seeded inputs.
 
 Errors are measured per lane: the largest |gpu - oracle| over a lane's tokens
 divided by the largest |oracle| of that lane, so a small gradient next to a
-large one in the same lane is judged at the lane's scale.  dw, du and the
+large one in the same lane is measured at the lane's scale.  dw, du and the
 state's gradient are divided by the larger of their own largest |oracle| and
 the call's largest |dv|.
 """
@@ -62,7 +62,7 @@ def check(d, out, tol=None):
     if rr is not None:
         errs["dr"] = lane_error(dr, rr)
     # sums over many tokens can cancel to ~0 (T = 1 from the empty state:
-    # du = 0 exactly), so they are judged at the call's gradient scale too
+    # du = 0 exactly), so they are measured at the call's gradient scale too
     g_scale = max(np.abs(rv).max(), 1e-30)
     errs["dw"] = float(np.abs(to_np64(dw) - rw).max() / max(np.abs(rw).max(), g_scale))
     errs["du"] = float(np.abs(to_np64(du) - ru).max() / max(np.abs(ru).max(), g_scale))
