@@ -206,3 +206,14 @@ def test_token_shift_validation(L):
     assert ts(2, 8, 64, F32, 3, x, mu, xp, out, x, None) == ALIAS               # x_last over x
     assert ts(2, 8, 64, F32, 3, x, mu, xp, out, xp + 4, None) == ALIAS          # x_last partly over x_prev
     assert ts(2, 8, 64, F32, 3, x, mu, xp, xp, xl, None) == ALIAS               # out over x_prev
+
+
+def test_token_shift_front_end_refuses_bad_arguments():
+    import torch
+    x = torch.zeros(2, 4, 8)
+    with pytest.raises(ValueError):
+        wkv.wkv_token_shift(x, torch.rand(3, 8))                       # CPU tensors
+    with pytest.raises(ValueError):
+        wkv.wkv_token_shift(torch.zeros(4, 8), torch.rand(3, 8))       # x not (B, T, C)
+    with pytest.raises(ValueError):
+        wkv.wkv_token_shift(x, torch.rand(8))                          # mu not (nmix, C)
