@@ -63,7 +63,7 @@ typedef enum {
     WKV_ERR_ALIAS = -5,      /* an output overlaps an input or another output */
     WKV_ERR_CUDA = -6,       /* CUDA launch error; see wkv_last_cuda_error() */
     WKV_ERR_TIMEOUT = -7,    /* a cross-block wait on the GPU gave up (from wkv_workspace_status) */
-    WKV_ERR_WORKSPACE = -8,  /* workspace NULL or smaller than wkv_forward_workspace_bytes() */
+    WKV_ERR_WORKSPACE = -8,  /* wkv_backward: workspace NULL or smaller than wkv_backward_workspace_bytes() */
     WKV_ERR_SCRATCH = -9     /* wkv_forward_noalloc: problem needs more than its built-in scratch */
 } wkv_status;
 
@@ -88,21 +88,35 @@ typedef enum {
  *   state_out    (3,B,C) float32 device array, or NULL.  May be the same
  *                pointer as state_in (in-place update); any other overlap
  *                with an input or with y is WKV_ERR_ALIAS.
- *   workspace    device scratch of at least wkv_forward_workspace_bytes(B,T,C,
- *                dtype) bytes, 256-byte aligned, zeroed once by
- *                wkv_workspace_init() before its first use and reusable by any
- *                later call with any shape.  May be NULL when the required
- *                size is 0.  Calls sharing a workspace must be ordered on the
- *                GPU (same stream, or synchronised); they race otherwise.
- *                NULL (or too small) is also accepted when every sequence
- *                fits one cluster of parts: 17 <= T <= 1024, C a multiple of
- *                4 (of 8 for bfloat16), k, v, r, w, u, state_in 16-byte
- *                aligned, y and state_out aligned to two elements.  Such a
- *                call runs the cluster kernel, which needs no scratch (thread
- *                block clusters of ceil(T/128) CTAs that combine their parts'
- *                summaries in distributed shared memory).  Any other call
- *                without an adequate workspace returns WKV_ERR_WORKSPACE.
+ *   workspace    optional device scratch of at least
+ *                wkv_forward_workspace_bytes(B,T,C,dtype) bytes, 256-byte
+ *                aligned, zeroed once by wkv_workspace_init() before its
+ *                first use and reusable by any later call with any shape.
+ *                Calls sharing a workspace must be ordered on the GPU (same
+ *                stream, or synchronised); they race otherwise.  With it,
+ *                CTAs that split one sequence exchange partial states
+ *                through it (decoupled look-back, state hand-off), which is
+ *                the fastest schedule for most shapes.
+ *                NULL (or too small: it is then not touched) is accepted for
+ *                every shape; the call then runs a schedule that needs no
+ *                scratch: the sequential kernel for T <= 16; the cluster
+ *                kernel (thread block clusters of ceil(T/128) CTAs that
+ *                combine their parts' summaries in distributed shared
+ *                memory) when 17 <= T <= 1024, C is a multiple of 4 (of 8
+ *                for bfloat16), k, v, r, w, u, state_in are 16-byte aligned
+ *                and y, state_out aligned to two elements; otherwise, for
+ *                such TMA-eligible arrays, the lane-resident kernel with
+ *                whole sequences' channel blocks per CTA, and for any other
+ *                layout the per-lane recurrence.  Those last two give the
+ *                same results but can be several times slower when there
+ *                are few lanes (one long sequence) or slightly more lane
+ *                blocks than the GPU holds at once.
  *   stream       CUDA stream of the launch.
+ *
+ * The operator's own call is (B, T, C, dtype, w, u, k, v, r, state_in, y,
+ * state_out, stream).  The two workspace arguments are an addition to it: the
+ * library allocates nothing, so the scratch of the fastest schedules has to
+ * come from the caller.  Passing NULL, 0 gives the plain call on every shape.
  */
 int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype,
                 const float* w, const float* u,
@@ -123,6 +137,64 @@ int wkv_workspace_init(void* workspace, size_t bytes, cudaStream_t stream);
  * workspace: WKV_OK, or WKV_ERR_TIMEOUT if a wait for another block's partial
  * result gave up (those outputs were written as NaN). */
 int wkv_workspace_status(const void* workspace, cudaStream_t stream);
+
+/*
+ * wkv_state -- the state a chunk leaves behind, without its outputs.
+ *
+ * state_out = the state after T tokens entered from state_in (NULL: the
+ * empty state): exactly wkv_forward's state_out for the same k, v, w and
+ * state_in, with no y.  The state does not depend on u or on the gate, so
+ * neither is taken.  Entered from the empty state it is the chunk's
+ * summary, the element of the scan that "並列学習の定式化" (article
+ * "RWKVアーキテクチャ徹底解説") says the parallel mode performs: summaries of
+ * consecutive chunks combine associatively (wkv_state_combine).  That is what
+ * lets one sequence be split along T across GPUs ("Process million-token
+ * sequences" on the skill page "rwkv-architecture" streams a long document
+ * through chunks with the state carried): each GPU forms its chunk's summary,
+ * the summaries are exchanged and folded into every chunk's entering state,
+ * and each GPU then runs wkv_forward on its chunk from that state.
+ *
+ *   B, T, C      sizes, each >= 0 (B == 0 or C == 0: nothing to do; T == 0:
+ *                state_out = state_in).
+ *   dtype        wkv_dtype of k and v.
+ *   w            (C,) float32.   k, v: (B,T,C) device arrays.
+ *   state_in     (3,B,C) float32 or NULL.
+ *   state_out    (3,B,C) float32, required; may equal state_in, must not
+ *                overlap anything else.
+ *   workspace    as for wkv_forward (optional; NULL runs a scratch-free
+ *                schedule).
+ * Reads k and v once; writes only state_out.  Errors as wkv_forward.
+ */
+int wkv_state(int64_t B, int64_t T, int64_t C, int dtype, const float* w,
+              const void* k, const void* v, const float* state_in, float* state_out,
+              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * wkv_state_combine -- fold chunk summaries into a state.
+ *
+ * state_out = the state after n consecutive chunks of lens[0], ...,
+ * lens[n-1] tokens entered from state_in (NULL: the empty state), given each
+ * chunk's own summary (wkv_state from the empty state).  With summary
+ * (q, A, B) of a chunk of L tokens and a state (p, a, b) before it, the
+ * state after it is p' = max(p - L w, q), a' = e^{p - L w - p'} a +
+ * e^{q - p'} A, b' likewise: the recurrence of "リカレント定式化" applied to a
+ * whole chunk at once.  Folding is associative, so the result equals one
+ * wkv_state call over the concatenated chunks (up to rounding).
+ *
+ *   B, C         sizes (>= 0).
+ *   n            number of chunks, 0 <= n <= 64 (0: state_out = state_in).
+ *   w            (C,) float32 device array.
+ *   lens         HOST array of n token counts (each >= 0), read during the
+ *                call.
+ *   states       (n,3,B,C) float32 device array of the summaries.
+ *   state_in     (3,B,C) float32 device array or NULL.
+ *   state_out    (3,B,C) float32 device array; may equal state_in, must not
+ *                overlap states or w.
+ * WKV_ERR_SHAPE for n outside 0..64 or a negative length.
+ */
+int wkv_state_combine(int64_t B, int64_t C, int n, const float* w, const int64_t* lens,
+                      const float* states, const float* state_in, float* state_out,
+                      cudaStream_t stream);
 
 /*
  * wkv_step -- RNN ("decode") mode: one token for L independent layers, each
@@ -158,23 +230,28 @@ int wkv_step(int64_t L, int64_t B, int64_t C, int dtype,
  * every GPU which loads the library keeps until the process exits), so
  * nothing is allocated.
  *
+ *   - It runs the kernels wkv_forward runs with a workspace, with the array
+ *     standing in for the workspace.
  *   - Limit: problems whose scratch need (wkv_forward_noalloc_scratch_bytes)
  *     exceeds WKV_NOALLOC_SCRATCH_BYTES are rejected with WKV_ERR_SCRATCH
- *     before anything runs.  Sequences of at most 64 tokens need none, and
- *     neither do TMA-eligible calls of at most 1024 tokens, which run the
- *     cluster kernel (described under wkv_forward's workspace): those share
- *     no array and need no ordering.  (A wkv_forward call with a NULL
- *     workspace takes the cluster kernel from 17 tokens on, also where the
- *     required size is 0.)
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before capturing a stream into a graph.
+ *     before anything runs (wkv_forward with a NULL workspace serves them
+ *     without scratch, more slowly).  Calls whose wkv_forward needs no
+ *     workspace, and TMA-eligible calls of at most 1024 tokens, which run
+ *     the cluster kernel (described under wkv_forward's workspace), use no
+ *     scratch: those share no array and need no ordering.
+ *   - The first call on a device that uses the array looks up its device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before capturing a stream into a graph.  The address is
+ *     kept per device ordinal for the process: it serves the device's
+ *     primary context (the CUDA runtime's) and is not looked up again after
+ *     cudaDeviceReset or for another driver context on the same device.
  *   - Every call on a device shares the one array and clears the part it
  *     uses at the start (a cudaMemsetAsync on `stream`).  Calls that may
  *     overlap on the GPU (different streams without ordering) race on it
  *     and give wrong results; order them.
- *   - A cross-block wait that runs out is recorded in the array like in a
- *     workspace; the next call clears it.
+ *   - A cross-block wait that runs out is recorded in the array's header
+ *     (outputs are NaN then); wkv_forward_noalloc_status() reads it.  The
+ *     next call that uses the array clears it.
  */
 #define WKV_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -188,6 +265,14 @@ int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype,
  * upper bound: calls that take the cluster kernel (see wkv_forward's
  * workspace) use none and are not subject to WKV_NOALLOC_SCRATCH_BYTES. */
 size_t wkv_forward_noalloc_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype);
+
+/* Synchronise `stream`, then read the error word of the built-in array on
+ * the current device: WKV_OK, or WKV_ERR_TIMEOUT if the last
+ * wkv_forward_noalloc call that used the array had a wait for another
+ * block's partial result give up (its outputs were written as NaN).  WKV_OK
+ * when no call on this device has used the array.  Order it after the call
+ * it checks and before the next one that uses the array. */
+int wkv_forward_noalloc_status(cudaStream_t stream);
 
 /*
  * wkv_backward -- gradients of wkv_forward over one chunk (reverse mode).

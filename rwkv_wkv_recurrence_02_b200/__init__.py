@@ -31,7 +31,8 @@ STATUS = {
 }
 # the functions include/wkv.h declares
 EXPORTS = ("wkv_forward", "wkv_forward_workspace_bytes", "wkv_workspace_init", "wkv_workspace_status",
-           "wkv_step", "wkv_forward_noalloc", "wkv_forward_noalloc_scratch_bytes", "wkv_backward",
+           "wkv_step", "wkv_forward_noalloc", "wkv_forward_noalloc_scratch_bytes", "wkv_forward_noalloc_status",
+           "wkv_backward", "wkv_state", "wkv_state_combine",
            "wkv_backward_workspace_bytes", "wkv_token_shift", "wkv_strerror", "wkv_last_cuda_error",
            "wkv_abi_version")
 
@@ -78,6 +79,12 @@ def lib():
         L.wkv_forward_noalloc.restype = i32
         L.wkv_forward_noalloc_scratch_bytes.argtypes = [i64, i64, i64, i32]
         L.wkv_forward_noalloc_scratch_bytes.restype = sz
+        L.wkv_state.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.wkv_state.restype = i32
+        L.wkv_state_combine.argtypes = [i64, i64, i32, vp, vp, vp, vp, vp, vp]
+        L.wkv_state_combine.restype = i32
+        L.wkv_forward_noalloc_status.argtypes = [vp]
+        L.wkv_forward_noalloc_status.restype = i32
         L.wkv_backward.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                    vp, sz, vp]
         L.wkv_backward.restype = i32
@@ -197,11 +204,12 @@ def workspace_bytes(B: int, T: int, C: int, dtype_code: int) -> int:
 
 
 def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, want_state=True,
-                workspace: Workspace = None, stream=None):
+                workspace: Workspace = None, use_workspace=True, stream=None):
     """Parallel mode over one chunk.  k, v, r: (B, T, C) CUDA tensors (float32
     or bfloat16); w, u: (C,) float32; state_in: (3, B, C) float32 or None.
     Returns (y, state_out) (state_out None if want_state is False and none
-    was given).  state_out may be state_in for an in-place update."""
+    was given).  state_out may be state_in for an in-place update.
+    use_workspace=False passes no workspace (the scratch-free schedules)."""
     torch = _torch()
     if k.dim() != 3:
         raise ValueError("k must be (B, T, C)")
@@ -222,9 +230,12 @@ def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, wa
     if state_out is None and want_state:
         state_out = torch.empty((3, B, C), dtype=torch.float32, device=dev)
     _need(state_out, "state_out", (3, B, C), torch.float32, dev)
-    ws = workspace if workspace is not None else default_workspace(dev)
     sp = _stream_ptr(stream, dev)
-    ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
+    if use_workspace:
+        ws = workspace if workspace is not None else default_workspace(dev)
+        ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
+    else:
+        ws_ptr, ws_bytes = None, 0
     _check(lib().wkv_forward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
                              _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, sp), "wkv_forward")
     return y, state_out
@@ -249,6 +260,69 @@ def wkv_forward_noalloc(w, u, k, v, r=None, state_in=None, *, y, state_out=None,
     _check(lib().wkv_forward_noalloc(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
                                      _ptr(y), _ptr(state_out), _stream_ptr(stream, dev)), "wkv_forward_noalloc")
     return y, state_out
+
+
+def wkv_state(w, k, v, state_in=None, *, state_out=None, workspace: Workspace = None, use_workspace=True,
+              stream=None):
+    """State after the chunk k, v (B, T, C) entered from state_in (None: the
+    empty state), without outputs; from the empty state it is the chunk's
+    summary.  Returns state_out (3, B, C) float32 (may be state_in)."""
+    torch = _torch()
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    dev = k.device
+    if dev.type != "cuda":
+        raise ValueError("wkv_state runs on CUDA tensors only")
+    code = _dtype_code(k)
+    _need(v, "v", (B, T, C), k.dtype, dev)
+    _need(w, "w", (C,), torch.float32, dev)
+    _need(k, "k", (B, T, C), k.dtype, dev)
+    _need(state_in, "state_in", (3, B, C), torch.float32, dev)
+    if state_out is None:
+        state_out = torch.empty((3, B, C), dtype=torch.float32, device=dev)
+    _need(state_out, "state_out", (3, B, C), torch.float32, dev)
+    sp = _stream_ptr(stream, dev)
+    if use_workspace:
+        ws = workspace if workspace is not None else default_workspace(dev)
+        ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
+    else:
+        ws_ptr, ws_bytes = None, 0
+    _check(lib().wkv_state(B, T, C, code, _ptr(w), _ptr(k), _ptr(v), _ptr(state_in), _ptr(state_out), ws_ptr,
+                           ws_bytes, sp), "wkv_state")
+    return state_out
+
+
+def wkv_state_combine(w, lens, states, state_in=None, *, state_out=None, stream=None):
+    """Fold the summaries states (n, 3, B, C) of n consecutive chunks of
+    lens[j] tokens into the state entering from state_in (None: empty).
+    Returns state_out (3, B, C)."""
+    torch = _torch()
+    n = len(lens)
+    if states.dim() != 4 or states.shape[0] < n or states.shape[1] != 3:
+        raise ValueError("states must be (n, 3, B, C)")
+    _, _, B, C = states.shape
+    dev = states.device
+    if dev.type != "cuda":
+        raise ValueError("wkv_state_combine runs on CUDA tensors only")
+    _need(states, "states", tuple(states.shape), torch.float32, dev)
+    _need(w, "w", (C,), torch.float32, dev)
+    _need(state_in, "state_in", (3, B, C), torch.float32, dev)
+    if state_out is None:
+        state_out = torch.empty((3, B, C), dtype=torch.float32, device=dev)
+    _need(state_out, "state_out", (3, B, C), torch.float32, dev)
+    arr = (ctypes.c_int64 * max(1, n))(*[int(x) for x in lens])
+    _check(lib().wkv_state_combine(B, C, n, _ptr(w), arr, _ptr(states), _ptr(state_in), _ptr(state_out),
+                                   _stream_ptr(stream, dev)), "wkv_state_combine")
+    return state_out
+
+
+def wkv_forward_noalloc_status(stream=None, device=None) -> int:
+    """Synchronise the stream and return the error word of the library's
+    built-in scratch array on the current device: 0, or WKV_ERR_TIMEOUT (-7)
+    if the last wkv_forward_noalloc call that used it had a cross-block wait
+    give up."""
+    return int(lib().wkv_forward_noalloc_status(_stream_ptr(stream, device)))
 
 
 @functools.lru_cache(maxsize=1024)

@@ -300,13 +300,14 @@ int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
     }
     const int64_t grid = a.nLB < capacity[dev] ? a.nLB : capacity[dev];
     // fewer CTAs than lane blocks: equal shares of the chunk order, with one
-    // state handed between neighbouring CTAs through the workspace
-    if (grid < a.nLB && a.nchunks > 1) {
-        if (workspace == nullptr) return WKV_ERR_WORKSPACE;
+    // state handed between neighbouring CTAs through the workspace.  Without
+    // an adequate workspace (the forward only) every CTA takes whole lane
+    // blocks instead (no hand-off; shares differ by up to one lane block).
+    const bool ws_adequate = workspace != nullptr && workspace_bytes >= 256 + size_t(a.nLB) * G::CB * sizeof(wkv::Word) &&
+                             (CKPT || workspace_bytes >= wkv_forward_workspace_bytes(a.B, a.T, a.C, dtype));
+    if (grid < a.nLB && a.nchunks > 1 && (CKPT || ws_adequate)) {
+        if (!ws_adequate) return WKV_ERR_WORKSPACE;
         if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
-        if (workspace_bytes < 256 + size_t(a.nLB) * G::CB * sizeof(wkv::Word) ||
-            (!CKPT && workspace_bytes < wkv_forward_workspace_bytes(a.B, a.T, a.C, dtype)))
-            return WKV_ERR_WORKSPACE;
         a.hdr = reinterpret_cast<wkv::WsHeader*>(workspace);
         a.incw = reinterpret_cast<wkv::Word*>(static_cast<char*>(workspace) + 256);
     } else {
@@ -512,6 +513,40 @@ int launch_shift(int64_t B, int64_t T, int64_t C, int nmix, const void* x, const
                                           static_cast<IO*>(out), static_cast<IO*>(x_last)));
 }
 
+// Host-side checks of a forward call with T >= 1 and B, C >= 1: required
+// pointers, alignment to the element types, and overlaps (y must be disjoint
+// from every input and from state_out; state_out may equal state_in but
+// overlap nothing else).
+int forward_args(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u, const void* k,
+                 const void* v, const void* r, const float* state_in, const void* y, const float* state_out) {
+    const size_t eb = elem_bytes(dtype);
+    const size_t io_bytes = size_t(B) * size_t(T) * size_t(C) * eb, st_bytes = size_t(B) * size_t(C) * 3 * 4,
+                 p_bytes = size_t(C) * 4;
+    if (!w || !u || !k || !v || !y) return WKV_ERR_NULLPTR;
+    if (!aligned(w, 4) || !aligned(u, 4) || !aligned(k, eb) || !aligned(v, eb) || !aligned(y, eb) ||
+        (r && !aligned(r, eb)) || (state_in && !aligned(state_in, 4)) || (state_out && !aligned(state_out, 4)))
+        return WKV_ERR_ALIGN;
+    const void* ins[] = {k, v, r};
+    for (const void* p : ins)
+        if (overlaps(y, io_bytes, p, io_bytes)) return WKV_ERR_ALIAS;
+    if (overlaps(y, io_bytes, w, p_bytes) || overlaps(y, io_bytes, u, p_bytes) ||
+        overlaps(y, io_bytes, state_in, st_bytes) || overlaps(y, io_bytes, state_out, st_bytes))
+        return WKV_ERR_ALIAS;
+    if (state_out) {
+        for (const void* p : ins)
+            if (overlaps(state_out, st_bytes, p, io_bytes)) return WKV_ERR_ALIAS;
+        if (overlaps(state_out, st_bytes, w, p_bytes) || overlaps(state_out, st_bytes, u, p_bytes))
+            return WKV_ERR_ALIAS;
+        if (state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes))
+            return WKV_ERR_ALIAS;
+    }
+    return WKV_OK;
+}
+
+int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u, const void* k,
+                const void* v, const void* r, const float* state_in, void* y, float* state_out, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream);
+
 }  // namespace
 
 extern "C" {
@@ -572,8 +607,7 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
     if (B == 0 || C == 0) return WKV_OK;
     const int64_t lanes = B * C;
-    const size_t eb = elem_bytes(dtype);
-    const size_t io_bytes = size_t(n) * eb, st_bytes = size_t(lanes) * 3 * 4, p_bytes = size_t(C) * 4;
+    const size_t st_bytes = size_t(lanes) * 3 * 4;
     if (T == 0) {
         if (state_out == nullptr) return WKV_OK;
         if (!aligned(state_out, 4) || (state_in && !aligned(state_in, 4))) return WKV_ERR_ALIGN;
@@ -584,26 +618,20 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
             lanes, state_in, state_out);
         return check_launch();
     }
-    if (!w || !u || !k || !v || !y) return WKV_ERR_NULLPTR;
-    if (!aligned(w, 4) || !aligned(u, 4) || !aligned(k, eb) || !aligned(v, eb) || !aligned(y, eb) ||
-        (r && !aligned(r, eb)) || (state_in && !aligned(state_in, 4)) || (state_out && !aligned(state_out, 4)))
-        return WKV_ERR_ALIGN;
-    // y must be disjoint from every input and from state_out
-    const void* ins[] = {k, v, r};
-    for (const void* p : ins)
-        if (overlaps(y, io_bytes, p, io_bytes)) return WKV_ERR_ALIAS;
-    if (overlaps(y, io_bytes, w, p_bytes) || overlaps(y, io_bytes, u, p_bytes) ||
-        overlaps(y, io_bytes, state_in, st_bytes) || overlaps(y, io_bytes, state_out, st_bytes))
-        return WKV_ERR_ALIAS;
-    if (state_out) {
-        for (const void* p : ins)
-            if (overlaps(state_out, st_bytes, p, io_bytes)) return WKV_ERR_ALIAS;
-        if (overlaps(state_out, st_bytes, w, p_bytes) || overlaps(state_out, st_bytes, u, p_bytes))
-            return WKV_ERR_ALIAS;
-        if (state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes))
-            return WKV_ERR_ALIAS;
-    }
+    const int vrc = forward_args(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out);
+    if (vrc != WKV_OK) return vrc;
+    return run_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, workspace, workspace_bytes, stream);
+}
 
+}  // extern "C"
+
+namespace {
+
+// Kernel choice and launch of a forward call whose arguments passed the host
+// checks (B, C, T >= 1).  y == nullptr: only the state is wanted.
+int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u, const void* k,
+                const void* v, const void* r, const float* state_in, void* y, float* state_out, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
     const void* io[] = {k, v, r, y};
     const float* f32[] = {w, u, state_in, state_out};
     const int V = pick_vec(C, dtype, io, 4, f32, 4);
@@ -641,6 +669,30 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
             return dtype == WKV_F32
                        ? dispatch_cluster<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
                        : dispatch_cluster<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
+        }
+        // No adequate workspace and no cluster fits: schedules that need no
+        // scratch.  TMA-eligible calls take the lane-resident kernel over
+        // whole lane blocks; any other layout walks the plain recurrence per
+        // lane (the sequential kernel takes any T and any alignment).
+        if (force == 0 && !ws_ok) {
+            if (!tma) {
+                if (B * (C / V) > int64_t(0x7fffffff) * 256) return WKV_ERR_SHAPE;
+                if (dtype == WKV_F32) {
+                    if (V == 2) dispatch_forward<float, 2>(r != nullptr, true, a, 0, stream);
+                    else dispatch_forward<float, 1>(r != nullptr, true, a, 0, stream);
+                } else {
+                    if (V == 2) dispatch_forward<__nv_bfloat16, 2>(r != nullptr, true, a, 0, stream);
+                    else dispatch_forward<__nv_bfloat16, 1>(r != nullptr, true, a, 0, stream);
+                }
+                return check_launch();
+            }
+            const ChunkGeom g = chunk_geom(B, T, C, 2, kLaneW * kLaneLS);
+            a.nCB = g.nCB;
+            a.nLB = g.nLB;
+            a.nchunks = g.nchunks;
+            a.units = g.units;
+            return dtype == WKV_F32 ? dispatch_lane<float>(r != nullptr, a, dtype, nullptr, 0, stream)
+                                    : dispatch_lane<__nv_bfloat16>(r != nullptr, a, dtype, nullptr, 0, stream);
         }
         const bool part = part_ok && (force == 5 || (force == 0 && nLB < sm_count()));
         if (part) {
@@ -684,6 +736,65 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
         if (V == 2) dispatch_forward<__nv_bfloat16, 2>(r != nullptr, seq, a, grid, stream);
         else dispatch_forward<__nv_bfloat16, 1>(r != nullptr, seq, a, grid, stream);
     }
+    return check_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+int wkv_state(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const void* k, const void* v,
+              const float* state_in, float* state_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
+    if (B == 0 || C == 0) return WKV_OK;
+    if (state_out == nullptr) return WKV_ERR_NULLPTR;
+    if (T == 0)   // the state passes through (the same as wkv_forward with T = 0)
+        return wkv_forward(B, 0, C, dtype, nullptr, nullptr, nullptr, nullptr, nullptr, state_in, nullptr,
+                           state_out, nullptr, 0, stream);
+    if (!w || !k || !v) return WKV_ERR_NULLPTR;
+    const size_t eb = elem_bytes(dtype);
+    const size_t io_bytes = size_t(n) * eb, st_bytes = size_t(B) * size_t(C) * 3 * 4, p_bytes = size_t(C) * 4;
+    if (!aligned(w, 4) || !aligned(k, eb) || !aligned(v, eb) || (state_in && !aligned(state_in, 4)) ||
+        !aligned(state_out, 4))
+        return WKV_ERR_ALIGN;
+    if (overlaps(state_out, st_bytes, k, io_bytes) || overlaps(state_out, st_bytes, v, io_bytes) ||
+        overlaps(state_out, st_bytes, w, p_bytes) ||
+        (state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes)))
+        return WKV_ERR_ALIAS;
+    // the state does not depend on u or on the gate: w stands in for u (any
+    // finite row would do; it only steers the choice between two evaluations
+    // of the same summary), no gate, no output
+    return run_forward(B, T, C, dtype, w, w, k, v, nullptr, state_in, nullptr, state_out, workspace,
+                       workspace_bytes, stream);
+}
+
+int wkv_state_combine(int64_t B, int64_t C, int n, const float* w, const int64_t* lens, const float* states,
+                      const float* state_in, float* state_out, cudaStream_t stream) {
+    int64_t lanes = 0;
+    if (!mul_ok(B, C, 1, &lanes) || n < 0 || n > wkv::kCombineMax) return WKV_ERR_SHAPE;
+    if (lanes == 0) return WKV_OK;
+    if (state_out == nullptr || (n > 0 && (w == nullptr || lens == nullptr || states == nullptr)))
+        return WKV_ERR_NULLPTR;
+    wkv::CombineLens L{};
+    for (int j = 0; j < n; ++j) {
+        if (lens[j] < 0) return WKV_ERR_SHAPE;
+        L.len[j] = lens[j];
+    }
+    if (!aligned(state_out, 4) || (w && !aligned(w, 4)) || (states && !aligned(states, 4)) ||
+        (state_in && !aligned(state_in, 4)))
+        return WKV_ERR_ALIGN;
+    const size_t st_bytes = size_t(lanes) * 3 * 4;
+    if (overlaps(state_out, st_bytes, states, st_bytes * size_t(n)) || overlaps(state_out, st_bytes, w, size_t(C) * 4) ||
+        (state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes)))
+        return WKV_ERR_ALIAS;
+    if ((lanes + 255) / 256 > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    if (n == 0)
+        return wkv_forward(B, 0, C, WKV_F32, nullptr, nullptr, nullptr, nullptr, nullptr, state_in, nullptr,
+                           state_out, nullptr, 0, stream);
+    wkv::state_combine_kernel<<<static_cast<unsigned>((lanes + 255) / 256), 256, 0, stream>>>(
+        B, C, n, w, L, states, state_in, state_out);
     return check_launch();
 }
 
@@ -793,11 +904,10 @@ int noalloc_scratch(void** out) {
     return WKV_OK;
 }
 
-// Scratch of the register-load look-back kernel (chunks of kW * kLS tokens)
-// at the vector width the call will use; 0 when one chunk covers T.
-size_t noalloc_need(int64_t B, int64_t T, int64_t C, int V) {
-    if (T <= kSeqMaxT) return 0;
-    return chunk_geom(B, T, C, V, kW * kLS).bytes;
+// Scratch a call would use: the workspace wkv_forward takes for these sizes
+// (its look-back and hand-off words), or 0 when wkv_forward needs none.
+size_t noalloc_need(int64_t B, int64_t T, int64_t C, int dtype) {
+    return wkv_forward_workspace_bytes(B, T, C, dtype);
 }
 
 }  // namespace
@@ -807,8 +917,7 @@ extern "C" {
 size_t wkv_forward_noalloc_scratch_bytes(int64_t B, int64_t T, int64_t C, int dtype) {
     int64_t n = 0;
     if (!mul_ok(B, T, C, &n) || n == 0 || (dtype != WKV_F32 && dtype != WKV_BF16)) return 0;
-    const size_t a = noalloc_need(B, T, C, 1), b = noalloc_need(B, T, C, 2);
-    return a > b ? a : b;
+    return noalloc_need(B, T, C, dtype);
 }
 
 int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
@@ -817,77 +926,42 @@ int wkv_forward_noalloc(int64_t B, int64_t T, int64_t C, int dtype, const float*
     if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
     int64_t n = 0;
     if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
-    if (B == 0 || C == 0 || T <= kSeqMaxT) {
-        // nothing to do, or a sequence short enough for the kernel that needs
-        // no scratch: the regular entry point does exactly that
+    const size_t need = (B == 0 || C == 0 || T == 0) ? 0 : noalloc_need(B, T, C, dtype);
+    if (need > 0) {
+        // argument errors first: nothing, not even the array, is written then
+        const int vrc = forward_args(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out);
+        if (vrc != WKV_OK) return vrc;
+    }
+    if (need == 0 || (fits_cluster(dtype, B, T, C, k, v, r, w, u, state_in, y, state_out) && forced_kernel() == 0)) {
+        // nothing to do, or a call whose kernel needs no scratch (short
+        // sequences, or one cluster of parts per sequence): the regular entry
+        // point without a workspace does exactly that, and touches no array
         return wkv_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, nullptr, 0, stream);
     }
-    if (fits_cluster(dtype, B, T, C, k, v, r, w, u, state_in, y, state_out) && forced_kernel() == 0) {
-        // the cluster kernel needs no scratch: no shared array, no clearing
-        return wkv_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, nullptr, 0, stream);
-    }
-    if (!w || !u || !k || !v || !y) return WKV_ERR_NULLPTR;
-    const size_t eb = elem_bytes(dtype);
-    if (!aligned(w, 4) || !aligned(u, 4) || !aligned(k, eb) || !aligned(v, eb) || !aligned(y, eb) ||
-        (r && !aligned(r, eb)) || (state_in && !aligned(state_in, 4)) || (state_out && !aligned(state_out, 4)))
-        return WKV_ERR_ALIGN;
-    const size_t io_bytes = size_t(n) * eb, st_bytes = size_t(B * C) * 3 * 4, p_bytes = size_t(C) * 4;
-    const void* ins[] = {k, v, r};
-    for (const void* p : ins)
-        if (overlaps(y, io_bytes, p, io_bytes) || (state_out && overlaps(state_out, st_bytes, p, io_bytes)))
-            return WKV_ERR_ALIAS;
-    if (overlaps(y, io_bytes, w, p_bytes) || overlaps(y, io_bytes, u, p_bytes) ||
-        overlaps(y, io_bytes, state_in, st_bytes) || overlaps(y, io_bytes, state_out, st_bytes))
-        return WKV_ERR_ALIAS;
-    if (state_out && (overlaps(state_out, st_bytes, w, p_bytes) || overlaps(state_out, st_bytes, u, p_bytes) ||
-                      (state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes))))
-        return WKV_ERR_ALIAS;
+    if (need > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_SCRATCH;
+    void* ws = nullptr;
+    int rc = noalloc_scratch(&ws);
+    if (rc != WKV_OK) return rc;
+    // every call starts from a zeroed header and zeroed words: counters,
+    // error word and epoch at 0, and no word left over from an earlier call
+    rc = record_cuda(cudaMemsetAsync(ws, 0, need, stream));
+    if (rc != WKV_OK) return rc;
+    return wkv_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, ws, need, stream);
+}
 
-    const void* io[] = {k, v, r, y};
-    const float* f32[] = {w, u, state_in, state_out};
-    const int V = pick_vec(C, dtype, io, 4, f32, 4);
-    const ChunkGeom g = chunk_geom(B, T, C, V, kW * kLS);
-    if (g.units > 0x7fffffffLL) return WKV_ERR_SHAPE;
-    if (g.bytes > WKV_NOALLOC_SCRATCH_BYTES) return WKV_ERR_SCRATCH;
-
-    wkv::ChunkArgs a{};
-    a.w = w;
-    a.u = u;
-    a.k = k;
-    a.v = v;
-    a.r = r;
-    a.s_in = state_in;
-    a.y = y;
-    a.s_out = state_out;
-    a.B = B;
-    a.T = T;
-    a.C = C;
-    a.nCB = g.nCB;
-    a.nLB = g.nLB;
-    a.nchunks = g.nchunks;
-    a.units = g.units;
-    a.wait_limit_ns = wait_limit_ns();
-    if (g.bytes > 0) {
-        void* ws = nullptr;
-        int rc = noalloc_scratch(&ws);
-        if (rc != WKV_OK) return rc;
-        // every call starts from a zeroed header and zeroed words: counters,
-        // error word and epoch at 0, and no word left over from an earlier call
-        rc = record_cuda(cudaMemsetAsync(ws, 0, g.bytes, stream));
-        if (rc != WKV_OK) return rc;
-        char* base = static_cast<char*>(ws);
-        a.hdr = reinterpret_cast<wkv::WsHeader*>(base);
-        a.aggw = reinterpret_cast<wkv::Word*>(base + g.aggw_off);
-        a.incw = reinterpret_cast<wkv::Word*>(base + g.incw_off);
+int wkv_forward_noalloc_status(cudaStream_t stream) {
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    void* ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        ws = g_noalloc_ptr[dev];
     }
-    if (dtype == WKV_F32) {
-        if (V == 2) dispatch_forward<float, 2>(r != nullptr, false, a, g.units, stream);
-        else dispatch_forward<float, 1>(r != nullptr, false, a, g.units, stream);
-    } else {
-        if (V == 2) dispatch_forward<__nv_bfloat16, 2>(r != nullptr, false, a, g.units, stream);
-        else dispatch_forward<__nv_bfloat16, 1>(r != nullptr, false, a, g.units, stream);
-    }
-    return check_launch();
+    // no call on this device has used the array yet: nothing can have failed
+    if (ws == nullptr) return record_cuda(cudaStreamSynchronize(stream));
+    return wkv_workspace_status(ws, stream);
 }
 
 }  // extern "C"

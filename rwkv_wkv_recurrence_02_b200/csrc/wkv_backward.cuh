@@ -212,7 +212,7 @@ lane_backward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
     }
     pdl_begin();
     if (threadIdx.x == 0) {
-        s_range.init(A.nLB, A.nchunks, blockIdx.x, gridDim.x);
+        s_range.init(A.nLB, A.nchunks, blockIdx.x, gridDim.x, A.hdr == nullptr);
         s_epoch = A.hdr != nullptr ? ld_relaxed_u32(&A.hdr->epoch) : 0u;
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);

@@ -56,7 +56,7 @@ struct WsHeader {
     uint32_t done;      // CTAs finished in the current launch
     uint32_t error;     // kErrTimeout bits, sticky until the workspace is re-initialised
     uint32_t err_unit;  // a unit that hit the error
-    uint32_t ticket;    // next unit to claim (persistent kernel)
+    uint32_t ticket;    // next unit to claim (part and register-load look-back kernels)
 };
 
 // One published state of one channel, (p, a, b) as is, plus a tag = (launch
@@ -77,7 +77,7 @@ struct ChunkArgs {
     const void* v;
     const void* r;
     const float* s_in;
-    void* y;
+    void* y;            // null: only the state is wanted (no pass 2, no output)
     float* s_out;
     int64_t B, T, C;
     int64_t nCB;        // channel blocks per sequence
@@ -89,7 +89,6 @@ struct ChunkArgs {
     Word* incw;         // [units][CB] states after each chunk
     St* ckpt;           // lane-resident kernel only, or null: [nchunks + 1][nLB][CB] base-2 states
                         // entering each chunk, the last one the state after the sequence
-    int64_t unit_offset;
     uint64_t wait_limit_ns;
 };
 
@@ -465,9 +464,9 @@ __device__ __forceinline__ void unit_body(const ChunkArgs& A, int64_t unit, uint
         for (int j = 0; j < V; ++j) s_x[j][lane] = x[j];
     }
     __syncthreads();
-    if (nvalid == 0 || !cvalid) return;
+    if (nvalid == 0 || !cvalid || A.y == nullptr) return;
 
-    // ---- pass 2: outputs of this segment ----
+    // ---- pass 2: outputs of this segment (none when only the state is wanted) ----
     St st[V];
 #pragma unroll
     for (int j = 0; j < V; ++j)
@@ -558,20 +557,27 @@ __device__ __forceinline__ void finish_launch(const ChunkArgs& A, uint32_t ctas)
 }
 
 // One unit per CTA, rows loaded from global memory into registers.  Takes
-// any alignment that the vector width allows.
+// any alignment that the vector width allows.  With a workspace, a CTA
+// claims its unit from the workspace's ticket counter, so units are taken in
+// chunk-major order whatever order the hardware starts the CTAs in: a unit
+// only waits on units of earlier chunks, which CTAs already running hold.
 template <typename IO, int V, bool GATE, int W, int LS>
 __global__ void __launch_bounds__(W * 32)
 chunk_forward_kernel(const ChunkArgs A) {
     __shared__ St s_agg[W][V][32];
     __shared__ St s_x[V][32];
     __shared__ uint32_t s_epoch;
+    __shared__ int64_t s_unit;
     constexpr int TT = W * LS;
-    const int64_t unit = A.unit_offset + blockIdx.x;
-    const int64_t chunk = unit / A.nLB;
     const bool need_ws = A.nchunks > 1;
-    if (threadIdx.x == 0) s_epoch = need_ws ? ld_relaxed_u32(&A.hdr->epoch) : 0u;
+    if (threadIdx.x == 0) {
+        s_epoch = need_ws ? ld_relaxed_u32(&A.hdr->epoch) : 0u;
+        s_unit = need_ws ? static_cast<int64_t>(atomicAdd(&A.hdr->ticket, 1u)) : static_cast<int64_t>(blockIdx.x);
+    }
     __syncthreads();
     const uint32_t epoch = s_epoch;
+    const int64_t unit = s_unit;
+    const int64_t chunk = unit / A.nLB;
     if ((chunk + 1) * TT <= A.T)
         unit_body<IO, V, GATE, W, LS, true, false>(A, unit, epoch, nullptr, s_agg, s_x);
     else

@@ -195,7 +195,7 @@ cluster_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_cons
     // this CTA reads no other CTA's shared memory from here on
     cluster_arrive_relaxed();
     __syncthreads();
-    if (ok && cx.nvalid > 0 && cx.cvalid) {
+    if (ok && cx.nvalid > 0 && cx.cvalid && A.y != nullptr) {
         St st[V];
 #pragma unroll
         for (int j = 0; j < V; ++j) st[j] = st_combine(s_x[j][lane], pre[j], static_cast<float>(pre_len) * cx.w2[j]);

@@ -43,7 +43,9 @@ struct LaneGeometry {
 // block (starting inside the block from the state the previous CTA handed
 // over).  With at least as many lane blocks as CTAs every range spans a lane
 // block boundary, so a CTA has at most one head and one tail and no hand-off
-// depends on another.
+// depends on another.  `whole` (no workspace to hand states through) rounds
+// every range to whole lane blocks: CTA g takes lane blocks
+// [g*nLB/G, (g+1)*nLB/G), and no range has a head or a tail.
 struct LaneRange {
     int64_t nc;            // chunks per lane block
     int64_t f0, nfull;     // whole lane blocks [f0, f0 + nfull)
@@ -51,10 +53,11 @@ struct LaneRange {
     bool head, tail;
     int count;
 
-    __device__ __forceinline__ void init(int64_t nLB, int64_t nchunks, int64_t g, int64_t G) {
+    __device__ __forceinline__ void init(int64_t nLB, int64_t nchunks, int64_t g, int64_t G, bool whole) {
         nc = nchunks;
         const int64_t U = nLB * nchunks;
-        const int64_t s = g * U / G, e = (g + 1) * U / G;
+        const int64_t s = whole ? (g * nLB / G) * nchunks : g * U / G;
+        const int64_t e = whole ? ((g + 1) * nLB / G) * nchunks : (g + 1) * U / G;
         tail = s % nc != 0;
         lb_tail = s / nc;
         tail_begin = s % nc;
@@ -225,7 +228,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     }
     pdl_begin();
     if (threadIdx.x == 0) {
-        s_range.init(A.nLB, A.nchunks, blockIdx.x, gridDim.x);
+        s_range.init(A.nLB, A.nchunks, blockIdx.x, gridDim.x, A.hdr == nullptr);
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], W);
@@ -368,7 +371,7 @@ lane_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 #pragma unroll
                 for (int j = 0; j < V; ++j) s_carry[par ^ 1][j][lane] = nx[j];
             }
-            if (!CKPT && cx.nvalid > 0 && cx.cvalid) {
+            if (!CKPT && cx.nvalid > 0 && cx.cvalid && A.y != nullptr) {
                 if (full_chunk) seg_pass2<IO, V, GATE, W, LS, true>(A, stage, cx, st);
                 else seg_pass2<IO, V, GATE, W, LS, false>(A, stage, cx, st);
             }

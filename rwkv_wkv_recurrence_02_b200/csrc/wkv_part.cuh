@@ -295,7 +295,7 @@ part_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
                                   reinterpret_cast<const float*>(stage + G::NARR * G::TILE), &s_x[0][0]);
         }
         __syncthreads();
-        if (cx.nvalid > 0 && cx.cvalid) {
+        if (cx.nvalid > 0 && cx.cvalid && A.y != nullptr) {
             St st[V];
 #pragma unroll
             for (int j = 0; j < V; ++j) st[j] = st_combine(s_x[j][lane], pre[j], static_cast<float>(pre_len) * cx.w2[j]);

@@ -1,4 +1,5 @@
 // wkv_seq.cuh -- sequential-over-T forward kernel: one thread owns V lanes.
+// (y == NULL: only the state is wanted; no output is written.)
 //
 // The plain log-space recurrence (running max, one ex2 per max) walked token
 // by token, the parallel-mode loop of "並列学習の定式化" with the max
@@ -59,7 +60,7 @@ seq_forward_kernel(int64_t B, int64_t T, int64_t C, const float* __restrict__ w,
             out[j] = lane_token(sa[j], sb[j], sp[j], wj[j], uj[j], Ld::get(kr, j), Ld::get(vr, j), gd,
                                 kLog2e);
         }
-        Ld::store(yp, out);
+        if (y != nullptr) Ld::store(yp, out);
         kp += C;
         vp += C;
         if (GATE) rp += C;
@@ -73,6 +74,35 @@ seq_forward_kernel(int64_t B, int64_t T, int64_t C, const float* __restrict__ w,
             s_out[2 * lanes + lane0 + j] = sp[j];
         }
     }
+}
+
+// Fold of segment summaries: state_out = the state after n consecutive
+// segments of len[0..n-1] tokens entered from state_in (or the empty state),
+// where summary j is segment j's own state from the empty state.  Each fold
+// is the scan combine of the segment summaries (max form, one ex2).  One
+// thread per lane; states in natural-log units at the boundary.
+constexpr int kCombineMax = 64;
+struct CombineLens {
+    int64_t len[kCombineMax];
+};
+
+__global__ void __launch_bounds__(256)
+state_combine_kernel(int64_t B, int64_t C, int n, const float* __restrict__ w, CombineLens lens,
+                     const float* __restrict__ seg, const float* __restrict__ s_in, float* __restrict__ s_out) {
+    const int64_t lanes = B * C;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= lanes) return;
+    const float w2 = __ldg(w + i % C) * kLog2e;
+    St s = st_identity();
+    if (s_in != nullptr) s = St{s_in[2 * lanes + i] * kLog2e, s_in[i], s_in[lanes + i]};
+    for (int j = 0; j < n; ++j) {
+        const float* x = seg + static_cast<int64_t>(j) * 3 * lanes;
+        const St xs{x[2 * lanes + i] * kLog2e, x[i], x[lanes + i]};
+        s = st_combine(s, xs, static_cast<float>(lens.len[j]) * w2);
+    }
+    s_out[i] = s.a;
+    s_out[lanes + i] = s.b;
+    s_out[2 * lanes + i] = s.p * kLn2;
 }
 
 // T == 0: state_out = state_in (or the empty state).

@@ -19,6 +19,14 @@ F32, BF16 = 0, 1
 BASE = 1 << 40
 
 
+def _gpu_present():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return True
+
+
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
@@ -95,11 +103,19 @@ def test_forward_aliasing(L):
     assert fwd(L, s_out=BASE + (3 << 30)) == ALIAS      # state_out inside y
 
 
-def test_forward_workspace_checks(L):
-    n = L.wkv_forward_workspace_bytes(2, 100, 64, F32)
-    assert n > 0
-    assert fwd(L, ws=None, ws_bytes=0) == WORKSPACE
-    assert fwd(L, ws=BASE + (7 << 30), ws_bytes=n - 1) == WORKSPACE
+@pytest.mark.skipif(_gpu_present(), reason="launches on fake addresses; only where no GPU can run them")
+@pytest.mark.parametrize("B,T,C,dt", [(2, 100, 64, F32), (4, 8192, 5120, BF16), (1, 65536, 4096, BF16),
+                                      (1, 1 << 20, 4096, BF16), (3, 5000, 130, F32), (2, 2000, 7, BF16),
+                                      (64, 4096, 4096, F32)])
+def test_forward_runs_without_a_workspace(L, B, T, C, dt):
+    """No shape needs a caller workspace: with none (or too small a one) the
+    call passes every host check and goes on to a launch.  Without a GPU the
+    launch itself fails (WKV_ERR_CUDA); WKV_ERR_WORKSPACE never comes."""
+    assert L.wkv_forward_workspace_bytes(B, T, C, dt) > 0
+    ext = dict(k=BASE + (1 << 36), v=BASE + (2 << 36), y=BASE + (3 << 36))
+    assert fwd(L, B=B, T=T, C=C, dt=dt, ws=None, ws_bytes=0, **ext) not in (WORKSPACE, NULLPTR, ALIGN, ALIAS, SHAPE)
+    n = L.wkv_forward_workspace_bytes(B, T, C, dt)
+    assert fwd(L, B=B, T=T, C=C, dt=dt, ws=BASE + (7 << 36), ws_bytes=n - 1, **ext) not in (WORKSPACE, ALIGN)
 
 
 def test_workspace_size_rules(L):
@@ -217,3 +233,33 @@ def test_token_shift_front_end_refuses_bad_arguments():
         wkv.wkv_token_shift(torch.zeros(4, 8), torch.rand(3, 8))       # x not (B, T, C)
     with pytest.raises(ValueError):
         wkv.wkv_token_shift(x, torch.rand(8))                          # mu not (nmix, C)
+
+
+def test_state_validation(L):
+    st = BASE + (5 << 30)
+    call = lambda B=2, T=100, C=64, dt=F32, w=BASE, k=BASE + (1 << 30), v=BASE + (2 << 30), s_in=None, s_out=st: \
+        L.wkv_state(B, T, C, dt, w, k, v, s_in, s_out, None, 0, None)
+    assert call(dt=5) == DTYPE
+    assert call(B=-1) == SHAPE
+    assert call(B=0) == OK and call(C=0) == OK
+    assert call(s_out=None) == NULLPTR
+    assert call(k=None) == NULLPTR and call(w=None) == NULLPTR
+    assert call(k=BASE + (1 << 30) + 2) == ALIGN
+    assert call(s_out=BASE + (1 << 30)) == ALIAS                  # state_out inside k
+    assert call(s_in=st + 4, s_out=st) == ALIAS                   # partial state overlap
+
+
+def test_state_combine_validation(L):
+    import ctypes as ct
+    lens = (ct.c_int64 * 3)(5, 0, 7)
+    neg = (ct.c_int64 * 1)(-1)
+    st, seg = BASE + (5 << 30), BASE + (6 << 30)
+    call = lambda B=2, C=64, n=3, w=BASE, ln=lens, sg=seg, s_in=None, s_out=st: \
+        L.wkv_state_combine(B, C, n, w, ln, sg, s_in, s_out, None)
+    assert call(n=-1) == SHAPE and call(n=65) == SHAPE
+    assert call(n=1, ln=neg) == SHAPE
+    assert call(B=0) == OK
+    assert call(s_out=None) == NULLPTR
+    assert call(ln=None) == NULLPTR and call(sg=None) == NULLPTR and call(w=None) == NULLPTR
+    assert call(s_out=st + 2) == ALIGN
+    assert call(s_out=seg + 64) == ALIAS                          # state_out inside the summaries

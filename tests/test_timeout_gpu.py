@@ -56,3 +56,35 @@ def test_expired_wait_is_reported(name, script, kernel, shape):
     assert out["STATUS"] == "-7"           # WKV_ERR_TIMEOUT
     assert out["NAN"] == "True"            # affected outputs are NaN, not stale values
     assert out["AFTER_RESET"] == "0"
+
+
+NOALLOC = r"""
+import sys, torch
+sys.path.insert(0, %r)
+import rwkv_wkv_recurrence_02_b200 as wkv
+from rwkv_wkv_recurrence_02_b200 import inputs as I
+B, T, C = %d, %d, %d
+wl = I.Workload("t", B, T, C, "f32", False, -3.0, 1.0, 1.0, 1.0, False, seed=5)
+d = I.make_forward_inputs(wl, device="cuda")
+print("BEFORE", wkv.wkv_forward_noalloc_status())
+y = torch.empty_like(d["k"])
+wkv.wkv_forward_noalloc(d["w"], d["u"], d["k"], d["v"], y=y)
+print("STATUS", wkv.wkv_forward_noalloc_status(), "NAN", bool(torch.isnan(y).any().item()))
+"""
+
+
+@pytest.mark.gpu
+def test_noalloc_expired_wait_is_reported():
+    """The allocation-free entry point keeps its error word in the built-in
+    array; wkv_forward_noalloc_status reads it.  C = 130 (not a multiple of
+    4) takes the register-load look-back kernel, whose chunks wait on one
+    another."""
+    env = dict(os.environ, WKV_WAIT_LIMIT_NS="1")
+    env.pop("WKV_FORWARD_KERNEL", None)
+    r = subprocess.run([sys.executable, "-c", NOALLOC % (ROOT, 1, 64 * 300, 130)], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    out = dict(zip(r.stdout.split()[::2], r.stdout.split()[1::2]))
+    assert out["BEFORE"] == "0"            # nothing has used the array yet
+    assert out["STATUS"] == "-7"           # WKV_ERR_TIMEOUT
+    assert out["NAN"] == "True"
