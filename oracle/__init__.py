@@ -34,6 +34,7 @@ def lib():
         L.oracle_wkv_combine.argtypes = [d, d, d, d, d, d, d, i64, p]
         L.oracle_wkv_backward.argtypes = [i64, i64, i64, p, p, p, p, p, p, p, p, p, p, p, p, p, p, i32]
         L.oracle_token_shift.argtypes = [i64, i64, i64, i64, p, p, p, p, p]
+        L.oracle_wkv5_forward.argtypes = [i64, i64, i64, i64, i32, p, p, p, p, p, p, p, p, p]
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -147,6 +148,33 @@ def token_shift(x, mu, x_prev=None):
     last = np.empty((B, C), np.float64)
     lib().oracle_token_shift(B, T, C, nmix, _ptr(x), _ptr(mu), _ptr(x_prev), _ptr(out), _ptr(last))
     return out, last
+
+
+def wkv5_forward(w, u, k, v, r, H, state_in=None, want_scale=False):
+    """Multi-head matrix-state WKV (v5: w of shape (C,); v6: w of shape
+    (B, T, C), a decay rate per token).  k, v, r: (B, T, C) with C = H * N;
+    u: (C,); state_in: (B, H, N, N) float64 or None (zeros).  Returns
+    (y, state_out[, yscale]) in float64; see wkv5_oracle.c."""
+    w, u, k, v, r, state_in = _f32(w), _f32(u), _f32(k), _f32(v), _f32(r), _f64(state_in)
+    if k.ndim != 3 or v.shape != k.shape or r.shape != k.shape:
+        raise ValueError("k, v, r must share one (B, T, C) shape")
+    B, T, C = k.shape
+    if C % H != 0:
+        raise ValueError("C must be a multiple of H")
+    N = C // H
+    wmode = 0 if w.shape == (C,) else 1
+    if wmode == 1 and w.shape != (B, T, C):
+        raise ValueError("w must be (C,) or (B, T, C)")
+    if u.shape != (C,):
+        raise ValueError("u must be (C,)")
+    if state_in is not None and state_in.shape != (B, H, N, N):
+        raise ValueError("state must be (B, H, N, N)")
+    y = np.empty((B, T, C), np.float64)
+    ys = np.empty((B, T, C), np.float64) if want_scale else None
+    st = np.empty((B, H, N, N), np.float64)
+    lib().oracle_wkv5_forward(B, T, H, N, wmode, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
+                              _ptr(y), _ptr(ys), _ptr(st))
+    return (y, st, ys) if want_scale else (y, st)
 
 
 def fresh_state(B, C):
