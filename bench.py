@@ -4,18 +4,21 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one pass of the whole operator over one batch of synthetic inputs
-already resident in HBM.  The default workload is the RWKV-4 1.5B-shaped layer
-(B=8, T=1024, C=2048, float32 k/v/r/y, sigmoid gate, random initial state):
-one wkv_forward call per step.  Other workloads (layer_14b, stream_1m: one
-1024-token chunk with the state carried, decode: one wkv_step over 24 layers)
-are available with --workload.
+already resident in HBM.  The default workload is the long-context stream:
+B=1, C=4096, T=1,048,576 bfloat16 tokens fed as 1024 chunks of 1024 tokens,
+the state (num, den, max) carried in place from the empty state; one step is
+the whole stream, 1024 wkv_forward calls replayed from one CUDA graph.  Other
+workloads (layer_1b5, layer_14b, stream_1m_chunk: one chunk per step,
+stream_1m_single: the whole stream in one call, decode: one wkv_step over 24
+layers) are available with --workload.
 
 Timing: W warm-up steps, then exactly K steps between a barrier +
 synchronize on both sides, timed with CUDA events on the launching stream;
-the inputs rotate over two sets whose size exceeds the 126 MB L2, so no step
-finds its inputs in L2.  With N GPUs (torchrun) every rank runs the same
-per-GPU workload on its own seeds (independent sequences: no collective on the
-data path), the time is the max over ranks and the value is the total.
+the inputs exceed the 126 MB L2 (the stream: 25.8 GB; the others rotate over
+sets larger than twice L2), so no step finds its inputs in L2.  With N GPUs
+(torchrun) every rank runs the same per-GPU workload on its own seeds
+(independent sequences: no collective on the data path), the time is the max
+over ranks and the value is the total.
 
 `--impl reference` times the fp64 CPU oracle on the host cores on a bounded
 lane sample per step (rank 0 only).
@@ -37,6 +40,10 @@ if ROOT not in sys.path:
 METRIC = "WKV elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
 METRIC_BWD = "WKV backward elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
 METRIC_SHIFT = "token shift elements/s (B·T·C) and achieved HBM GB/s as % of B200 peak, 1 GPU"
+METRIC_WKV5 = "matrix-state WKV elements/s (B·T·C) and achieved FP32 rate as % of B200 peak, 1 GPU"
+# FP32 pipe of one B200: 148 SMs x 128 fused multiply-adds per clock at the
+# 1965 MHz clocks.max.sm (the recipe's unit counts and clock)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 SHIFT_MIXES = 3   # RWKV-4 time mixing: one mix each for K, V and R
 UNIT = "elements/s"
 SPEC_HBM_GBS = 8000.0
@@ -102,6 +109,24 @@ def algorithmic_bytes_shift(wl, B, T, C, nmix=SHIFT_MIXES) -> int:
     the next one written, mu read."""
     eb = wl.elem_bytes
     return B * T * C * eb * (1 + nmix) + 2 * B * C * eb + nmix * C * 4
+
+
+def algorithmic_bytes_wkv5(wl, B, T, C, H, state=False) -> int:
+    """Bytes one wkv5_forward call must move at minimum: r, k, v read and y
+    written once, the decay rates (per channel, or per token and channel),
+    u, and the (B, H, N, N) state written (and read when given)."""
+    eb = wl.elem_bytes
+    n = B * T * C
+    N = C // H
+    w = n * 4 if wl.per_token_decay else C * 4
+    return n * eb * 4 + w + C * 4 + B * H * N * N * 4 * (2 if state else 1)
+
+
+def flops_wkv5(B, T, C, H) -> int:
+    """FP32 operations of the recurrence: per token, head and state entry a
+    multiply-add for the output, a multiply-add and a multiply for the update
+    (5 flops), N^2 entries per head: 5 N per element."""
+    return B * T * C * 5 * (C // H)
 
 
 def max_over_ranks(value: float, dist=None) -> float:
@@ -174,16 +199,25 @@ class ClockSampler:
             self.ok = False
         self.thread = threading.Thread(target=self._run, daemon=True)
 
+    def _one(self):
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            util = self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+            self.samples.append((time.time(), mhz, reasons, util))
+        except Exception:
+            pass
+
     def _run(self):
         while not self.stop_evt.is_set():
-            try:
-                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-                reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                util = self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu
-                self.samples.append((time.time(), mhz, reasons, util))
-            except Exception:
-                pass
+            self._one()
             time.sleep(self.period)
+
+    def sample_now(self):
+        """One extra sample now (the timed region's edges, so that a short
+        region still has samples inside it)."""
+        if self.ok:
+            self._one()
 
     def start(self):
         if self.ok:
@@ -198,7 +232,7 @@ class ClockSampler:
     def summary(self, t0: float, t1: float):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
-        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        inside = [s for s in sorted(self.samples) if t0 - 1e-3 <= s[0] <= t1 + 1e-3]
         src = inside if inside else [s for s in self.samples if s[0] >= t0 - 1.0]
         if not src:
             src = self.samples[-3:]
@@ -246,6 +280,52 @@ class ForwardCase:
         else:
             wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"], y=self.y[i % len(self.y)],
                             state_out=self.s_out[i % len(self.s_out)], workspace=ws)
+
+
+class StreamCase:
+    """The streaming workload as its definition reads: one step feeds the whole
+    stream (T = 1,048,576 tokens) through wkv_forward as T / chunk carried
+    chunks, the state in place and reset to the empty state at the start of
+    the step.  k, v and y of the whole stream are resident (25.8 GB for the
+    1M-token stream), so every chunk reads fresh inputs from HBM.
+    inputs_ready passes WKV_FLAG_INPUTS_READY: the chunks' inputs are written
+    before the step and never by the chain itself."""
+
+    def __init__(self, wl, device, seed_base, inputs_ready=True):
+        import dataclasses
+        import torch
+        from rwkv_wkv_recurrence_02_b200 import inputs as I
+        self.wl = wl
+        self.B, self.T, self.C, self.chunk = wl.B, wl.T, wl.C, wl.chunk
+        self.n = wl.T // wl.chunk
+        wr = dataclasses.replace(wl, seed=wl.seed + seed_base)
+        self.w, self.u = I.make_params(wr, device=device)
+        dt = wl.torch_dtype
+        self.k = torch.empty((self.B, self.T, self.C), dtype=dt, device=device)
+        self.v = torch.empty_like(self.k)
+        for i in range(self.n):
+            kc, vc, _ = I.make_chunk(wr, i, device=device)
+            self.k[:, i * self.chunk:(i + 1) * self.chunk] = kc
+            self.v[:, i * self.chunk:(i + 1) * self.chunk] = vc
+        self.y = torch.empty_like(self.k)
+        self.fresh = I.fresh_state(self.B, self.C, device=device)
+        self.state = self.fresh.clone()
+        self.ready = inputs_ready
+        self.elements = self.B * self.T * self.C
+        self.bytes = algorithmic_bytes(wl, self.B, self.chunk, self.C)      # per launch (one chunk)
+        self.launches_per_step = self.n
+        self.roofline_per_step = False
+        self.period = 1
+
+    def chunk_slice(self, i):
+        return slice(i * self.chunk, (i + 1) * self.chunk)
+
+    def step(self, i, wkv, ws):
+        self.state.copy_(self.fresh)
+        for j in range(self.n):
+            sl = self.chunk_slice(j)
+            wkv.wkv_forward(self.w, self.u, self.k[:, sl], self.v[:, sl], None, self.state, y=self.y[:, sl],
+                            state_out=self.state, workspace=ws, inputs_ready=self.ready)
 
 
 class DecodeCase:
@@ -319,6 +399,36 @@ class BackwardCase:
                          workspace=ws, **self.out[i % 2])
 
 
+class Wkv5Case:
+    """wkv5_forward on a matrix-state workload: inputs rotating over sets
+    larger than twice L2, outputs preallocated, a fresh state per call."""
+
+    def __init__(self, wl, device, seed_base):
+        import torch
+        from rwkv_wkv_recurrence_02_b200 import inputs as I
+        self.wl = wl
+        self.B, self.T, self.C, self.H = wl.B, wl.T, wl.C, wl.H
+        one = algorithmic_bytes_wkv5(wl, self.B, self.T, self.C, self.H)
+        nsets = 2
+        while nsets * one < 2 * L2_BYTES:
+            nsets += 1
+        self.sets = [I.make_matrix_inputs(wl, device=device, seed_offset=seed_base + i) for i in range(nsets)]
+        N = self.C // self.H
+        self.y = [torch.empty((self.B, self.T, self.C), dtype=wl.torch_dtype, device=device) for _ in range(2)]
+        self.s_out = [torch.empty((self.B, self.H, N, N), device=device) for _ in range(2)]
+        self.elements = self.B * self.T * self.C
+        self.bytes = one
+        self.flops = flops_wkv5(self.B, self.T, self.C, self.H)
+        self.launches_per_step = 1
+        self.roofline_per_step = False
+        self.period = nsets * 2 // math.gcd(nsets, 2)
+
+    def step(self, i, wkv, ws):
+        d = self.sets[i % len(self.sets)]
+        wkv.wkv5_forward(d["w"], d["u"], d["r"], d["k"], d["v"], self.H, None, y=self.y[i % 2],
+                         state_out=self.s_out[i % 2])
+
+
 class TokenShiftCase:
     """Token shift on a workload's shape (decode: one token of one layer):
     x of the workload's dtype, SHIFT_MIXES mixes, the previous token carried;
@@ -353,19 +463,35 @@ class TokenShiftCase:
         wkv.wkv_token_shift(d["x"], d["mu"], d["xp"], out=self.out[i % 2], x_last=self.last[i % 2])
 
 
+WORKLOAD_NAMES = ["stream_1m", "stream_1m_chunk", "stream_1m_single", "layer_1b5", "layer_14b", "decode", "tiny",
+                  "v5_layer", "v6_layer"]
+
+
 def workload(name):
-    """A workload by name.  `stream_1m_single` is the streaming workload's
-    whole 1M-token sequence in one call instead of 1024-token chunks."""
+    """A workload by name.  `stream_1m` is the whole stream as 1024 carried
+    chunks per step; `stream_1m_chunk` one of those chunks per step;
+    `stream_1m_single` the whole 1M-token sequence in one call."""
     import dataclasses
     from rwkv_wkv_recurrence_02_b200 import inputs as I
     if name == "stream_1m_single":
         return dataclasses.replace(I.WORKLOADS["stream_1m"], name=name, chunk=0)
+    if name == "stream_1m_chunk":
+        return dataclasses.replace(I.WORKLOADS["stream_1m"], name=name)
+    if name in I.MATRIX_WORKLOADS:
+        return I.MATRIX_WORKLOADS[name]
     return I.WORKLOADS[name]
 
 
-def make_case(name, device, seed_base, op="forward", per_layer=False):
-    from rwkv_wkv_recurrence_02_b200 import inputs as I
+def whole_stream(name) -> bool:
+    return name == "stream_1m"
+
+
+def make_case(name, device, seed_base, op="forward", per_layer=False, inputs_ready=True):
     wl = workload(name)
+    if op == "wkv5" or hasattr(wl, "H"):
+        if not hasattr(wl, "H"):
+            raise SystemExit("--op wkv5 takes the matrix-state workloads (v5_layer, v6_layer)")
+        return Wkv5Case(wl, device, seed_base)
     if op == "token_shift":
         return TokenShiftCase(wl, device, seed_base)
     if op == "backward":
@@ -374,19 +500,82 @@ def make_case(name, device, seed_base, op="forward", per_layer=False):
         return BackwardCase(wl, device, seed_base)
     if wl.layers:
         return DecodeCase(wl, device, seed_base, per_layer)
+    if whole_stream(name):
+        return StreamCase(wl, device, seed_base, inputs_ready)
     return ForwardCase(wl, device, seed_base)
+
+
+def e2e_measure_wkv5(case, wkv, steps, warmup, stream):
+    """wkv5_forward through the public API with host buffers: r, k, v, w, u
+    in from pinned host memory, y and the state out."""
+    import torch
+    d = case.sets[0]
+    names = ("w", "u", "r", "k", "v")
+    host = {n: d[n].to("cpu").pin_memory() for n in names}
+    dev = {n: torch.empty_like(x, device=d["k"].device) for n, x in host.items()}
+    y_h = torch.empty(case.y[0].shape, dtype=case.y[0].dtype).pin_memory()
+    s_h = torch.empty(case.s_out[0].shape).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = y_h.numel() * y_h.element_size() + s_h.numel() * 4
+
+    def one():
+        for n, x in host.items():
+            dev[n].copy_(x, non_blocking=True)
+        wkv.wkv5_forward(dev["w"], dev["u"], dev["r"], dev["k"], dev["v"], case.H, None, y=case.y[0],
+                         state_out=case.s_out[0])
+        y_h.copy_(case.y[0], non_blocking=True)
+        s_h.copy_(case.s_out[0], non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h,
+            "path": "pinned host -> wkv5_forward (C ABI) -> pinned host"}
+
+
+def cpu_baseline_wkv5(name: str, budget_s: float, max_reps: int = 1000):
+    """The oracle's matrix-state WKV on this host's cores over a sample of
+    (sequence, head) pairs of the workload, repeated for about `budget_s`."""
+    import oracle
+    from rwkv_wkv_recurrence_02_b200 import inputs as I
+    wl = workload(name)
+    heads = max(1, oracle.max_threads())
+    N = wl.C // wl.H
+    d = I.make_matrix_inputs(wl, B=1, C=heads * N, H=heads)
+    f = lambda x: x.float().numpy()
+    run = lambda: oracle.wkv5_forward(f(d["w"]), f(d["u"]), f(d["k"]), f(d["v"]), f(d["r"]), heads)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        run()
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= max_reps:
+            break
+    sec = time.perf_counter() - t0
+    return {"value": wl.T * heads * N * reps / sec, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{heads} heads of one sequence (T={wl.T}, N={N}), repeated {reps}x over {sec:.1f} s"}
 
 
 def e2e_measure(case, wkv, ws, steps, warmup, stream):
     """Same metric through the public API with host buffers: each step copies
     its inputs from pinned host memory and reads the result back."""
     import torch
+    if isinstance(case, Wkv5Case):
+        return e2e_measure_wkv5(case, wkv, steps, warmup, stream)
     if isinstance(case, BackwardCase):
         return e2e_measure_backward(case, wkv, ws, steps, warmup, stream)
     if isinstance(case, DecodeCase):
         return e2e_measure_decode(case, wkv, steps, warmup, stream)
     if isinstance(case, TokenShiftCase):
         return e2e_measure_shift(case, wkv, steps, warmup, stream)
+    if isinstance(case, StreamCase):
+        return e2e_measure_stream(case, wkv, ws, steps, warmup, stream)
     d = case.sets[0]
     host = {k: (None if v is None else v.to("cpu").pin_memory()) for k, v in d.items()}
     y_host = torch.empty(case.y[0].shape, dtype=case.y[0].dtype).pin_memory()
@@ -415,6 +604,67 @@ def e2e_measure(case, wkv, ws, steps, warmup, stream):
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) / 1e3
     return {"seconds": sec, "steps": steps, "h2d": h2d, "d2h": d2h}
+
+
+def e2e_measure_stream(case, wkv, ws, steps, warmup, stream, ring=8):
+    """The whole stream through the public API from pinned host memory: every
+    chunk's k, v are copied in on one stream, the chunk's wkv_forward runs on
+    the compute stream, and its y is copied back on a third, with two device
+    buffers per array so that chunk i+1's upload and chunk i-1's download
+    overlap chunk i's kernel.  The host side cycles over `ring` pinned chunks
+    (the bytes per step are those of the whole stream)."""
+    import torch
+    ch, n = case.chunk, case.n
+    host_k = [case.k[:, case.chunk_slice(j)].to("cpu").pin_memory() for j in range(ring)]
+    host_v = [case.v[:, case.chunk_slice(j)].to("cpu").pin_memory() for j in range(ring)]
+    host_y = [torch.empty_like(host_k[0]).pin_memory() for _ in range(ring)]
+    s_host = torch.empty((3, case.B, case.C), dtype=torch.float32).pin_memory()
+    dk = [torch.empty_like(host_k[0], device=case.k.device) for _ in range(2)]
+    dv = [torch.empty_like(dk[0]) for _ in range(2)]
+    dy = [torch.empty_like(dk[0]) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    h2d = n * 2 * host_k[0].numel() * host_k[0].element_size()
+    d2h = n * host_y[0].numel() * host_y[0].element_size() + s_host.numel() * 4
+
+    def one():
+        case.state.copy_(case.fresh)
+        s_in.wait_stream(stream)
+        for j in range(n):
+            b = j & 1
+            with torch.cuda.stream(s_in):
+                if j >= 2:
+                    s_in.wait_event(ev_comp[b])          # the kernel that read buffer b is done
+                dk[b].copy_(host_k[j % ring], non_blocking=True)
+                dv[b].copy_(host_v[j % ring], non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if j >= 2:
+                stream.wait_event(ev_out[b])             # y buffer b has been read back
+            wkv.wkv_forward(case.w, case.u, dk[b], dv[b], None, case.state, y=dy[b], state_out=case.state,
+                            workspace=ws, stream=stream)
+            ev_comp[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b])
+                host_y[j % ring].copy_(dy[b], non_blocking=True)
+                ev_out[b].record(s_out)
+        s_host.copy_(case.state, non_blocking=True)
+        stream.wait_stream(s_out)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"seconds": e0.elapsed_time(e1) / 1e3, "steps": steps, "h2d": h2d, "d2h": d2h,
+            "path": (f"pinned host (ring of {ring} chunks) -> {n} x wkv_forward (C ABI), uploads, kernels and "
+                     "downloads on three streams with double-buffered chunks -> pinned host")}
 
 
 def e2e_measure_decode(case, wkv, steps, warmup, stream):
@@ -601,7 +851,7 @@ def cpu_baseline_sample(name: str, budget_s: float, max_reps: int = 1000):
         run = lambda: oracle.wkv_step(args[0], args[1], args[2], args[3], args[4], args[5])
         elems, sample = L * B * C, f"one decode step of all {L} layers (B={B}, C={C})"
     else:
-        T = wl.chunk or wl.T
+        T = wl.T if whole_stream(name) else (wl.chunk or wl.T)
         B, C = wl.B, wl.C
         # lanes so that one repetition takes a bounded time
         lanes_total = B * C
@@ -614,6 +864,8 @@ def cpu_baseline_sample(name: str, budget_s: float, max_reps: int = 1000):
         elems = B * T * csub
         sample = (f"full step B={B}, T={T}, C={C}" if csub == C else
                   f"lane sample B={B}, T={T}, C={csub} of {C}")
+        if whole_stream(name):
+            sample += " (the whole stream in one oracle call, which equals the carried chunks exactly)"
     t0 = time.perf_counter()
     reps = 0
     while True:
@@ -631,12 +883,19 @@ def cpu_baseline_sample(name: str, budget_s: float, max_reps: int = 1000):
 # ---------------------------------------------------------------------------
 def config_of(case, workload, world):
     wl = case.wl
-    cfg = {"workload": workload, "B": wl.B, "T": (wl.chunk or wl.T), "C": wl.C, "io_dtype": wl.dtype,
-           "gate": wl.gate, "parallelism": f"dp{world}" if world > 1 else "single",
+    cfg = {"workload": workload, "B": wl.B, "T": (getattr(wl, "chunk", 0) or wl.T), "C": wl.C,
+           "io_dtype": wl.dtype, "gate": getattr(wl, "gate", False),
+           "parallelism": f"dp{world}" if world > 1 else "single",
            "l2": "inputs rotate over sets totalling >2x the 126 MB L2"}
-    if wl.layers:
+    if getattr(wl, "layers", 0):
         cfg.update({"layers": wl.layers, "T": 1, "steps_per_sequence": wl.steps})
-    if wl.chunk:
+    if whole_stream(workload):
+        cfg.update({"T": wl.T, "chunk": wl.chunk,
+                    "stream": (f"the whole stream per step: {wl.T // wl.chunk} wkv_forward calls of {wl.chunk} "
+                               "tokens, state carried in place from the empty state"),
+                    "inputs_ready": bool(getattr(case, "ready", False)),
+                    "l2": "inputs of the whole stream resident (25.8 GB), far above the 126 MB L2"})
+    elif getattr(wl, "chunk", 0):
         cfg["stream"] = f"one chunk of {wl.chunk} tokens per step, state carried in place"
     return cfg
 
@@ -666,14 +925,15 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     wkv.lib()
-    case = make_case(args.workload, device, rank_seed(0, rank), args.op, args.decode_per_layer)
+    case = make_case(args.workload, device, rank_seed(0, rank), args.op, args.decode_per_layer,
+                     not args.no_inputs_ready)
     ws = wkv.Workspace(device)
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
         case.step(i, wkv, ws)
     torch.cuda.synchronize()
     graphs = None
-    if args.graph:
+    if args.graph or (isinstance(case, StreamCase) and not args.no_graph):
         # one CUDA graph per distinct step (inputs rotate with period case.period)
         graphs = []
         for p in range(case.period):
@@ -692,6 +952,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    clocks.sample_now()
     t0 = time.time()
     e0.record(stream)
     for i in range(args.steps):
@@ -700,6 +961,7 @@ def run_ours(args):
         else:
             case.step(args.warmup + i, wkv, ws)
     e1.record(stream)
+    clocks.sample_now()
     torch.cuda.synchronize()
     t1 = time.time()
     if world > 1:
@@ -723,7 +985,8 @@ def run_ours(args):
         "data": "synthetic (seeded; distributions of the workload definition)",
         "config": dict(config_of(case, args.workload, world), **({"op": args.op} if args.op != "forward" else {}),
                        **(shift_config(case) if args.op == "token_shift" else {}),
-                       **({"graph": f"{len(graphs)} captured steps replayed"} if graphs is not None else {}),
+                       **({"graph": (f"{len(graphs)} captured step(s) of {case.launches_per_step} launches "
+                                     "replayed")} if graphs is not None else {}),
                        **({"decode_form": "one wkv_step per layer (L = 1)"} if args.decode_per_layer else {})),
         "hbm_gbs": achieved, "hbm_pct_of_spec_8tbs": 100.0 * achieved / SPEC_HBM_GBS,
         "hbm_pct_of_measured": 100.0 * achieved / peak,
@@ -737,16 +1000,31 @@ def run_ours(args):
         "gpu_launches": args.steps * case.launches_per_step,
         "clocks": clocks.summary(t0, t1),
     }
+    if isinstance(case, Wkv5Case):
+        # the recurrence is bound by FP32 arithmetic: the roofline is the FP32
+        # pipe; the memory fraction stays beside it
+        tflops = case.flops / per_launch / 1e12
+        out["metric"] = METRIC_WKV5
+        out["config"].update({"H": case.H, "head_size": case.C // case.H, "decay": (
+            "per token and channel (v6)" if case.wl.per_token_decay else "per channel (v5)"), "gate": False})
+        out["roofline"] = {"bound": "alu", "achieved": tflops, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                           "frac": tflops / FP32_PEAK_TFLOPS,
+                           "peak_kind": "derived: 148 SMs x 128 FP32 FMA/clock x 2 x 1965 MHz",
+                           "flops_per_launch": case.flops, "algorithmic_bytes_per_launch": case.bytes,
+                           "hbm_frac_of_measured": achieved / peak, "scope": "the step's one kernel",
+                           "traffic": load_traffic(args.workload + "_wkv5")}
     if not args.no_e2e:
-        e = e2e_measure(case, wkv, ws, min(args.steps, args.e2e_steps), 2, stream)
+        e2e_steps = min(args.steps, 2 if isinstance(case, StreamCase) else args.e2e_steps)
+        e = e2e_measure(case, wkv, ws, e2e_steps, 1 if isinstance(case, StreamCase) else 2, stream)
         if e is not None:
             out["e2e"] = {"value": whole_job_rate(case.elements, world, e["steps"],
                                                   max_over_ranks(e["seconds"], dist if world > 1 else None)),
                           "unit": UNIT, "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                           "steps": e["steps"], "path": e.get("path", "pinned host -> wkv_forward (C ABI) -> pinned host")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = {"backward": cpu_baseline_backward, "token_shift": cpu_baseline_shift}.get(
-            args.op, cpu_baseline_sample)(args.workload, args.cpu_seconds)
+        out["cpu_baseline"] = {"backward": cpu_baseline_backward, "token_shift": cpu_baseline_shift,
+                               "wkv5": cpu_baseline_wkv5}.get(
+            "wkv5" if isinstance(case, Wkv5Case) else args.op, cpu_baseline_sample)(args.workload, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -770,7 +1048,7 @@ def run_reference(args):
         return run_reference_shift(args, wl)
     if wl.layers:
         raise SystemExit("--impl reference times the forward workloads")
-    T, B, C = (wl.chunk or wl.T), wl.B, wl.C
+    T, B, C = (wl.T if whole_stream(args.workload) else (wl.chunk or wl.T)), wl.B, wl.C
     backward = args.op == "backward"
 
     def call(d, n):
@@ -783,11 +1061,12 @@ def run_reference(args):
         return lambda: oracle.wkv_backward(*a, dy, ds)
 
     # calibrate: seconds per lane (all T tokens) with all cores busy
-    cal = I.make_forward_inputs(wl, B=1, T=T, C=min(C, 256))
-    run = call(cal, min(C, 256))
+    ncal = min(C, 256 if T <= 65536 else 16)
+    cal = I.make_forward_inputs(wl, B=1, T=T, C=ncal)
+    run = call(cal, ncal)
     t0 = time.perf_counter()
     run()
-    per_lane = (time.perf_counter() - t0) / min(C, 256)
+    per_lane = (time.perf_counter() - t0) / ncal
     lanes = int(max(1, min(B * C, budget / max(1, args.steps + args.warmup) / per_lane)))
     csub = max(1, min(C, lanes))
     d = I.make_forward_inputs(wl, B=1, T=T, C=csub)
@@ -801,6 +1080,8 @@ def run_reference(args):
     elems = T * csub
     value = elems * args.steps / sec
     sample = f"lane sample B=1, T={T}, C={csub} of the workload's B={B}, C={C} per step"
+    if whole_stream(args.workload):
+        sample += " (the whole stream in one oracle call, which equals the carried chunks exactly)"
     out = {
         "metric": METRIC_BWD if backward else METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True,
@@ -855,16 +1136,20 @@ def run_reference_shift(args, wl):
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=3000)
-    p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--workload", default="layer_1b5",
-                   choices=["tiny", "layer_1b5", "layer_14b", "stream_1m", "stream_1m_single", "decode"])
+    p.add_argument("--steps", type=int, default=None,
+                   help="timed steps (default: 20 for the whole stream, 3000 for the other workloads)")
+    p.add_argument("--warmup", type=int, default=None, help="warm-up steps (default: 5 / 20)")
+    p.add_argument("--workload", default="stream_1m", choices=WORKLOAD_NAMES)
+    p.add_argument("--no-graph", action="store_true",
+                   help="the whole stream: launch the chunk calls instead of replaying a CUDA graph")
+    p.add_argument("--no-inputs-ready", action="store_true",
+                   help="the whole stream: do not pass WKV_FLAG_INPUTS_READY")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--graph", action="store_true",
                    help="replay each step from a captured CUDA graph instead of launching it")
     p.add_argument("--decode-per-layer", action="store_true",
                    help="decode: one wkv_step per layer (L = 1) instead of one call over all layers")
-    p.add_argument("--op", default="forward", choices=["forward", "backward", "token_shift"],
+    p.add_argument("--op", default="forward", choices=["forward", "backward", "token_shift", "wkv5"],
                    help="forward (the headline), the reverse mode, or the token shift on the workload's shape")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -872,6 +1157,10 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     a = p.parse_args(argv)
+    if a.steps is None:
+        a.steps = 20 if whole_stream(a.workload) and a.op == "forward" else 3000
+    if a.warmup is None:
+        a.warmup = 5 if whole_stream(a.workload) and a.op == "forward" else 20
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
     return a

@@ -124,6 +124,34 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype,
                 const float* state_in, void* y, float* state_out,
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * wkv_forward_ex -- wkv_forward with launch flags.  flags == 0 is exactly
+ * wkv_forward.  Any bit other than those below is WKV_ERR_SHAPE.
+ *
+ *   WKV_FLAG_INPUTS_READY  the caller declares that k, v, r, w and u are not
+ *       written by any work still running on `stream` when this call is
+ *       enqueued (they were produced earlier and are left alone).  Every
+ *       kernel here is launched with programmatic dependent launch, so its
+ *       thread blocks can start while the stream's previous kernel drains;
+ *       with this flag the stream kernel (the chunk of a carried stream: few
+ *       lane blocks, up to 8 parts of 256 bfloat16 / 128 float32 tokens)
+ *       loads its inputs and forms every segment summary and prefix before
+ *       it waits for that kernel, and only the state fold and the outputs
+ *       wait.  state_in (written by the previous chunk), y and state_out are
+ *       touched only after the wait, so chaining chunks with the state in
+ *       place stays correct.  Without the flag, every kernel waits for the
+ *       previous kernel before its first memory access.  Setting it while
+ *       an input is still being written gives wrong results.
+ */
+#define WKV_FLAG_INPUTS_READY 1u
+
+int wkv_forward_ex(int64_t B, int64_t T, int64_t C, int dtype,
+                   const float* w, const float* u,
+                   const void* k, const void* v, const void* r,
+                   const float* state_in, void* y, float* state_out,
+                   void* workspace, size_t workspace_bytes, unsigned flags,
+                   cudaStream_t stream);
+
 /* Bytes of workspace wkv_forward needs for these sizes (0: none).  Returns 0
  * for invalid sizes too; wkv_forward then reports the argument error. */
 size_t wkv_forward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype);
@@ -337,6 +365,48 @@ const char* wkv_last_cuda_error(void);
 
 /* ABI version of this header: 1. */
 int wkv_abi_version(void);
+
+/*
+ * wkv5_forward -- multi-head WKV with matrix-valued states (the v5 "Eagle"
+ * and v6 "Finch" generations of the article's "RWKVバージョンの進化 / v4から
+ * v7まで": "multi-headed WKV, matrix-valued states" of h * (d/h)^2 numbers
+ * per layer, and "data-dependent time decay").  The pages give no formula
+ * beyond that line; this library reads it as follows.  Channels form H heads
+ * of N = C / H; each head of each sequence keeps an N x N state S (key
+ * channel i, value channel j).  Token t reads the state before its own
+ * update, as the v4 operator's parallel loop does ("並列学習の定式化"), and
+ * then every key row decays by e^{-w_t[i]} and the token's outer product is
+ * added:
+ *
+ *   y[b,t,hN+j] = sum_i r_t[i] ( S[i][j] + u[hN+i] k_t[i] v_t[j] )
+ *   S[i][j]    <- e^{-w_t[i]} S[i][j] + k_t[i] v_t[j]
+ *
+ * (r_t, k_t, v_t, w_t: the head's N channels of token t.)  There is no
+ * normalising denominator and no exponential of k: with one channel per
+ * head, k = e^{k4}, u = e^{u4} and r = 1 this is the v4 sum's numerator.
+ *
+ *   B, T, C, H   sizes; C % H == 0 and N = C / H is 32 or 64 (the pages' head
+ *                size is 64); B == 0 or C == 0: nothing to do; T == 0:
+ *                state_out = state_in (zeros if NULL).
+ *   dtype        wkv_dtype of r, k, v, y.
+ *   w            decay rates (>= 0), float32: (C,) when w_per_token == 0
+ *                (v5), (B,T,C) when w_per_token != 0 (v6).
+ *   u            (C,) float32 bonus.
+ *   r, k, v      (B,T,C) device arrays in dtype.
+ *   state_in     (B,H,N,N) float32 or NULL (zeros); S[b][h][i][j].
+ *   y            (B,T,C) output in dtype (computed in float32, rounded once).
+ *   state_out    (B,H,N,N) float32 or NULL; may equal state_in, must not
+ *                overlap anything else.  Feeding it back as the next call's
+ *                state_in chains chunks exactly like one pass.
+ * Errors as wkv_forward (WKV_ERR_SHAPE for a head size other than 32 or 64).
+ * The recurrence runs in float32 on the CUDA cores: 2 N multiply-adds per
+ * element.  Asynchronous on `stream`; no workspace.
+ */
+int wkv5_forward(int64_t B, int64_t T, int64_t C, int64_t H, int dtype,
+                 const float* w, int w_per_token, const float* u,
+                 const void* r, const void* k, const void* v,
+                 const float* state_in, void* y, float* state_out,
+                 cudaStream_t stream);
 
 /*
  * wkv_token_shift -- the token shift that precedes the R, K, V projections of

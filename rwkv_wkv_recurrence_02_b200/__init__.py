@@ -30,9 +30,9 @@ STATUS = {
     -8: "WKV_ERR_WORKSPACE", -9: "WKV_ERR_SCRATCH",
 }
 # the functions include/wkv.h declares
-EXPORTS = ("wkv_forward", "wkv_forward_workspace_bytes", "wkv_workspace_init", "wkv_workspace_status",
+EXPORTS = ("wkv_forward", "wkv_forward_ex", "wkv_forward_workspace_bytes", "wkv_workspace_init", "wkv_workspace_status",
            "wkv_step", "wkv_forward_noalloc", "wkv_forward_noalloc_scratch_bytes", "wkv_forward_noalloc_status",
-           "wkv_backward", "wkv_state", "wkv_state_combine",
+           "wkv_backward", "wkv_state", "wkv_state_combine", "wkv5_forward",
            "wkv_backward_workspace_bytes", "wkv_token_shift", "wkv_strerror", "wkv_last_cuda_error",
            "wkv_abi_version")
 
@@ -65,6 +65,8 @@ def lib():
         i64, vp, i32, sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         L.wkv_forward.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.wkv_forward.restype = i32
+        L.wkv_forward_ex.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.c_uint, vp]
+        L.wkv_forward_ex.restype = i32
         L.wkv_forward_workspace_bytes.argtypes = [i64, i64, i64, i32]
         L.wkv_forward_workspace_bytes.restype = sz
         L.wkv_workspace_init.argtypes = [vp, sz, vp]
@@ -83,6 +85,8 @@ def lib():
         L.wkv_state.restype = i32
         L.wkv_state_combine.argtypes = [i64, i64, i32, vp, vp, vp, vp, vp, vp]
         L.wkv_state_combine.restype = i32
+        L.wkv5_forward.argtypes = [i64, i64, i64, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.wkv5_forward.restype = i32
         L.wkv_forward_noalloc_status.argtypes = [vp]
         L.wkv_forward_noalloc_status.restype = i32
         L.wkv_backward.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
@@ -203,13 +207,18 @@ def workspace_bytes(B: int, T: int, C: int, dtype_code: int) -> int:
     return int(lib().wkv_forward_workspace_bytes(B, T, C, dtype_code))
 
 
+WKV_FLAG_INPUTS_READY = 1
+
+
 def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, want_state=True,
-                workspace: Workspace = None, use_workspace=True, stream=None):
+                workspace: Workspace = None, use_workspace=True, inputs_ready=False, stream=None):
     """Parallel mode over one chunk.  k, v, r: (B, T, C) CUDA tensors (float32
     or bfloat16); w, u: (C,) float32; state_in: (3, B, C) float32 or None.
     Returns (y, state_out) (state_out None if want_state is False and none
     was given).  state_out may be state_in for an in-place update.
-    use_workspace=False passes no workspace (the scratch-free schedules)."""
+    use_workspace=False passes no workspace (the scratch-free schedules).
+    inputs_ready=True passes WKV_FLAG_INPUTS_READY: k, v, r, w, u are not
+    written by work still running on the stream (see include/wkv.h)."""
     torch = _torch()
     if k.dim() != 3:
         raise ValueError("k must be (B, T, C)")
@@ -236,8 +245,13 @@ def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, wa
         ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
     else:
         ws_ptr, ws_bytes = None, 0
-    _check(lib().wkv_forward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
-                             _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, sp), "wkv_forward")
+    if inputs_ready:
+        _check(lib().wkv_forward_ex(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
+                                    _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, WKV_FLAG_INPUTS_READY, sp),
+               "wkv_forward_ex")
+    else:
+        _check(lib().wkv_forward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
+                                 _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, sp), "wkv_forward")
     return y, state_out
 
 
@@ -315,6 +329,39 @@ def wkv_state_combine(w, lens, states, state_in=None, *, state_out=None, stream=
     _check(lib().wkv_state_combine(B, C, n, _ptr(w), arr, _ptr(states), _ptr(state_in), _ptr(state_out),
                                    _stream_ptr(stream, dev)), "wkv_state_combine")
     return state_out
+
+
+def wkv5_forward(w, u, r, k, v, H, state_in=None, *, y=None, state_out=None, want_state=True, stream=None):
+    """Multi-head matrix-state WKV (v5 / v6).  r, k, v: (B, T, C) float32 or
+    bfloat16 CUDA tensors, C = H * N with N in {32, 64}; w: (C,) decay rates
+    (v5) or (B, T, C) float32 per token (v6); u: (C,) float32; state_in:
+    (B, H, N, N) float32 or None (zeros).  Returns (y, state_out)."""
+    torch = _torch()
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    if C % H != 0:
+        raise ValueError("C must be a multiple of H")
+    N = C // H
+    dev = k.device
+    if dev.type != "cuda":
+        raise ValueError("wkv5_forward runs on CUDA tensors only")
+    code = _dtype_code(k)
+    for t, name in ((r, "r"), (v, "v"), (k, "k")):
+        _need(t, name, (B, T, C), k.dtype, dev)
+    per_token = w.dim() == 3
+    _need(w, "w", (B, T, C) if per_token else (C,), torch.float32, dev)
+    _need(u, "u", (C,), torch.float32, dev)
+    _need(state_in, "state_in", (B, H, N, N), torch.float32, dev)
+    if y is None:
+        y = torch.empty((B, T, C), dtype=k.dtype, device=dev)
+    _need(y, "y", (B, T, C), k.dtype, dev)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, N, N), dtype=torch.float32, device=dev)
+    _need(state_out, "state_out", (B, H, N, N), torch.float32, dev)
+    _check(lib().wkv5_forward(B, T, C, H, code, _ptr(w), int(per_token), _ptr(u), _ptr(r), _ptr(k), _ptr(v),
+                              _ptr(state_in), _ptr(y), _ptr(state_out), _stream_ptr(stream, dev)), "wkv5_forward")
+    return y, state_out
 
 
 def wkv_forward_noalloc_status(stream=None, device=None) -> int:

@@ -17,10 +17,12 @@
 #include "wkv_lane.cuh"
 #include "wkv_part.cuh"
 #include "wkv_cluster.cuh"
+#include "wkv_stream.cuh"
 #include "wkv_backward.cuh"
 #include "wkv_seq.cuh"
 #include "wkv_step.cuh"
 #include "wkv_shift.cuh"
+#include "wkv5.cuh"
 
 namespace {
 
@@ -59,6 +61,14 @@ constexpr int kClusterLS = 32;
 constexpr int kClusterPT = kClusterW * kClusterLS;
 constexpr int kClusterMax = 8;
 constexpr int kClusterMinBlocks = 4;
+// Stream kernel: 8 compute warps x LS-token segments (32 for bfloat16, 16 for
+// float32: 32 registers of k either way), one CTA per part, at most 8 parts
+// (a portable cluster) per call.
+constexpr int kStreamW = 8;
+constexpr int kStreamMax = 8;
+template <typename IO>
+constexpr int stream_ls() { return sizeof(IO) == 2 ? 32 : 16; }
+constexpr int64_t stream_pt(int dtype) { return kStreamW * (dtype == WKV_BF16 ? 32 : 16); }
 // Sequences at most this long take the sequential kernel.
 constexpr int64_t kSeqMaxT = 16;
 // Limit of every wait on another CTA's result: 1 s, or WKV_WAIT_LIMIT_NS (read
@@ -230,10 +240,10 @@ bool fits_cluster(int dtype, int64_t B, int64_t T, int64_t C, const void* k, con
 }
 
 // Kernel choice: 0 = automatic; the environment variable WKV_FORWARD_KERNEL
-// (seq | chunk | part | lane | cluster) forces one, for ablation
+// (seq | chunk | part | lane | cluster | stream) forces one, for ablation
 // measurements: chunk = register-load look-back kernel, part = part kernel,
-// lane = lane-resident kernel, each even where another would run; cluster =
-// cluster kernel wherever every sequence fits one cluster.
+// lane = lane-resident kernel, each even where another would run; cluster /
+// stream = cluster or stream kernel wherever every sequence fits one cluster.
 int forced_kernel() {
     static int f = []() {
         const char* e = std::getenv("WKV_FORWARD_KERNEL");
@@ -243,6 +253,7 @@ int forced_kernel() {
         if (std::strcmp(e, "part") == 0) return 5;
         if (std::strcmp(e, "lane") == 0) return 6;
         if (std::strcmp(e, "cluster") == 0) return 7;
+        if (std::strcmp(e, "stream") == 0) return 8;
         return 0;
     }();
     return f;
@@ -431,6 +442,63 @@ int dispatch_cluster(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, si
                 : launch_cluster<IO, false>(a, dtype, ws, ws_bytes, st);
 }
 
+// Stream kernel: one cluster of ceil(T / PT) CTAs per lane block.
+template <typename IO, bool GATE>
+int launch_stream(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+    constexpr int LS = stream_ls<IO>();
+    using G = wkv::StreamGeometry<IO, GATE, kStreamW, LS>;
+    auto kern = wkv::stream_forward_kernel<IO, GATE, kStreamW, LS, 3>;
+    static bool ready[kMaxDevices] = {false};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (!ready[dev]) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        ready[dev] = true;
+    }
+    const ChunkGeom g = chunk_geom(a.B, a.T, a.C, 2, G::PT);
+    if (g.nchunks < 1 || g.nchunks > kStreamMax || g.units > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    a.nCB = g.nCB;
+    a.nLB = g.nLB;
+    a.nchunks = g.nchunks;
+    a.units = g.units;
+    a.hdr = workspace != nullptr && aligned(workspace, 256) && workspace_bytes >= sizeof(wkv::WsHeader)
+                ? reinterpret_cast<wkv::WsHeader*>(workspace)
+                : nullptr;
+    a.aggw = nullptr;
+    a.incw = nullptr;
+    CUtensorMap tv, tr;
+    if (!encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
+    if (GATE) {
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
+    } else {
+        tr = tv;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(g.units));
+    cfg.blockDim = dim3(G::THREADS);
+    cfg.dynamicSmemBytes = G::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(g.nchunks);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tv, tr, a));
+}
+
+template <typename IO>
+int dispatch_stream(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
+    return gate ? launch_stream<IO, true>(a, dtype, ws, ws_bytes, st)
+                : launch_stream<IO, false>(a, dtype, ws, ws_bytes, st);
+}
+
 // Part buffers per CTA: as many as fit beside kPartMinBlocks CTAs per SM
 // (up to three), at least one.
 template <typename IO, bool GATE>
@@ -545,7 +613,7 @@ int forward_args(int64_t B, int64_t T, int64_t C, int dtype, const float* w, con
 
 int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u, const void* k,
                 const void* v, const void* r, const float* state_in, void* y, float* state_out, void* workspace,
-                size_t workspace_bytes, cudaStream_t stream);
+                size_t workspace_bytes, unsigned flags, cudaStream_t stream);
 
 }  // namespace
 
@@ -602,7 +670,16 @@ int wkv_workspace_status(const void* workspace, cudaStream_t stream) {
 int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
                 const void* k, const void* v, const void* r, const float* state_in, void* y,
                 float* state_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return wkv_forward_ex(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, workspace, workspace_bytes, 0u,
+                          stream);
+}
+
+int wkv_forward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                   const void* k, const void* v, const void* r, const float* state_in, void* y,
+                   float* state_out, void* workspace, size_t workspace_bytes, unsigned flags,
+                   cudaStream_t stream) {
     if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    if ((flags & ~unsigned(WKV_FLAG_INPUTS_READY)) != 0) return WKV_ERR_SHAPE;
     int64_t n = 0;
     if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
     if (B == 0 || C == 0) return WKV_OK;
@@ -620,7 +697,8 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     }
     const int vrc = forward_args(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out);
     if (vrc != WKV_OK) return vrc;
-    return run_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, workspace, workspace_bytes, stream);
+    return run_forward(B, T, C, dtype, w, u, k, v, r, state_in, y, state_out, workspace, workspace_bytes, flags,
+                       stream);
 }
 
 }  // extern "C"
@@ -631,7 +709,7 @@ namespace {
 // checks (B, C, T >= 1).  y == nullptr: only the state is wanted.
 int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u, const void* k,
                 const void* v, const void* r, const float* state_in, void* y, float* state_out, void* workspace,
-                size_t workspace_bytes, cudaStream_t stream) {
+                size_t workspace_bytes, unsigned flags, cudaStream_t stream) {
     const void* io[] = {k, v, r, y};
     const float* f32[] = {w, u, state_in, state_out};
     const int V = pick_vec(C, dtype, io, 4, f32, 4);
@@ -651,6 +729,7 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     a.T = T;
     a.C = C;
     a.wait_limit_ns = wait_limit_ns();
+    a.early = (flags & WKV_FLAG_INPUTS_READY) ? 1u : 0u;
     int64_t grid = 0;
     if (!seq) {
         const bool tma = force != 2 && tma_eligible(V, dtype, B, T, C, k, v, r, w, u, state_in);
@@ -665,6 +744,20 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
         // measured a little faster on the streaming chunk.
         const bool cluster_ok = part_ok && (T + kClusterPT - 1) / kClusterPT <= kClusterMax;
         const bool ws_ok = workspace != nullptr && workspace_bytes >= wkv_forward_workspace_bytes(B, T, C, dtype);
+        // Few lane blocks and a call that fits one cluster of stream-kernel
+        // parts (a chunk of a carried stream): the stream kernel, which needs
+        // no workspace and, with WKV_FLAG_INPUTS_READY, does everything but
+        // the entering state's fold and the outputs before the previous
+        // kernel of the stream ends.
+        const int64_t spt = stream_pt(dtype);
+        const size_t eb = elem_bytes(dtype);
+        const bool stream_ok = part_ok && C % 2 == 0 && aligned(y, 2 * eb) &&
+                               (state_out == nullptr || aligned(state_out, 8)) && (T + spt - 1) / spt <= kStreamMax;
+        if (stream_ok && (force == 8 || (force == 0 && nLB < sm_count()))) {
+            return dtype == WKV_F32
+                       ? dispatch_stream<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
+                       : dispatch_stream<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
+        }
         if (cluster_ok && (force == 7 || (force == 0 && !ws_ok))) {
             return dtype == WKV_F32
                        ? dispatch_cluster<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
@@ -767,7 +860,7 @@ int wkv_state(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const 
     // finite row would do; it only steers the choice between two evaluations
     // of the same summary), no gate, no output
     return run_forward(B, T, C, dtype, w, w, k, v, nullptr, state_in, nullptr, state_out, workspace,
-                       workspace_bytes, stream);
+                       workspace_bytes, 0u, stream);
 }
 
 int wkv_state_combine(int64_t B, int64_t C, int n, const float* w, const int64_t* lens, const float* states,
@@ -1178,6 +1271,108 @@ int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, con
     }
     wkv::bwd_reduce_kernel<<<static_cast<unsigned>((C + 255) / 256), 256, 0, stream>>>(b.part, B, C, L.nCB, dw, du);
     return check_launch();
+}
+
+}  // extern "C"
+
+
+// ---------------------------------------------------------------------------
+// multi-head matrix-state WKV (v5 / v6)
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kWkv5TB = 32;
+
+template <typename IO, int N, bool PERTOK>
+int launch_wkv5(const wkv::Wkv5Args& a, cudaStream_t st) {
+    using G = wkv::Wkv5Geometry<N, kWkv5TB>;
+    auto kern = wkv::wkv5_forward_kernel<IO, N, kWkv5TB, PERTOK>;
+    static bool ready[kMaxDevices] = {false};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (!ready[dev]) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+        if (rc != WKV_OK) return rc;
+        ready[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.H));
+    cfg.blockDim = dim3(G::THREADS);
+    cfg.dynamicSmemBytes = G::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return record_cuda(cudaLaunchKernelEx(&cfg, kern, a));
+}
+
+template <typename IO, int N>
+int dispatch_wkv5(bool pertok, const wkv::Wkv5Args& a, cudaStream_t st) {
+    return pertok ? launch_wkv5<IO, N, true>(a, st) : launch_wkv5<IO, N, false>(a, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int wkv5_forward(int64_t B, int64_t T, int64_t C, int64_t H, int dtype, const float* w, int w_per_token,
+                 const float* u, const void* r, const void* k, const void* v, const float* state_in, void* y,
+                 float* state_out, cudaStream_t stream) {
+    if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
+    int64_t n = 0;
+    if (!mul_ok(B, T, C, &n) || H <= 0 || C % H != 0) return WKV_ERR_SHAPE;
+    const int64_t N = C / H;
+    if (B == 0 || C == 0) return WKV_OK;
+    if (N != 32 && N != 64) return WKV_ERR_SHAPE;
+    if (B * H > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    const size_t st_bytes = size_t(B) * size_t(H) * size_t(N) * size_t(N) * 4;
+    if (T == 0) {
+        if (state_out == nullptr || state_out == state_in) return WKV_OK;
+        if (!aligned(state_out, 4) || (state_in && !aligned(state_in, 4))) return WKV_ERR_ALIGN;
+        if (state_in && overlaps(state_in, st_bytes, state_out, st_bytes)) return WKV_ERR_ALIAS;
+        if (state_in) return record_cuda(cudaMemcpyAsync(state_out, state_in, st_bytes, cudaMemcpyDeviceToDevice, stream));
+        return record_cuda(cudaMemsetAsync(state_out, 0, st_bytes, stream));
+    }
+    if (!w || !u || !r || !k || !v || !y) return WKV_ERR_NULLPTR;
+    const size_t eb = elem_bytes(dtype);
+    const size_t io_bytes = size_t(n) * eb, p_bytes = size_t(C) * 4;
+    const size_t w_bytes = w_per_token ? size_t(n) * 4 : p_bytes;
+    if (!aligned(w, 4) || !aligned(u, 4) || !aligned(r, eb) || !aligned(k, eb) || !aligned(v, eb) ||
+        !aligned(y, eb) || (state_in && !aligned(state_in, 4)) || (state_out && !aligned(state_out, 4)))
+        return WKV_ERR_ALIGN;
+    struct Span { const void* p; size_t n; };
+    const Span ins[] = {{w, w_bytes}, {u, p_bytes}, {r, io_bytes}, {k, io_bytes}, {v, io_bytes}};
+    for (const Span& i : ins) {
+        if (overlaps(y, io_bytes, i.p, i.n)) return WKV_ERR_ALIAS;
+        if (state_out && overlaps(state_out, st_bytes, i.p, i.n)) return WKV_ERR_ALIAS;
+    }
+    if (overlaps(y, io_bytes, state_in, st_bytes) || overlaps(y, io_bytes, state_out, st_bytes)) return WKV_ERR_ALIAS;
+    if (state_out && state_in && state_in != state_out && overlaps(state_out, st_bytes, state_in, st_bytes))
+        return WKV_ERR_ALIAS;
+    wkv::Wkv5Args a{};
+    a.w = w;
+    a.u = u;
+    a.r = r;
+    a.k = k;
+    a.v = v;
+    a.s_in = state_in;
+    a.y = y;
+    a.s_out = state_out;
+    a.B = B;
+    a.T = T;
+    a.C = C;
+    a.H = H;
+    const bool pt = w_per_token != 0;
+    int rc;
+    if (dtype == WKV_F32)
+        rc = N == 64 ? dispatch_wkv5<float, 64>(pt, a, stream) : dispatch_wkv5<float, 32>(pt, a, stream);
+    else
+        rc = N == 64 ? dispatch_wkv5<__nv_bfloat16, 64>(pt, a, stream) : dispatch_wkv5<__nv_bfloat16, 32>(pt, a, stream);
+    return rc != WKV_OK ? rc : check_launch();
 }
 
 }  // extern "C"

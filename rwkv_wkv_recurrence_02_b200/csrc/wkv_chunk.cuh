@@ -90,6 +90,7 @@ struct ChunkArgs {
     St* ckpt;           // lane-resident kernel only, or null: [nchunks + 1][nLB][CB] base-2 states
                         // entering each chunk, the last one the state after the sequence
     uint64_t wait_limit_ns;
+    uint32_t early;     // stream kernel: inputs may be read before the previous kernel of the stream ends
 };
 
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {

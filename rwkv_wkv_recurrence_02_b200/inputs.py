@@ -24,6 +24,15 @@ measured on; N(m, s) means mean m and standard deviation s):
 
 w = exp(decay) is the parameterisation of the decay (w > 0); it is formed
 here once, in float32, because the library takes w itself.
+
+Matrix-state workloads (multi-head WKV, v5 / v6), from the training
+configuration on the pages (n_embd 2048, head size 64, context 4096):
+
+  v5_layer    B=8, T=4096, C=2048 in H=32 heads of 64, bf16 r/k/v, fp32 state,
+              decay rate w = exp(d) per channel with d ~ U(-4, 0.5),
+              u ~ N(0, 1), r, k, v ~ N(0, 1), fresh (zero) state.
+  v6_layer    the same with a decay rate per token and channel,
+              w = exp(d), d ~ U(-4, 0.5) drawn per element (float32).
 """
 from dataclasses import dataclass
 from typing import Optional
@@ -165,3 +174,49 @@ def fresh_state(B: int, C: int, layers: int = 0, device="cpu"):
     s = torch.zeros(shape, dtype=torch.float32, device=device)
     s[..., 2, :, :] = -1e38
     return s
+
+
+@dataclass(frozen=True)
+class MatrixWorkload:
+    name: str
+    B: int
+    T: int
+    C: int
+    H: int
+    dtype: str            # "f32" or "bf16": dtype of r, k, v, y
+    per_token_decay: bool
+    decay_lo: float = -4.0
+    decay_hi: float = 0.5
+    seed: int = 0
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == "f32" else 2
+
+
+MATRIX_WORKLOADS = {
+    "v5_layer": MatrixWorkload("v5_layer", 8, 4096, 2048, 32, "bf16", False, seed=1005),
+    "v6_layer": MatrixWorkload("v6_layer", 8, 4096, 2048, 32, "bf16", True, seed=1006),
+}
+
+
+def make_matrix_inputs(wl, B=None, T=None, C=None, H=None, device="cpu", seed_offset: int = 0, state=False):
+    """r, k, v (B, T, C) in the workload's dtype, w (C,) or (B, T, C) and u
+    (C,) float32, and the state (B, H, N, N) float32 (None unless `state`)."""
+    B = wl.B if B is None else B
+    T = wl.T if T is None else T
+    C = wl.C if C is None else C
+    H = wl.H if H is None else H
+    g = _gen(device, wl.seed * 1000 + seed_offset * 7 + 3)
+    wshape = (B, T, C) if wl.per_token_decay else (C,)
+    d = torch.empty(wshape, dtype=torch.float32, device=device).uniform_(wl.decay_lo, wl.decay_hi, generator=g)
+    w = torch.exp(d)
+    u = torch.randn((C,), dtype=torch.float32, device=device, generator=g)
+    r, k, v = (torch.randn((B, T, C), dtype=torch.float32, device=device, generator=g).to(wl.torch_dtype)
+               for _ in range(3))
+    s0 = torch.randn((B, H, C // H, C // H), dtype=torch.float32, device=device, generator=g) if state else None
+    return dict(w=w.contiguous(), u=u, r=r.contiguous(), k=k.contiguous(), v=v.contiguous(), state=s0)

@@ -39,6 +39,18 @@ def output_error(y_gpu, y_ref, scale):
     return float(np.max(np.abs(y - y_ref) / scale))
 
 
+def plain_relative_error(y_gpu, y_ref, scale, floor=1e-3):
+    """The plain relative error |y - y_ref| / |y_ref| over the outputs with
+    |y_ref| >= floor * scale (elsewhere y_ref is near a cancellation and the
+    plain ratio says nothing), and how many outputs that covers.  It is at
+    most the scale-relative error divided by `floor`."""
+    y = to_np64(y_gpu)
+    keep = np.abs(y_ref) >= floor * scale
+    if not np.any(keep):
+        return 0.0, 0
+    return float(np.max(np.abs(y - y_ref)[keep] / np.abs(y_ref)[keep])), int(keep.sum())
+
+
 def state_error(s_gpu, s_ref):
     """Errors of the state's represented quantities: ratio N/D (against the
     scale 1 + |N/D|) and log D, and of the running-max exponent p

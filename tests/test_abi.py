@@ -30,7 +30,7 @@ def _gpu_present():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s*(wkv_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s*(wkv[0-9]*_[a-z_0-9]+)\s*\(", text, flags=re.M)))
 
 
 @pytest.fixture(scope="module")
@@ -263,3 +263,19 @@ def test_state_combine_validation(L):
     assert call(ln=None) == NULLPTR and call(sg=None) == NULLPTR and call(w=None) == NULLPTR
     assert call(s_out=st + 2) == ALIGN
     assert call(s_out=seg + 64) == ALIAS                          # state_out inside the summaries
+
+
+def test_wkv5_validation(L):
+    y, st = BASE + (3 << 30), BASE + (5 << 30)
+    call = lambda B=2, T=10, C=128, H=2, dt=BF16, w=BASE, pt=0, u=BASE + 4096, r=BASE + (4 << 30), \
+        k=BASE + (1 << 30), v=BASE + (2 << 30), s_in=None, yy=y, s_out=st: \
+        L.wkv5_forward(B, T, C, H, dt, w, pt, u, r, k, v, s_in, yy, s_out, None)
+    assert call(dt=3) == DTYPE
+    assert call(H=0) == SHAPE and call(H=3) == SHAPE              # C not a multiple of H
+    assert call(C=96, H=2) == SHAPE                               # head size 48
+    assert call(B=0) == OK
+    assert call(r=None) == NULLPTR and call(w=None) == NULLPTR
+    assert call(k=BASE + (1 << 30) + 1) == ALIGN
+    assert call(yy=BASE + (1 << 30)) == ALIAS                     # y is k
+    assert call(s_out=BASE + (2 << 30) + 64) == ALIAS             # state_out inside v
+    assert call(pt=1, w=y - 64) == ALIAS                          # per-token w (B, T, C) runs into y

@@ -132,7 +132,7 @@ def test_reference_arm_prints_one_line():
     out = json.loads(lines[0])
     assert out["impl"] == "reference" and out["unit"] == "elements/s" and out["value"] > 0
     assert out["cpu_baseline"]["kind"] == "oracle" and out["e2e"]["h2d_bytes_per_step"] == 0
-    assert out["config"]["workload"] == "layer_1b5"
+    assert out["config"]["workload"] == "stream_1m" and out["config"]["T"] == 1 << 20
 
 
 def test_decode_forms_and_graph_period():
@@ -215,3 +215,21 @@ def test_token_shift_bytes_and_reference_arm(capsys):
 def test_token_shift_cpu_baseline_is_bounded():
     r = bench.cpu_baseline_shift("layer_1b5", 0.5)
     assert r["value"] > 0 and r["kind"] == "oracle" and "mixes" in r["sample"]
+
+
+def test_defaults_follow_the_workload():
+    a = bench.parse_args([])
+    assert a.workload == "stream_1m" and a.steps == 20 and a.warmup == 5
+    b = bench.parse_args(["--workload", "layer_1b5"])
+    assert b.steps == 3000 and b.warmup == 20
+    c = bench.parse_args(["--gpus", "1", "--steps", "20", "--warmup", "5"])
+    assert (c.steps, c.warmup, c.workload) == (20, 5, "stream_1m")
+
+
+def test_whole_stream_bytes_and_names():
+    wl = bench.workload("stream_1m")
+    assert bench.whole_stream("stream_1m") and not bench.whole_stream("stream_1m_chunk")
+    assert wl.T == 1 << 20 and wl.chunk == 1024 and wl.T // wl.chunk == 1024
+    assert bench.workload("stream_1m_chunk").chunk == 1024
+    # per launch (one chunk): k, v read, y written (2 B each), state in and out, w and u
+    assert bench.algorithmic_bytes(wl, 1, wl.chunk, wl.C) == 1024 * 4096 * 6 + 4096 * 24 + 4096 * 8

@@ -5,8 +5,10 @@ with the oracle on the same seeded inputs.
 
 - part: short sequences of few lane blocks, which take the cluster kernel
   when the call brings no workspace (at most 64 tokens need none);
-- cluster: many lane blocks (more clusters than fit the GPU at once), which
-  with a workspace take the lane-resident kernel.
+- cluster: few lane blocks (where the stream kernel runs) and many (more
+  clusters than fit the GPU at once), which with a workspace take the
+  lane-resident kernel;
+- stream: many lane blocks, which take the lane-resident kernel.
 """
 import os
 import subprocess
@@ -47,11 +49,21 @@ FORCED = {
         (3, 777, 1000, "bfloat16", False, True),
     ],
     "cluster": [
+        (1, 100, 64, "float32", True, True),         # few lane blocks (where the stream kernel runs by default)
+        (2, 1000, 72, "bfloat16", True, True),
+        (1, 1024, 4096, "bfloat16", False, True),
         (40, 130, 256, "bfloat16", True, False),     # 160 lane blocks
         (160, 64, 64, "float32", False, True),
         (300, 40, 64, "bfloat16", True, True),
         (5, 1000, 3840, "float32", True, True),      # 300 clusters of 8 CTAs
         (7, 130, 2728, "bfloat16", True, True),      # ragged channel block
+    ],
+    "stream": [
+        (40, 130, 256, "bfloat16", True, False),     # 160 lane blocks: more clusters than fit at once
+        (300, 40, 64, "bfloat16", True, True),
+        (5, 1000, 3840, "float32", True, True),      # 300 clusters of 8 CTAs
+        (7, 130, 2728, "bfloat16", True, True),      # ragged channel block
+        (3, 2048, 4096, "bfloat16", False, True),    # 8 parts of 256 tokens, 192 lane blocks
     ],
 }
 

@@ -12,8 +12,8 @@ import torch
 import oracle
 import rwkv_wkv_recurrence_02_b200 as wkv
 from rwkv_wkv_recurrence_02_b200 import inputs as I
-from tests.parity import (TOL, argmax_index, gpu_argmax_index, oracle_forward, output_error, sample_channels,
-                          state_error, to_np32, to_np64)
+from tests.parity import (TOL, argmax_index, gpu_argmax_index, oracle_forward, output_error, plain_relative_error,
+                          sample_channels, state_error, to_np32, to_np64)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,11 +33,16 @@ def run_forward(d, **kw):
     return y, s
 
 
-def check_forward(d, y, s, tol=None, state_tol=None):
+def check_forward(d, y, s, tol=None, state_tol=None, report=None):
     tol = TOL[d["k"].dtype] if tol is None else tol
     y_ref, s_ref, scale = oracle_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"])
     err = output_error(y, y_ref, scale)
     assert err <= tol, f"output error {err:.3e} > {tol:.1e}"
+    plain, covered = plain_relative_error(y, y_ref, scale)
+    assert plain <= tol / 1e-3
+    if report is not None:
+        report(f"scale-relative error {err:.3e}; plain relative error {plain:.3e} over {covered} outputs "
+               f"with |y| >= 1e-3 s")
     if s is not None:
         ratio, logd, pe = state_error(s, s_ref)
         st = tol if state_tol is None else state_tol
@@ -163,6 +168,51 @@ def test_cluster_chain_in_place_equals_one_call():
         sl = slice(i * 1000, (i + 1) * 1000)
         wkv.wkv_forward_noalloc(d["w"], d["u"], d["k"][:, sl], d["v"][:, sl], d["r"][:, sl], state, y=y[:, sl],
                                 state_out=state)
+    torch.cuda.synchronize()
+    check_forward(d, y, state)
+
+
+# Few lane blocks and at most 8 parts of 256 (bf16) / 128 (fp32) tokens: the
+# stream kernel, one cluster per lane block.  With inputs_ready it forms
+# every summary before waiting for the previous kernel of the stream.
+STREAM = [
+    # B, T, C, dtype, gate, state
+    (1, 17, 64, torch.float32, True, True),        # one part, shorter than a segment run
+    (1, 256, 64, torch.bfloat16, False, True),     # exactly one part
+    (1, 257, 128, torch.bfloat16, True, False),    # one token in the second part
+    (2, 1000, 72, torch.bfloat16, True, True),     # ragged channel block and last part
+    (1, 1024, 4096, torch.bfloat16, False, True),  # the streaming workload's chunk shape
+    (1, 1024, 4096, torch.float32, True, True),    # fp32: eight parts of 128 tokens
+    (2, 2048, 4096, torch.bfloat16, True, False),  # eight parts of 256 tokens
+    (3, 777, 1000, torch.float32, False, True),
+    (1, 300, 200, torch.bfloat16, True, True),
+]
+
+
+@pytest.mark.parametrize("ready", [False, True])
+@pytest.mark.parametrize("B,T,C,dtype,gate,state", STREAM)
+def test_stream_kernel_shapes(B, T, C, dtype, gate, state, ready):
+    d = gen_case(B, T, C, dtype, gate, state, seed=B * 23 + T + C)
+    y, s = run_forward(d, inputs_ready=ready)
+    check_forward(d, y, s)
+
+
+@pytest.mark.parametrize("ready", [False, True])
+def test_stream_chain_in_place_equals_one_pass(ready):
+    """Chunks of one sequence through the stream kernel back to back with the
+    state carried in place, each chunk's inputs resident before the chain
+    starts (what WKV_FLAG_INPUTS_READY declares), against the oracle over the
+    whole sequence."""
+    n, T, C = 12, 1024, 512
+    d = gen_case(1, n * T, C, torch.bfloat16, False, True, seed=97)
+    d["k"][:, ::997] = 50.0    # outliers: the exact path inside a chain
+    state = d["state"].clone()
+    y = torch.empty_like(d["k"])
+    torch.cuda.synchronize()
+    for i in range(n):
+        sl = slice(i * T, (i + 1) * T)
+        wkv.wkv_forward(d["w"], d["u"], d["k"][:, sl], d["v"][:, sl], None, state, y=y[:, sl], state_out=state,
+                        inputs_ready=ready)
     torch.cuda.synchronize()
     check_forward(d, y, state)
 
@@ -324,12 +374,12 @@ def sampled(d, idx):
                 state=f(d["state"]))
 
 
-def test_layer_1b5_full():
+def test_layer_1b5_full(record_property):
     d = I.make_forward_inputs("layer_1b5", device=DEV)
     y, s = run_forward(d)
     idx = sample_channels(d["k"].shape[2], n=512)
     ds = sampled(d, idx)
-    check_forward(ds, y[..., idx.to(DEV)], s[..., idx.to(DEV)])
+    check_forward(ds, y[..., idx.to(DEV)], s[..., idx.to(DEV)], report=lambda m: record_property("errors", m))
     # the index of the term that sets the final running max
     T = d["k"].shape[1]
     j_ref, gap, cand = argmax_index(to_np32(ds["k"]), to_np32(ds["w"]), T, p0=to_np64(ds["state"][2]))
@@ -339,12 +389,12 @@ def test_layer_1b5_full():
     assert np.array_equal(j_gpu[clear], j_ref[clear])
 
 
-def test_layer_14b_full():
+def test_layer_14b_full(record_property):
     d = I.make_forward_inputs("layer_14b", device=DEV)
     y, s = run_forward(d)
     idx = sample_channels(d["k"].shape[2], n=64)
     ds = sampled(d, idx)
-    check_forward(ds, y[..., idx.to(DEV)], s[..., idx.to(DEV)])
+    check_forward(ds, y[..., idx.to(DEV)], s[..., idx.to(DEV)], report=lambda m: record_property("errors", m))
     T = d["k"].shape[1]
     j_ref, gap, cand = argmax_index(to_np32(ds["k"]), to_np32(ds["w"]), T)
     j_gpu = gpu_argmax_index(to_np64(s[2][..., idx.to(DEV)]), cand, 0)
@@ -352,7 +402,7 @@ def test_layer_14b_full():
     assert np.array_equal(j_gpu[clear], j_ref[clear])
 
 
-def test_stream_1m_chunked_equals_single_pass():
+def test_stream_1m_chunked_equals_single_pass(record_property):
     wl = I.WORKLOADS["stream_1m"]
     C, n = wl.C, wl.T // wl.chunk
     w, u = I.make_params(wl, device=DEV)
@@ -375,9 +425,20 @@ def test_stream_1m_chunked_equals_single_pass():
     for s in (s_single, state):
         ratio, logd, pe = state_error(s[..., dv], s_ref)
         assert max(ratio, logd, pe) <= 1e-3, (ratio, logd, pe)
+    # the index of the term that sets the final running max, on both
+    j_ref, gap, cand = argmax_index(to_np32(k[..., dv]), to_np32(w[dv]), wl.T)
+    clear = gap > 1e-2
+    assert clear.mean() > 0.9
+    for s in (s_single, state):
+        j_gpu = gpu_argmax_index(to_np64(s[2][..., dv]), cand, 0)
+        assert np.array_equal(j_gpu[clear], j_ref[clear])
+    del cand
     # chained and single pass agree everywhere, not only on sampled lanes
     diff = (y_single.float() - y_chain.float()).abs().max().item()
     assert diff <= 2e-2 * max(1.0, y_single.float().abs().max().item())
+    same = torch.equal(y_single, y_chain) and torch.equal(s_single, state)
+    record_property("chunked_vs_single_pass", "bit-identical" if same else
+                    f"not bit-identical (different kernels); largest difference {diff:.3e}")
 
 
 def test_decode_full():
@@ -390,7 +451,7 @@ def test_decode_full():
     g = np.random.default_rng(5)
     bsel = torch.tensor(sorted(g.choice(B, 8, replace=False)), device=DEV)
     csel = sample_channels(C, n=16).to(DEV)
-    steps = 200
+    steps = wl.steps
     ys = []
     for s in range(steps):
         a = I.decode_ring_start(wl, s)
@@ -416,3 +477,13 @@ def test_decode_full():
     so = np.stack(ost)                                       # (L, 3, nb, nc)
     ratio, logd, pe = state_error(torch.from_numpy(sg.transpose(1, 0, 2, 3).copy()), so.transpose(1, 0, 2, 3))
     assert max(ratio, logd, pe) <= 1e-3, (ratio, logd, pe)
+    # the index of the step whose key sets each layer's final running max
+    ring_rows = np.array([[(s * L + l) % wl.ring for s in range(steps)] for l in range(L)])   # (L, steps)
+    kn = to_np32(kr[:wl.ring][:, bsel][:, :, csel])                                        # (ring, nb, nc)
+    for l in range(L):
+        seq = kn[ring_rows[l]].transpose(1, 0, 2)                                          # (nb, steps, nc)
+        j_ref, gap, cand = argmax_index(seq, wn[l], steps)
+        j_gpu = gpu_argmax_index(sg[l, 2], cand, 0)
+        clear = gap > 1e-2
+        assert clear.mean() > 0.9
+        assert np.array_equal(j_gpu[clear], j_ref[clear]), l
