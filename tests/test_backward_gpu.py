@@ -4,8 +4,10 @@ reverse mode, on identical seeded inputs.
 Errors are measured per lane: the largest |gpu - oracle| over a lane's tokens
 divided by the largest |oracle| of that lane, so a small gradient next to a
 large one in the same lane is measured at the lane's scale.  dw, du and the
-state's gradient are divided by the larger of their own largest |oracle| and
-the call's largest |dv|.
+state's gradient are measured per channel (per lane for the state): each
+against its own |oracle|, floored at FLOOR times the largest |oracle| of the
+array (or of dv, where the array's sums cancel to zero), so a channel whose
+gradient is small is still checked at its own scale down to that floor.
 """
 import numpy as np
 import pytest
@@ -19,9 +21,12 @@ from tests.parity import to_np32, to_np64
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-# fp32: float32 recurrences over up to a few thousand tokens; bf16: outputs
-# rounded to bf16 (2^-8 relative) on top of that
-TOL = {torch.float32: 2e-3, torch.bfloat16: 2e-2}
+# Tolerances from the largest errors the kernels reach on the cases below,
+# with a margin of about 3x: float32 1.35e-4 (dw of one channel against its
+# own value; dk 7.2e-5 against its lane), bfloat16 3.9e-3 (dk, dv, dr: the
+# bf16 rounding of the outputs, 2^-8 relative).
+TOL = {torch.float32: 4e-4, torch.bfloat16: 1e-2}
+FLOOR = 1e-3
 
 
 def gen(B, T, C, dtype, gate, state, with_ds, seed):
@@ -62,14 +67,19 @@ def check(d, out, tol=None):
     if rr is not None:
         errs["dr"] = lane_error(dr, rr)
     # sums over many tokens can cancel to ~0 (T = 1 from the empty state:
-    # du = 0 exactly), so they are measured at the call's gradient scale too
+    # du = 0 exactly): the floor then comes from the call's dv scale
     g_scale = max(np.abs(rv).max(), 1e-30)
-    errs["dw"] = float(np.abs(to_np64(dw) - rw).max() / max(np.abs(rw).max(), g_scale))
-    errs["du"] = float(np.abs(to_np64(du) - ru).max() / max(np.abs(ru).max(), g_scale))
+
+    def per_element(got, ref):
+        ref = np.asarray(ref)
+        floor = FLOOR * max(np.abs(ref).max(), g_scale if np.abs(ref).max() == 0 else 0.0, 1e-30)
+        return float((np.abs(to_np64(got) - ref) / np.maximum(np.abs(ref), floor)).max())
+
+    errs["dw"] = per_element(dw, rw)
+    errs["du"] = per_element(du, ru)
     if dsi is not None and d["state"] is not None:
         for i, name in enumerate(("ds_a", "ds_b", "ds_p")):
-            scale = max(np.abs(rs[i]).max(), g_scale)
-            errs[name] = float(np.abs(to_np64(dsi[i]) - rs[i]).max() / scale)
+            errs[name] = per_element(dsi[i], rs[i])
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, (bad, errs)
     return errs
