@@ -469,12 +469,19 @@ int launch_stream(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace
                 : nullptr;
     a.aggw = nullptr;
     a.incw = nullptr;
-    CUtensorMap tv, tr;
+    CUtensorMap tk, tv, tr, ty;
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
     if (!encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
     if (GATE) {
         if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
     } else {
         tr = tv;
+    }
+    // outputs: one box of a warp's LS rows (no y when only the state is wanted)
+    if (a.y != nullptr) {
+        if (!encode_map(&ty, a.y, dtype, a.B, a.T, a.C, G::CB, LS)) return WKV_ERR_CUDA;
+    } else {
+        ty = tv;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(g.units));
@@ -490,7 +497,7 @@ int launch_stream(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tv, tr, a));
+    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tk, tv, tr, ty, a));
 }
 
 template <typename IO>
@@ -751,7 +758,7 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
         // kernel of the stream ends.
         const int64_t spt = stream_pt(dtype);
         const size_t eb = elem_bytes(dtype);
-        const bool stream_ok = part_ok && C % 2 == 0 && aligned(y, 2 * eb) &&
+        const bool stream_ok = part_ok && (y == nullptr || aligned(y, 16)) &&
                                (state_out == nullptr || aligned(state_out, 8)) && (T + spt - 1) / spt <= kStreamMax;
         if (stream_ok && (force == 8 || (force == 0 && nLB < sm_count()))) {
             return dtype == WKV_F32

@@ -10,12 +10,10 @@
 // independent of the state entering the chunk.  This kernel does all of that
 // first and only then touches the entering state:
 //
-//   load      k rows straight into registers (each thread: its two channels
-//             of its segment); the v (and r) tile of the part by one TMA copy
-//             into shared memory, w and u by bulk copies.
+//   load      the k, v (and r) tiles of the part by one TMA copy each into
+//             shared memory, w and u by bulk copies.
 //   pass 0/1  segment summary per warp (fixed-scale fast path, exact
-//             running-max fallback), from k in registers and v in shared
-//             memory.
+//             running-max fallback).
 //   fold      summaries of the warps before each warp (shared memory), the
 //             part's summary, and through distributed shared memory the
 //             summaries of the cluster's earlier parts: every warp ends with
@@ -23,12 +21,17 @@
 //   -------- the entering state is needed from here on --------
 //   state     each warp reads state_in for its channels and folds it with
 //             its prefix (one combine).
-//   pass 2    outputs: k from registers, v (and r) from shared memory; the
-//             per-token exponentials are recomputed rather than held, which
-//             keeps the kernel small enough that the next chunk's CTAs fit
-//             beside this chunk's.
+//   pass 2    outputs; the per-token exponentials are recomputed rather than
+//             held in registers, which keeps the kernel small enough that
+//             most of the next chunk's CTAs fit beside this chunk's.  Each
+//             output overwrites the v entry it was
+//             computed from, and every warp stores its finished rows with one
+//             TMA copy (rows and channels outside the arrays are clipped).
 //   state_out the last part's warp W-1 writes it, after a cluster barrier at
 //             which every CTA has read state_in (state_out may be state_in).
+//
+// Full parts (every segment LS tokens long) run a copy of the passes without
+// per-token bounds tests; a part that ends inside T takes the checked copy.
 //
 // One thread block cluster of P = ceil(T / PT) CTAs per 64-channel lane block,
 // one CTA per part of PT = W * LS tokens.  With the launch flag `early` (the
@@ -51,20 +54,206 @@ struct StreamGeometry {
     static constexpr int PT = W * LS;
     static constexpr int ROW = CB * static_cast<int>(sizeof(IO));
     static constexpr uint32_t TILE = PT * ROW;                 // one array's part tile
-    static constexpr int NT = GATE ? 2 : 1;                    // tiles in shared memory: v (, r)
+    static constexpr int NT = GATE ? 3 : 2;                    // tiles in shared memory: k, v (, r)
     static constexpr uint32_t PARAM = 2 * CB * sizeof(float);  // w, u of the lane block
     static constexpr uint32_t SMEM = NT * TILE + PARAM;
     static constexpr int THREADS = W * 32;
 };
 
-template <typename IO>
-__device__ __forceinline__ typename Vec<IO, 2>::raw ldg_pair(const IO* p) {
-    return Vec<IO, 2>::load(p);
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Per-thread values of one segment between the passes.
+template <int LS>
+struct StreamSeg {
+    float w2[2], u2[2], dk[2], eu[2];
+    float kmax[2], kmin[2];
+    bool fast1;
+};
+
+// Pass 0 + pass 1 of one warp's segment: key range, running-max exponent
+// and the segment's summary (fixed-scale fast path, or the exact running-max
+// recurrence when the keys span too wide a range).  FULL: every one of the
+// LS tokens is valid, so no per-token test.
+template <typename IO, int LS, bool FULL>
+__device__ __forceinline__ void stream_pass01(const unsigned char* krow, const unsigned char* vrow, int nvalid,
+                                              StreamSeg<LS>& sg, St* seg) {
+    using Raw = typename Vec<IO, 2>::raw;
+    constexpr int ROW = 64 * static_cast<int>(sizeof(IO));
+    auto kr = [&](int i) { return *reinterpret_cast<const Raw*>(krow + i * ROW); };
+    const F2 L2 = f2s(kLog2e);
+    const F2 W2 = f2(sg.w2[0], sg.w2[1]);
+    const int n = FULL ? LS : nvalid;
+    // ---- pass 0: q = max_i (k2_i - (n-1-i) w2), each candidate from one product ----
+    float kx[2] = {-3.0e38f, -3.0e38f}, kn[2] = {3.0e38f, 3.0e38f}, qm[2] = {-3.0e38f, -3.0e38f};
+#pragma unroll
+    for (int i = 0; i < LS; ++i) {
+        if (FULL || i < nvalid) {
+            const F2 kk = raw_pair<IO>(kr(i));
+            const F2 cand = fma2(kk, L2, mul2(f2s(static_cast<float>(i - (n - 1))), W2));
+            kx[0] = fmaxf(kx[0], f2lo(kk));
+            kx[1] = fmaxf(kx[1], f2hi(kk));
+            kn[0] = fminf(kn[0], f2lo(kk));
+            kn[1] = fminf(kn[1], f2hi(kk));
+            qm[0] = fmaxf(qm[0], f2lo(cand));
+            qm[1] = fmaxf(qm[1], f2hi(cand));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        sg.kmax[j] = kx[j] * kLog2e;
+        sg.kmin[j] = kn[j] * kLog2e;
+    }
+    sg.fast1 = (sg.kmax[0] - sg.kmin[0] + fabsf(sg.u2[0]) <= kFastSpan) &&
+               (sg.kmax[1] - sg.kmin[1] + fabsf(sg.u2[1]) <= kFastSpan);
+    // ---- pass 1: the segment's summary ----
+    if (sg.fast1) {
+        const F2 KM = f2(-sg.kmax[0], -sg.kmax[1]);
+        const F2 DK = f2(sg.dk[0], sg.dk[1]);
+        F2 nn = f2s(0.f), db = f2s(0.f);
+#pragma unroll
+        for (int i = 0; i < LS; ++i) {
+            if (FULL || i < nvalid) {
+                const F2 ek = ex2x2(fma2(raw_pair<IO>(kr(i)), L2, KM));
+                const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW)));
+                nn = fma2(nn, DK, ekv);
+                db = fma2(db, DK, ek);
+            }
+        }
+        const float sc0 = ex2(sg.kmax[0] - qm[0]), sc1 = ex2(sg.kmax[1] - qm[1]);
+        seg[0] = St{qm[0], f2lo(nn) * sc0, f2lo(db) * sc0};
+        seg[1] = St{qm[1], f2hi(nn) * sc1, f2hi(db) * sc1};
+    } else {
+        // keys too spread for one reference: the exact running-max recurrence
+        // with its exponent held as pb - m w2 (see lane_token_pm)
+        float pb[2], m[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            seg[j] = st_identity();
+            pb[j] = seg[j].p;
+            m[j] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < LS; ++i) {
+            if (FULL || i < nvalid) {
+                const F2 kk = raw_pair<IO>(kr(i));
+                const F2 vv = raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW));
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                    const float v1 = j == 0 ? f2lo(vv) : f2hi(vv);
+                    const float pd = fmaf(-(m[j] + 1.f), sg.w2[j], pb[j]);
+                    const float d2 = pd - k2;
+                    const float e = ex2(-fabsf(d2));
+                    if (d2 >= 0.f) {
+                        seg[j].a = fmaf(e, v1, seg[j].a);
+                        seg[j].b += e;
+                        m[j] += 1.f;
+                    } else {
+                        seg[j].a = fmaf(e, seg[j].a, v1);
+                        seg[j].b = fmaf(e, seg[j].b, 1.f);
+                        pb[j] = k2;
+                        m[j] = 0.f;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) seg[j].p = fmaf(-m[j], sg.w2[j], pb[j]);
+    }
+}
+
+// Pass 2 of one warp's segment: the outputs from the segment's start state
+// st, each written over the v entry it was computed from (in shared memory).
+template <typename IO, bool GATE, int LS, bool FULL>
+__device__ __forceinline__ void stream_pass2(const unsigned char* krow, unsigned char* vrow, const unsigned char* rrow,
+                                             int nvalid, const StreamSeg<LS>& sg, St* st) {
+    using Raw = typename Vec<IO, 2>::raw;
+    using Ld = Vec<IO, 2>;
+    constexpr int ROW = 64 * static_cast<int>(sizeof(IO));
+    auto kr = [&](int i) { return *reinterpret_cast<const Raw*>(krow + i * ROW); };
+    const F2 L2 = f2s(kLog2e);
+    bool fast2 = sg.fast1;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const bool near = st[j].p >= sg.kmax[j] - kFastState;
+        const bool negligible = st[j].p < sg.kmax[j] - 1.5f * kFastState && st[j].b <= 16777216.f;
+        fast2 = fast2 && (st[j].p - sg.kmin[j] + fabsf(sg.u2[j]) <= kFastState) && (near || negligible);
+    }
+    if (fast2) {
+        float nr[2], ss[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const float R = fmaxf(sg.kmax[j], st[j].p);
+            nr[j] = -R;
+            ss[j] = ex2(st[j].p - R);
+        }
+        const F2 NR = f2(nr[0], nr[1]);
+        const F2 EU = f2(sg.eu[0], sg.eu[1]);
+        const F2 DK = f2(sg.dk[0], sg.dk[1]);
+        const F2 NL = f2s(-kLog2e);
+        F2 n = f2(st[0].a * ss[0], st[1].a * ss[1]);
+        F2 db = f2(st[0].b * ss[0], st[1].b * ss[1]);
+#pragma unroll
+        for (int i = 0; i < LS; ++i) {
+            if (FULL || i < nvalid) {
+                Raw* vp = reinterpret_cast<Raw*>(vrow + i * ROW);
+                const F2 ek = ex2x2(fma2(raw_pair<IO>(kr(i)), L2, NR));
+                const F2 ekv = mul2(ek, raw_pair<IO>(*vp));
+                const F2 num = fma2(EU, ekv, n);
+                F2 den = fma2(EU, ek, db);
+                if (GATE) {
+                    const F2 g = ex2x2(mul2(raw_pair<IO>(*reinterpret_cast<const Raw*>(rrow + i * ROW)), NL));
+                    den = fma2(den, g, den);
+                }
+                const F2 y = mul2(num, rcpx2(den));
+                n = fma2(n, DK, ekv);
+                db = fma2(db, DK, ek);
+                const float out[2] = {f2lo(y), f2hi(y)};
+                Ld::store(reinterpret_cast<IO*>(vp), out);
+            }
+        }
+    } else {
+        float pb[2], m[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            pb[j] = st[j].p;
+            m[j] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < LS; ++i) {
+            if (FULL || i < nvalid) {
+                Raw* vp = reinterpret_cast<Raw*>(vrow + i * ROW);
+                const F2 kk = raw_pair<IO>(kr(i));
+                const F2 vv = raw_pair<IO>(*vp);
+                F2 rv = f2s(0.f);
+                if (GATE) rv = raw_pair<IO>(*reinterpret_cast<const Raw*>(rrow + i * ROW));
+                float out[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float gd = GATE ? gate_den(j == 0 ? f2lo(rv) : f2hi(rv)) : 1.f;
+                    const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
+                    out[j] = lane_token_pm(st[j].a, st[j].b, pb[j], m[j], sg.w2[j], sg.u2[j], k2,
+                                           j == 0 ? f2lo(vv) : f2hi(vv), gd);
+                }
+                Ld::store(reinterpret_cast<IO*>(vp), out);
+            }
+        }
+    }
 }
 
 template <typename IO, bool GATE, int W, int LS, int MINB>
 __global__ void __launch_bounds__(W * 32, MINB)
-stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tr,
+stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                      const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap ty,
                       const ChunkArgs A) {
     using G = StreamGeometry<IO, GATE, W, LS>;
     constexpr int V = 2;
@@ -72,7 +261,6 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_const
     constexpr int PT = G::PT;
     constexpr int ROW = G::ROW;
     using Raw = typename Vec<IO, V>::raw;
-    using Ld = Vec<IO, V>;
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ __align__(8) uint64_t full;
     __shared__ St s_seg[W][V][32];                   // segment summaries of the part
@@ -90,131 +278,56 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_const
     const float nan = __int_as_float(0x7fc00000);
 
     if (threadIdx.x == 0) {
+        prefetch_tensormap(&tk);
         prefetch_tensormap(&tv);
         if (GATE) prefetch_tensormap(&tr);
+        prefetch_tensormap(&ty);
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // ---- load: v (, r) tiles and w, u by TMA; k rows into registers ----
+    // ---- load: k, v (, r) tiles and w, u by TMA ----
     const int64_t t_part = q * PT;
     const int part_len = static_cast<int>(min(static_cast<int64_t>(PT), A.T - t_part));
+    const bool full_part = part_len == PT;
     float* prm = reinterpret_cast<float*>(smem + G::NT * G::TILE);
     if (threadIdx.x == 0) {
         mbar_init(&full, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         const uint32_t pbytes = static_cast<uint32_t>(min(static_cast<int64_t>(CB), A.C - x0)) * 4u;
         mbar_expect_tx(&full, G::NT * G::TILE + 2u * pbytes);
-        tma_load_3d(smem, &tv, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
-        if (GATE) tma_load_3d(smem + G::TILE, &tr, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
+        tma_load_3d(smem, &tk, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
+        tma_load_3d(smem + G::TILE, &tv, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
+        if (GATE) tma_load_3d(smem + 2 * G::TILE, &tr, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
         bulk_load(prm, A.w + x0, pbytes, &full);
         bulk_load(prm + CB, A.u + x0, pbytes, &full);
     }
     const int64_t t_seg = t_part + warp * LS;
     const int nvalid = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(LS), A.T - t_seg)));
-    Raw kr[LS];
-    {
-        const IO* kp = static_cast<const IO*>(A.k) + (bs * A.T + t_seg) * A.C + c;
-#pragma unroll
-        for (int i = 0; i < LS; ++i) kr[i] = (cvalid && i < nvalid) ? ldg_pair<IO>(kp + i * A.C) : Raw{};
-    }
     __syncthreads();   // the barrier's initialisation is visible to every waiter
     const bool got = mbar_wait(&full, 0u, kCopyWaitNs);
 
-    float w2[V], u2[V], dk[V], eu[V];
+    StreamSeg<LS> sg;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
-        w2[j] = cvalid ? prm[lane * V + j] * kLog2e : 1.f;
-        u2[j] = cvalid ? prm[CB + lane * V + j] * kLog2e : 0.f;
-        dk[j] = ex2(-w2[j]);
-        eu[j] = ex2(u2[j]);
+        sg.w2[j] = cvalid ? prm[lane * V + j] * kLog2e : 1.f;
+        sg.u2[j] = cvalid ? prm[CB + lane * V + j] * kLog2e : 0.f;
+        sg.dk[j] = ex2(-sg.w2[j]);
+        sg.eu[j] = ex2(sg.u2[j]);
     }
-    const unsigned char* vrow = smem + warp * LS * ROW + lane * V * static_cast<int>(sizeof(IO));
-    const F2 L2 = f2s(kLog2e);
+    const unsigned char* krow = smem + warp * LS * ROW + lane * V * static_cast<int>(sizeof(IO));
+    unsigned char* vrow = smem + G::TILE + warp * LS * ROW + lane * V * static_cast<int>(sizeof(IO));
 
-    // ---- pass 0: key range and the segment's running-max exponent q ----
-    // q = max_i (k2_i - (n-1-i) w2), each candidate from one product
-    float kx[V] = {-3.0e38f, -3.0e38f}, kn[V] = {3.0e38f, 3.0e38f}, qm[V] = {-3.0e38f, -3.0e38f};
-#pragma unroll
-    for (int i = 0; i < LS; ++i) {
-        if (i < nvalid) {
-            const F2 kk = raw_pair<IO>(kr[i]);
-            const float o = static_cast<float>(i - (nvalid - 1));
-            const F2 cand = fma2(kk, L2, f2(o * w2[0], o * w2[1]));
-            kx[0] = fmaxf(kx[0], f2lo(kk));
-            kx[1] = fmaxf(kx[1], f2hi(kk));
-            kn[0] = fminf(kn[0], f2lo(kk));
-            kn[1] = fminf(kn[1], f2hi(kk));
-            qm[0] = fmaxf(qm[0], f2lo(cand));
-            qm[1] = fmaxf(qm[1], f2hi(cand));
-        }
-    }
-    float kmax[V], kmin[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-        kmax[j] = kx[j] * kLog2e;
-        kmin[j] = kn[j] * kLog2e;
-    }
-    const bool fast1 = (kmax[0] - kmin[0] + fabsf(u2[0]) <= kFastSpan) &&
-                       (kmax[1] - kmin[1] + fabsf(u2[1]) <= kFastSpan);
-
-    // ---- pass 1: segment summary ----
+    // ---- pass 0/1: the segment's summary ----
     St seg[V];
     if (nvalid == 0 || !got) {
         seg[0] = seg[1] = st_identity();
-    } else if (fast1) {
-        const F2 KM = f2(-kmax[0], -kmax[1]);
-        const F2 DK = f2(dk[0], dk[1]);
-        F2 n = f2s(0.f), db = f2s(0.f);
-#pragma unroll
-        for (int i = 0; i < LS; ++i) {
-            if (i < nvalid) {
-                const F2 ek = ex2x2(fma2(raw_pair<IO>(kr[i]), L2, KM));
-                const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW)));
-                n = fma2(n, DK, ekv);
-                db = fma2(db, DK, ek);
-            }
-        }
-        const float sc0 = ex2(kmax[0] - qm[0]), sc1 = ex2(kmax[1] - qm[1]);
-        seg[0] = St{qm[0], f2lo(n) * sc0, f2lo(db) * sc0};
-        seg[1] = St{qm[1], f2hi(n) * sc1, f2hi(db) * sc1};
+        sg.kmax[0] = sg.kmax[1] = sg.kmin[0] = sg.kmin[1] = 0.f;
+        sg.fast1 = false;
+    } else if (full_part) {
+        stream_pass01<IO, LS, true>(krow, vrow, nvalid, sg, seg);
     } else {
-        // keys too spread for one reference: the exact running-max recurrence
-        // with its exponent held as pb - m w2 (see lane_token_pm)
-        float pb[V], m[V];
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            seg[j] = st_identity();
-            pb[j] = seg[j].p;
-            m[j] = 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < LS; ++i) {
-            if (i < nvalid) {
-                const F2 kk = raw_pair<IO>(kr[i]);
-                const F2 vv = raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW));
-#pragma unroll
-                for (int j = 0; j < V; ++j) {
-                    const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                    const float v1 = j == 0 ? f2lo(vv) : f2hi(vv);
-                    const float pd = fmaf(-(m[j] + 1.f), w2[j], pb[j]);
-                    const float d2 = pd - k2;
-                    const float e = ex2(-fabsf(d2));
-                    if (d2 >= 0.f) {
-                        seg[j].a = fmaf(e, v1, seg[j].a);
-                        seg[j].b += e;
-                        m[j] += 1.f;
-                    } else {
-                        seg[j].a = fmaf(e, seg[j].a, v1);
-                        seg[j].b = fmaf(e, seg[j].b, 1.f);
-                        pb[j] = k2;
-                        m[j] = 0.f;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < V; ++j) seg[j].p = fmaf(-m[j], w2[j], pb[j]);
+        stream_pass01<IO, LS, false>(krow, vrow, nvalid, sg, seg);
     }
 #pragma unroll
     for (int j = 0; j < V; ++j) s_seg[warp][j][lane] = seg[j];
@@ -224,17 +337,17 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_const
     St pre[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) pre[j] = st_identity();
-    for (int sg = 0; sg < warp; ++sg) {
-        const int len = max(0, min(LS, part_len - sg * LS));
+    for (int s = 0; s < warp; ++s) {
+        const int len = max(0, min(LS, part_len - s * LS));
 #pragma unroll
-        for (int j = 0; j < V; ++j) pre[j] = st_combine(pre[j], s_seg[sg][j][lane], static_cast<float>(len) * w2[j]);
+        for (int j = 0; j < V; ++j) pre[j] = st_combine(pre[j], s_seg[s][j][lane], static_cast<float>(len) * sg.w2[j]);
     }
     const int pre_len = min(warp * LS, part_len);
     St agg[V];   // warp W-1: the part's summary
     if (warp == W - 1) {
 #pragma unroll
         for (int j = 0; j < V; ++j) {
-            agg[j] = ok ? st_combine(pre[j], seg[j], static_cast<float>(nvalid) * w2[j]) : St{nan, nan, nan};
+            agg[j] = ok ? st_combine(pre[j], seg[j], static_cast<float>(nvalid) * sg.w2[j]) : St{nan, nan, nan};
             s_slot[j][lane] = make_float4(agg[j].p, agg[j].a, agg[j].b, 0.f);
         }
     }
@@ -249,7 +362,7 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_const
 #pragma unroll
             for (int j = 0; j < V; ++j)
                 xs[j] = st_combine(xs[j], ld_cluster_state(&s_slot[j][lane], static_cast<uint32_t>(r)),
-                                   static_cast<float>(PT) * w2[j]);
+                                   static_cast<float>(PT) * sg.w2[j]);
         }
 #pragma unroll
         for (int j = 0; j < V; ++j) s_x[j][lane] = xs[j];
@@ -258,11 +371,12 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_const
     // summary of every token from the chunk start to this warp's segment
     St z[V];
 #pragma unroll
-    for (int j = 0; j < V; ++j) z[j] = st_combine(s_x[j][lane], pre[j], static_cast<float>(pre_len) * w2[j]);
+    for (int j = 0; j < V; ++j) z[j] = st_combine(s_x[j][lane], pre[j], static_cast<float>(pre_len) * sg.w2[j]);
     St chunk_sum[V];   // the last part's warp W-1: summary of the whole chunk
     if (warp == W - 1 && q == last) {
 #pragma unroll
-        for (int j = 0; j < V; ++j) chunk_sum[j] = st_combine(s_x[j][lane], agg[j], static_cast<float>(part_len) * w2[j]);
+        for (int j = 0; j < V; ++j)
+            chunk_sum[j] = st_combine(s_x[j][lane], agg[j], static_cast<float>(part_len) * sg.w2[j]);
     }
 
     // -------- the entering state from here on --------
@@ -285,7 +399,8 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_const
         if (A.s_out != nullptr && cvalid) {
 #pragma unroll
             for (int j = 0; j < V; ++j) {
-                const St so = ok ? st_combine(sin[j], chunk_sum[j], static_cast<float>(A.T) * w2[j]) : St{nan, nan, nan};
+                const St so = ok ? st_combine(sin[j], chunk_sum[j], static_cast<float>(A.T) * sg.w2[j])
+                                 : St{nan, nan, nan};
                 const int64_t li = bs * A.C + c + j;
                 A.s_out[li] = so.a;
                 A.s_out[lanes + li] = so.b;
@@ -294,89 +409,38 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tv, const __grid_const
         }
     }
 
-    // ---- pass 2: outputs from the segment's start state ----
-    if (ok && nvalid > 0 && cvalid && A.y != nullptr) {
-        St st[V];
+    // ---- pass 2: outputs from the segment's start state, then one store per warp ----
+    if (A.y != nullptr && nvalid > 0) {
+        if (cvalid) {
+            if (ok) {
+                St st[V];
 #pragma unroll
-        for (int j = 0; j < V; ++j) st[j] = st_combine(sin[j], z[j], static_cast<float>(t_seg) * w2[j]);
-        bool fast2 = fast1;
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const bool near = st[j].p >= kmax[j] - kFastState;
-            const bool negligible = st[j].p < kmax[j] - 1.5f * kFastState && st[j].b <= 16777216.f;
-            fast2 = fast2 && (st[j].p - kmin[j] + fabsf(u2[j]) <= kFastState) && (near || negligible);
-        }
-        IO* yp = static_cast<IO*>(A.y) + (bs * A.T + t_seg) * A.C + c;
-        const unsigned char* rrow = vrow + G::TILE;
-        if (fast2) {
-            float nr[V], ss[V];
-#pragma unroll
-            for (int j = 0; j < V; ++j) {
-                const float R = fmaxf(kmax[j], st[j].p);
-                nr[j] = -R;
-                ss[j] = ex2(st[j].p - R);
-            }
-            const F2 NR = f2(nr[0], nr[1]);
-            const F2 EU = f2(eu[0], eu[1]);
-            const F2 DK = f2(dk[0], dk[1]);
-            const F2 NL = f2s(-kLog2e);
-            F2 n = f2(st[0].a * ss[0], st[1].a * ss[1]);
-            F2 db = f2(st[0].b * ss[0], st[1].b * ss[1]);
-#pragma unroll
-            for (int i = 0; i < LS; ++i) {
-                if (i < nvalid) {
-                    const F2 ek = ex2x2(fma2(raw_pair<IO>(kr[i]), L2, NR));
-                    const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW)));
-                    const F2 num = fma2(EU, ekv, n);
-                    F2 den = fma2(EU, ek, db);
-                    if (GATE) {
-                        const F2 g = ex2x2(mul2(raw_pair<IO>(*reinterpret_cast<const Raw*>(rrow + i * ROW)), NL));
-                        den = fma2(den, g, den);
-                    }
-                    const F2 y = mul2(num, rcpx2(den));
-                    n = fma2(n, DK, ekv);
-                    db = fma2(db, DK, ek);
-                    const float out[2] = {f2lo(y), f2hi(y)};
-                    Ld::store(yp + i * A.C, out);
-                }
-            }
-        } else {
-            float pb[V], m[V];
-#pragma unroll
-            for (int j = 0; j < V; ++j) {
-                pb[j] = st[j].p;
-                m[j] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < LS; ++i) {
-                if (i < nvalid) {
-                    const F2 kk = raw_pair<IO>(kr[i]);
-                    const F2 vv = raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW));
-                    F2 rv = f2s(0.f);
-                    if (GATE) rv = raw_pair<IO>(*reinterpret_cast<const Raw*>(rrow + i * ROW));
-                    float out[V];
-#pragma unroll
-                    for (int j = 0; j < V; ++j) {
-                        const float gd = GATE ? gate_den(j == 0 ? f2lo(rv) : f2hi(rv)) : 1.f;
-                        const float k2 = (j == 0 ? f2lo(kk) : f2hi(kk)) * kLog2e;
-                        out[j] = lane_token_pm(st[j].a, st[j].b, pb[j], m[j], w2[j], u2[j], k2,
-                                               j == 0 ? f2lo(vv) : f2hi(vv), gd);
-                    }
-                    Ld::store(yp + i * A.C, out);
-                }
+                for (int j = 0; j < V; ++j) st[j] = st_combine(sin[j], z[j], static_cast<float>(t_seg) * sg.w2[j]);
+                const unsigned char* rrow = vrow + G::TILE;
+                if (full_part) stream_pass2<IO, GATE, LS, true>(krow, vrow, rrow, nvalid, sg, st);
+                else stream_pass2<IO, GATE, LS, false>(krow, vrow, rrow, nvalid, sg, st);
+            } else {
+                // a copy that did not land: NaN outputs, never stale values
+                const float out[2] = {nan, nan};
+                for (int i = 0; i < nvalid; ++i) Vec<IO, V>::store(reinterpret_cast<IO*>(vrow + i * ROW), out);
             }
         }
-    } else if (!ok && nvalid > 0 && cvalid && A.y != nullptr) {
-        // a copy that did not land: NaN outputs, never stale values
-        IO* yp = static_cast<IO*>(A.y) + (bs * A.T + t_seg) * A.C + c;
-        const float out[2] = {nan, nan};
-        for (int i = 0; i < nvalid; ++i) Ld::store(yp + i * A.C, out);
+        // the warp's rows were written through the generic proxy; the TMA
+        // store reads them through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_3d(&ty, smem + G::TILE + warp * LS * ROW, x0, static_cast<int>(t_seg), static_cast<int>(bs));
+            bulk_commit_group();
+        }
     }
     if (!ok && threadIdx.x == 0) {
         if (A.hdr != nullptr) record_timeout(A, q * A.nLB + lb);
         // let the copy land before the CTA's shared memory is released
         mbar_wait(&full, 0u, kCopyWaitNs);
     }
+    // the stores must have read shared memory before the CTA exits
+    if (lane == 0 && A.y != nullptr && nvalid > 0) bulk_wait_group_read0();
     if (!(warp == W - 1 && q == last)) cluster_wait_acquire();
 }
 
