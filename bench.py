@@ -289,9 +289,12 @@ class StreamCase:
     the step.  k, v and y of the whole stream are resident (25.8 GB for the
     1M-token stream), so every chunk reads fresh inputs from HBM.
     inputs_ready passes WKV_FLAG_INPUTS_READY: the chunks' inputs are written
-    before the step and never by the chain itself."""
+    before the step and never by the chain itself.  chain passes the chunk
+    chain flags instead (WKV_FLAG_CHAIN_BEGIN on the first call of the step,
+    WKV_FLAG_CHAIN_NEXT on the others, which imply WKV_FLAG_INPUTS_READY):
+    each call takes the state the previous one publishes in the workspace."""
 
-    def __init__(self, wl, device, seed_base, inputs_ready=True):
+    def __init__(self, wl, device, seed_base, inputs_ready=True, chain=True):
         import dataclasses
         import torch
         from rwkv_wkv_recurrence_02_b200 import inputs as I
@@ -311,6 +314,7 @@ class StreamCase:
         self.fresh = I.fresh_state(self.B, self.C, device=device)
         self.state = self.fresh.clone()
         self.ready = inputs_ready
+        self.chain = chain and inputs_ready
         self.elements = self.B * self.T * self.C
         self.bytes = algorithmic_bytes(wl, self.B, self.chunk, self.C)      # per launch (one chunk)
         self.launches_per_step = self.n
@@ -325,7 +329,8 @@ class StreamCase:
         for j in range(self.n):
             sl = self.chunk_slice(j)
             wkv.wkv_forward(self.w, self.u, self.k[:, sl], self.v[:, sl], None, self.state, y=self.y[:, sl],
-                            state_out=self.state, workspace=ws, inputs_ready=self.ready)
+                            state_out=self.state, workspace=ws, inputs_ready=self.ready,
+                            chain=("begin" if j == 0 else "next") if self.chain else None)
 
 
 class DecodeCase:
@@ -486,7 +491,7 @@ def whole_stream(name) -> bool:
     return name == "stream_1m"
 
 
-def make_case(name, device, seed_base, op="forward", per_layer=False, inputs_ready=True):
+def make_case(name, device, seed_base, op="forward", per_layer=False, inputs_ready=True, chain=True):
     wl = workload(name)
     if op == "wkv5" or hasattr(wl, "H"):
         if not hasattr(wl, "H"):
@@ -501,7 +506,7 @@ def make_case(name, device, seed_base, op="forward", per_layer=False, inputs_rea
     if wl.layers:
         return DecodeCase(wl, device, seed_base, per_layer)
     if whole_stream(name):
-        return StreamCase(wl, device, seed_base, inputs_ready)
+        return StreamCase(wl, device, seed_base, inputs_ready, chain)
     return ForwardCase(wl, device, seed_base)
 
 
@@ -894,6 +899,7 @@ def config_of(case, workload, world):
                     "stream": (f"the whole stream per step: {wl.T // wl.chunk} wkv_forward calls of {wl.chunk} "
                                "tokens, state carried in place from the empty state"),
                     "inputs_ready": bool(getattr(case, "ready", False)),
+                    "chain": bool(getattr(case, "chain", False)),
                     "l2": "inputs of the whole stream resident (25.8 GB), far above the 126 MB L2"})
     elif getattr(wl, "chunk", 0):
         cfg["stream"] = f"one chunk of {wl.chunk} tokens per step, state carried in place"
@@ -926,7 +932,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     wkv.lib()
     case = make_case(args.workload, device, rank_seed(0, rank), args.op, args.decode_per_layer,
-                     not args.no_inputs_ready)
+                     not args.no_inputs_ready, not args.no_chain)
     ws = wkv.Workspace(device)
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
@@ -955,11 +961,15 @@ def run_ours(args):
     clocks.sample_now()
     t0 = time.time()
     e0.record(stream)
+    # an NVTX range around the timed launches, so a profiler's launch list can
+    # be restricted to them (ncu --nvtx --nvtx-include bench_timed/)
+    torch.cuda.nvtx.range_push("bench_timed")
     for i in range(args.steps):
         if graphs is not None:
             graphs[i % len(graphs)].replay()
         else:
             case.step(args.warmup + i, wkv, ws)
+    torch.cuda.nvtx.range_pop()
     e1.record(stream)
     clocks.sample_now()
     torch.cuda.synchronize()
@@ -1133,15 +1143,23 @@ def run_reference_shift(args, wl):
     print(json.dumps(out), flush=True)
 
 
+# the workload each operation is measured on unless --workload names another
+DEFAULT_WORKLOAD = {"forward": "stream_1m", "backward": "layer_1b5", "token_shift": "layer_14b", "wkv5": "v5_layer"}
+
+
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=None,
                    help="timed steps (default: 20 for the whole stream, 3000 for the other workloads)")
     p.add_argument("--warmup", type=int, default=None, help="warm-up steps (default: 5 / 20)")
-    p.add_argument("--workload", default="stream_1m", choices=WORKLOAD_NAMES)
+    p.add_argument("--workload", default=None, choices=WORKLOAD_NAMES,
+                   help="default per --op: " + ", ".join(f"{k}: {v}" for k, v in DEFAULT_WORKLOAD.items()))
     p.add_argument("--no-graph", action="store_true",
                    help="the whole stream: launch the chunk calls instead of replaying a CUDA graph")
+    p.add_argument("--no-chain", action="store_true",
+                   help="the whole stream: plain calls (state read after the previous kernel ends) instead of a "
+                        "chunk chain")
     p.add_argument("--no-inputs-ready", action="store_true",
                    help="the whole stream: do not pass WKV_FLAG_INPUTS_READY")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -1157,6 +1175,10 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     a = p.parse_args(argv)
+    if a.workload is None:
+        a.workload = DEFAULT_WORKLOAD[a.op]
+    if a.op in ("backward", "token_shift") and whole_stream(a.workload):
+        p.error(f"--op {a.op} takes a single-call workload, not the whole stream {a.workload}")
     if a.steps is None:
         a.steps = 20 if whole_stream(a.workload) and a.op == "forward" else 3000
     if a.warmup is None:

@@ -144,6 +144,38 @@ int wkv_forward(int64_t B, int64_t T, int64_t C, int dtype,
  *       an input is still being written gives wrong results.
  */
 #define WKV_FLAG_INPUTS_READY 1u
+/*
+ *   WKV_FLAG_CHAIN_BEGIN, WKV_FLAG_CHAIN_NEXT  (each implies
+ *       WKV_FLAG_INPUTS_READY; setting both is WKV_ERR_SHAPE) a chain of
+ *       chunk calls on `stream` that carry one state: the first call passes
+ *       WKV_FLAG_CHAIN_BEGIN and reads state_in after the previous kernel of
+ *       the stream ends, as with WKV_FLAG_INPUTS_READY.  Every later call
+ *       passes WKV_FLAG_CHAIN_NEXT, declaring that its state_in is the
+ *       state_out of the previous call of the chain, that nothing has
+ *       written it since, and that that call was given the same workspace,
+ *       B, C and dtype.  When the stream kernel runs and the workspace holds
+ *       at least 256 + 16 * B * C bytes (every workspace of
+ *       wkv_forward_workspace_bytes() for T > 64 does), each call publishes
+ *       the state it leaves in the workspace as soon as that state is formed,
+ *       before its outputs (one 16-byte word per channel, tagged with the
+ *       call's position in the chain), and a WKV_FLAG_CHAIN_NEXT call waits
+ *       for that word instead of for the end of the previous kernel.  Each
+ *       call still writes state_out, and its kernel does not finish before
+ *       the previous one has.  The first call clears the words (one
+ *       cudaMemsetAsync of 16 * B * C bytes before its kernel).
+ *       The workspace belongs to the chain until the chain ends: any other
+ *       call on it ends the chain, and a WKV_FLAG_CHAIN_NEXT call with no
+ *       matching predecessor (other workspace, sizes, or a state_in that is
+ *       not the previous state_out) reads state_in as a first call does.
+ *       With either flag, y may be written before the previous kernel of the
+ *       stream ends: it must not be the previous call's y.  A wait for the
+ *       previous word that exceeds the wait limit records WKV_ERR_TIMEOUT in
+ *       the workspace (wkv_workspace_status) and makes the state and outputs
+ *       NaN.  A false declaration gives wrong results or a timeout, never a
+ *       hang.
+ */
+#define WKV_FLAG_CHAIN_BEGIN 2u
+#define WKV_FLAG_CHAIN_NEXT 4u
 
 int wkv_forward_ex(int64_t B, int64_t T, int64_t C, int dtype,
                    const float* w, const float* u,

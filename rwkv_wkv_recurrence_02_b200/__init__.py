@@ -208,17 +208,23 @@ def workspace_bytes(B: int, T: int, C: int, dtype_code: int) -> int:
 
 
 WKV_FLAG_INPUTS_READY = 1
+WKV_FLAG_CHAIN_BEGIN = 2
+WKV_FLAG_CHAIN_NEXT = 4
 
 
 def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, want_state=True,
-                workspace: Workspace = None, use_workspace=True, inputs_ready=False, stream=None):
+                workspace: Workspace = None, use_workspace=True, inputs_ready=False, chain=None, stream=None):
     """Parallel mode over one chunk.  k, v, r: (B, T, C) CUDA tensors (float32
     or bfloat16); w, u: (C,) float32; state_in: (3, B, C) float32 or None.
     Returns (y, state_out) (state_out None if want_state is False and none
     was given).  state_out may be state_in for an in-place update.
     use_workspace=False passes no workspace (the scratch-free schedules).
     inputs_ready=True passes WKV_FLAG_INPUTS_READY: k, v, r, w, u are not
-    written by work still running on the stream (see include/wkv.h)."""
+    written by work still running on the stream (see include/wkv.h).
+    chain="begin" / "next" passes WKV_FLAG_CHAIN_BEGIN / WKV_FLAG_CHAIN_NEXT
+    (a chain of chunk calls carrying one state through the workspace; see
+    include/wkv.h): the first call of a chain passes "begin", every later
+    one "next" with the previous call's state_out as its state_in."""
     torch = _torch()
     if k.dim() != 3:
         raise ValueError("k must be (B, T, C)")
@@ -242,12 +248,20 @@ def wkv_forward(w, u, k, v, r=None, state_in=None, *, y=None, state_out=None, wa
     sp = _stream_ptr(stream, dev)
     if use_workspace:
         ws = workspace if workspace is not None else default_workspace(dev)
-        ws_ptr, ws_bytes = ws.get(workspace_bytes(B, T, C, code), stream)
+        need = workspace_bytes(B, T, C, code)
+        if chain is not None:
+            need = max(need, 256 + 16 * B * C)   # the chain's words follow the header
+        ws_ptr, ws_bytes = ws.get(need, stream)
     else:
         ws_ptr, ws_bytes = None, 0
-    if inputs_ready:
+    flags = WKV_FLAG_INPUTS_READY if inputs_ready else 0
+    if chain is not None:
+        if chain not in ("begin", "next"):
+            raise ValueError("chain must be None, 'begin' or 'next'")
+        flags |= WKV_FLAG_CHAIN_BEGIN if chain == "begin" else WKV_FLAG_CHAIN_NEXT
+    if flags:
         _check(lib().wkv_forward_ex(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),
-                                    _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, WKV_FLAG_INPUTS_READY, sp),
+                                    _ptr(y), _ptr(state_out), ws_ptr, ws_bytes, flags, sp),
                "wkv_forward_ex")
     else:
         _check(lib().wkv_forward(B, T, C, code, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(state_in),

@@ -39,8 +39,25 @@ int g_sm_count[kMaxDevices] = {0};
 constexpr int kW = 8;
 constexpr int kLS = 8;
 constexpr int kMinTT = kW * kLS;
-// Lane-resident kernel: compute warps and tokens per warp segment (64-token
-// chunks).
+// Lane-resident kernel: compute warps, tokens per warp segment, ring depth
+// and CTAs per SM of the forward, per I/O type.  bf16 tiles are half as
+// large, so its CTAs carry more compute warps in the same shared memory,
+// which is what hides the recurrence's latency.
+template <typename IO>
+struct LaneCfg {
+    static constexpr int W = 4, LS = 16, S = 3, MINB = 2;
+};
+template <>
+struct LaneCfg<float> {
+    static constexpr int W = 4, LS = 16, S = 2, MINB = 2;
+};
+// tokens per chunk of the lane-resident forward
+inline int lane_tt(int dtype) {
+    return dtype == WKV_F32 ? LaneCfg<float>::W * LaneCfg<float>::LS
+                            : LaneCfg<__nv_bfloat16>::W * LaneCfg<__nv_bfloat16>::LS;
+}
+// The checkpoint sweep of the backward: 64-token chunks, the chunks the
+// reverse walk takes.
 constexpr int kLaneW = 4;
 constexpr int kLaneLS = 16;
 // Part kernel: compute warps and tokens per warp segment (64-token parts),
@@ -138,6 +155,57 @@ ChunkGeom chunk_geom(int64_t B, int64_t T, int64_t C, int V, int TT) {
 }
 
 bool use_sequential(int64_t T) { return T <= kSeqMaxT; }
+
+// Chunk chains (WKV_FLAG_CHAIN_BEGIN / WKV_FLAG_CHAIN_NEXT): per workspace,
+// the call that published last, so that the next call of the chain knows
+// which position's word to wait for.  A call without a matching record
+// starts a new chain.
+struct ChainRec {
+    const void* ws = nullptr;
+    const float* state = nullptr;   // that call's state_out
+    int64_t B = 0, C = 0;
+    int dtype = -1;
+    uint32_t next = 0;              // position tag of the words it published
+};
+constexpr int kChainSlots = 32;
+std::mutex g_chain_mutex;
+ChainRec g_chain[kChainSlots];
+int g_chain_evict = 0;
+
+// Any call that uses a workspace outside a chain ends the workspace's chain.
+void chain_forget(const void* ws) {
+    if (ws == nullptr) return;
+    std::lock_guard<std::mutex> lock(g_chain_mutex);
+    for (ChainRec& r : g_chain)
+        if (r.ws == ws) r = ChainRec{};
+}
+
+// Position whose words hold this call's entering state (0: none, the call
+// reads state_in), and the record of this call for the next one.
+uint32_t chain_enter(const void* ws, bool next, const float* state_in, const float* state_out, int64_t B, int64_t C,
+                     int dtype) {
+    std::lock_guard<std::mutex> lock(g_chain_mutex);
+    ChainRec* rec = nullptr;
+    for (ChainRec& r : g_chain)
+        if (r.ws == ws) rec = &r;
+    uint32_t in = 0;
+    if (rec != nullptr && next && state_in != nullptr && rec->state == state_in && rec->B == B && rec->C == C &&
+        rec->dtype == dtype)
+        in = rec->next;
+    if (rec == nullptr) {
+        for (ChainRec& r : g_chain)
+            if (r.ws == nullptr && rec == nullptr) rec = &r;
+    }
+    if (rec == nullptr) {
+        // every slot in use: end the oldest-placed chain (its next call starts over)
+        rec = &g_chain[g_chain_evict];
+        g_chain_evict = (g_chain_evict + 1) % kChainSlots;
+    }
+    // the position counter stays clear of 0, which marks no chain
+    const uint32_t out = (in + 1u) & 0x3fffffffu;
+    *rec = ChainRec{ws, state_out, B, C, dtype, out == 0u ? 1u : out};
+    return in;
+}
 
 int forced_kernel();
 
@@ -281,10 +349,10 @@ int launch_pdl(void (*kern)(P...), int64_t grid, int threads, uint32_t smem, cud
 
 // Lane-resident kernel: each CTA owns whole lane blocks; grid = min(lane
 // blocks, resident capacity).
-template <typename IO, bool GATE, int STAGES, bool CKPT = false>
+template <typename IO, bool GATE, int W, int LS, int STAGES, int MINB, bool CKPT = false>
 int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
-    using G = wkv::LaneGeometry<IO, 2, GATE, kLaneW, kLaneLS, STAGES>;
-    auto kern = wkv::lane_forward_kernel<IO, 2, GATE, kLaneW, kLaneLS, STAGES, 2, CKPT>;
+    using G = wkv::LaneGeometry<IO, 2, GATE, W, LS, STAGES>;
+    auto kern = wkv::lane_forward_kernel<IO, 2, GATE, W, LS, STAGES, MINB, CKPT>;
     static int capacity[kMaxDevices] = {0};
     int dev = 0;
     int rc = record_cuda(cudaGetDevice(&dev));
@@ -523,10 +591,9 @@ int dispatch_part(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_
 
 template <typename IO>
 int dispatch_lane(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
-    // ring depth: two CTAs per SM for either dtype
-    constexpr int S = sizeof(IO) == 4 ? 2 : 3;
-    return gate ? launch_lane<IO, true, S>(a, dtype, ws, ws_bytes, st)
-                : launch_lane<IO, false, S>(a, dtype, ws, ws_bytes, st);
+    using L = LaneCfg<IO>;
+    return gate ? launch_lane<IO, true, L::W, L::LS, L::S, L::MINB>(a, dtype, ws, ws_bytes, st)
+                : launch_lane<IO, false, L::W, L::LS, L::S, L::MINB>(a, dtype, ws, ws_bytes, st);
 }
 
 template <typename IO, int V>
@@ -657,6 +724,7 @@ size_t wkv_forward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype) {
 }
 
 int wkv_workspace_init(void* workspace, size_t bytes, cudaStream_t stream) {
+    chain_forget(workspace);
     if (bytes == 0) return WKV_OK;
     if (workspace == nullptr) return WKV_ERR_NULLPTR;
     if (!aligned(workspace, 256)) return WKV_ERR_ALIGN;
@@ -686,7 +754,9 @@ int wkv_forward_ex(int64_t B, int64_t T, int64_t C, int dtype, const float* w, c
                    float* state_out, void* workspace, size_t workspace_bytes, unsigned flags,
                    cudaStream_t stream) {
     if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
-    if ((flags & ~unsigned(WKV_FLAG_INPUTS_READY)) != 0) return WKV_ERR_SHAPE;
+    if ((flags & ~unsigned(WKV_FLAG_INPUTS_READY | WKV_FLAG_CHAIN_BEGIN | WKV_FLAG_CHAIN_NEXT)) != 0 ||
+        (flags & WKV_FLAG_CHAIN_BEGIN && flags & WKV_FLAG_CHAIN_NEXT))
+        return WKV_ERR_SHAPE;
     int64_t n = 0;
     if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;
     if (B == 0 || C == 0) return WKV_OK;
@@ -722,6 +792,7 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     const int V = pick_vec(C, dtype, io, 4, f32, 4);
     const int force = forced_kernel();
     const bool seq = force == 1 || (force == 0 && use_sequential(T));
+    if (seq) chain_forget(workspace);
 
     wkv::ChunkArgs a{};
     a.w = w;
@@ -736,7 +807,9 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
     a.T = T;
     a.C = C;
     a.wait_limit_ns = wait_limit_ns();
-    a.early = (flags & WKV_FLAG_INPUTS_READY) ? 1u : 0u;
+    a.early = (flags & (WKV_FLAG_INPUTS_READY | WKV_FLAG_CHAIN_BEGIN | WKV_FLAG_CHAIN_NEXT)) ? 1u : 0u;
+    a.chain = nullptr;
+    a.chain_in = 0u;
     int64_t grid = 0;
     if (!seq) {
         const bool tma = force != 2 && tma_eligible(V, dtype, B, T, C, k, v, r, w, u, state_in);
@@ -761,10 +834,33 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
         const bool stream_ok = part_ok && (y == nullptr || aligned(y, 16)) &&
                                (state_out == nullptr || aligned(state_out, 8)) && (T + spt - 1) / spt <= kStreamMax;
         if (stream_ok && (force == 8 || (force == 0 && nLB < sm_count()))) {
-            return dtype == WKV_F32
-                       ? dispatch_stream<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
-                       : dispatch_stream<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
+            // a chunk chain publishes each call's end state at the start of
+            // the workspace, right after its header
+            const size_t chain_bytes = size_t(B) * size_t(C) * sizeof(wkv::Word);
+            if ((flags & (WKV_FLAG_CHAIN_BEGIN | WKV_FLAG_CHAIN_NEXT)) && workspace != nullptr &&
+                aligned(workspace, 256) && workspace_bytes >= 256 + chain_bytes) {
+                a.chain = reinterpret_cast<wkv::Word*>(static_cast<char*>(workspace) + 256);
+                a.chain_in = chain_enter(workspace, (flags & WKV_FLAG_CHAIN_NEXT) != 0, state_in, state_out, B, C,
+                                         dtype);
+                if (a.chain_in == 0u) {
+                    // a new chain: no word of an earlier one may look current
+                    const int rc = record_cuda(cudaMemsetAsync(a.chain, 0, chain_bytes, stream));
+                    if (rc != WKV_OK) {
+                        chain_forget(workspace);
+                        return rc;
+                    }
+                }
+            } else {
+                chain_forget(workspace);
+            }
+            const int rc = dtype == WKV_F32
+                               ? dispatch_stream<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
+                               : dispatch_stream<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes,
+                                                                stream);
+            if (rc != WKV_OK) chain_forget(workspace);
+            return rc;
         }
+        chain_forget(workspace);
         if (cluster_ok && (force == 7 || (force == 0 && !ws_ok))) {
             return dtype == WKV_F32
                        ? dispatch_cluster<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
@@ -786,7 +882,7 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
                 }
                 return check_launch();
             }
-            const ChunkGeom g = chunk_geom(B, T, C, 2, kLaneW * kLaneLS);
+            const ChunkGeom g = chunk_geom(B, T, C, 2, lane_tt(dtype));
             a.nCB = g.nCB;
             a.nLB = g.nLB;
             a.nchunks = g.nchunks;
@@ -802,7 +898,7 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
                        : dispatch_part<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes, stream);
         }
         if (tma) {
-            const ChunkGeom g = chunk_geom(B, T, C, 2, kLaneW * kLaneLS);
+            const ChunkGeom g = chunk_geom(B, T, C, 2, lane_tt(dtype));
             a.nCB = g.nCB;
             a.nLB = g.nLB;
             a.nchunks = g.nchunks;
@@ -1156,7 +1252,7 @@ template <typename IO>
 int run_backward(const wkv::BwdArgs& b, wkv::ChunkArgs f, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
     // checkpoint sweep (ring depth as in the forward), then the reverse walk
     constexpr int SF = sizeof(IO) == 4 ? 2 : 3;
-    int rc = launch_lane<IO, false, SF, true>(f, dtype, ws, ws_bytes, st);
+    int rc = launch_lane<IO, false, kLaneW, kLaneLS, SF, 2, true>(f, dtype, ws, ws_bytes, st);
     if (rc != WKV_OK) return rc;
     rc = record_cuda(cudaMemsetAsync(b.part, 0, 2 * size_t(b.nLB) * 64 * sizeof(float), st));
     if (rc != WKV_OK) return rc;
@@ -1184,6 +1280,7 @@ int wkv_backward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, con
                  const void* k, const void* v, const void* r, const float* state_in, const void* dy,
                  const float* dstate_out, void* dk, void* dv, void* dr, float* dw, float* du, float* dstate_in,
                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    chain_forget(workspace);
     if (dtype != WKV_F32 && dtype != WKV_BF16) return WKV_ERR_DTYPE;
     int64_t n = 0;
     if (!mul_ok(B, T, C, &n)) return WKV_ERR_SHAPE;

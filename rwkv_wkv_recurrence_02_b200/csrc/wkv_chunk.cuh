@@ -44,6 +44,7 @@ namespace wkv {
 
 constexpr uint32_t kKindAgg = 1;  // chunk summary (from the empty state)
 constexpr uint32_t kKindInc = 2;  // inclusive state (state after the chunk)
+constexpr uint32_t kKindChain = 3; // state a call of a chunk chain leaves (epoch: position in the chain)
 constexpr uint32_t kErrTimeout = 1;
 // Limit of a wait for this CTA's own TMA copies to land.  Unlike the waits on
 // other CTAs it does not follow the configurable limit: a CTA must not exit
@@ -91,6 +92,11 @@ struct ChunkArgs {
                         // entering each chunk, the last one the state after the sequence
     uint64_t wait_limit_ns;
     uint32_t early;     // stream kernel: inputs may be read before the previous kernel of the stream ends
+    // stream kernel, chunk chains: [B * C] words the state after the call is
+    // published to (null: none), and the position in the chain whose word
+    // holds the entering state (0: the chain's first call reads s_in)
+    Word* chain;
+    uint32_t chain_in;
 };
 
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {

@@ -41,11 +41,28 @@
 // Otherwise the kernel waits at entry like the others.  No workspace, no wait
 // on another cluster; every thread reaches both cluster barriers on every
 // path (a copy that does not land turns into NaN outputs).
+//
+// Chunk chains (A.chain set): the last part's warp W-1 publishes the state
+// after the chunk as tagged words (tag = the next call's position in the
+// chain) right after writing state_out, before pass 2.  A call that
+// continues a chain (A.chain_in > 0) does not wait for the previous kernel
+// to end: one warp per CTA polls for the words tagged with its position
+// (bounded in time), and the kernel waits for the previous one only before
+// it exits, so the stream's kernels still end in order.  Its outputs then
+// overlap the previous call's outputs, and the chain's serial part is only
+// the fold of the entering state.  Programmatic launch starts a kernel only
+// once every CTA of the previous one has started, so the CTAs a call waits
+// on are resident and the wait ends.
 #pragma once
 
 #include "wkv_cluster.cuh"
 
 namespace wkv {
+
+// unroll depth of the per-token loops: deep enough to overlap the shared
+// memory loads and MUFU latencies, shallow enough that the code of the three
+// passes stays resident in the instruction cache
+constexpr int kStreamUnroll = 16;
 
 template <typename IO, bool GATE, int W, int LS>
 struct StreamGeometry {
@@ -94,18 +111,18 @@ __device__ __forceinline__ void stream_pass01(const unsigned char* krow, const u
     const int n = FULL ? LS : nvalid;
     // ---- pass 0: q = max_i (k2_i - (n-1-i) w2), each candidate from one product ----
     float kx[2] = {-3.0e38f, -3.0e38f}, kn[2] = {3.0e38f, 3.0e38f}, qm[2] = {-3.0e38f, -3.0e38f};
-#pragma unroll
-    for (int i = 0; i < LS; ++i) {
-        if (FULL || i < nvalid) {
-            const F2 kk = raw_pair<IO>(kr(i));
-            const F2 cand = fma2(kk, L2, mul2(f2s(static_cast<float>(i - (n - 1))), W2));
-            kx[0] = fmaxf(kx[0], f2lo(kk));
-            kx[1] = fmaxf(kx[1], f2hi(kk));
-            kn[0] = fminf(kn[0], f2lo(kk));
-            kn[1] = fminf(kn[1], f2hi(kk));
-            qm[0] = fmaxf(qm[0], f2lo(cand));
-            qm[1] = fmaxf(qm[1], f2hi(cand));
-        }
+    float back = static_cast<float>(1 - n);   // i - (n-1), exact in float
+#pragma unroll kStreamUnroll
+    for (int i = 0; i < n; ++i) {
+        const F2 kk = raw_pair<IO>(kr(i));
+        const F2 cand = fma2(kk, L2, mul2(f2s(back), W2));
+        back += 1.f;
+        kx[0] = fmaxf(kx[0], f2lo(kk));
+        kx[1] = fmaxf(kx[1], f2hi(kk));
+        kn[0] = fminf(kn[0], f2lo(kk));
+        kn[1] = fminf(kn[1], f2hi(kk));
+        qm[0] = fmaxf(qm[0], f2lo(cand));
+        qm[1] = fmaxf(qm[1], f2hi(cand));
     }
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -119,14 +136,12 @@ __device__ __forceinline__ void stream_pass01(const unsigned char* krow, const u
         const F2 KM = f2(-sg.kmax[0], -sg.kmax[1]);
         const F2 DK = f2(sg.dk[0], sg.dk[1]);
         F2 nn = f2s(0.f), db = f2s(0.f);
-#pragma unroll
-        for (int i = 0; i < LS; ++i) {
-            if (FULL || i < nvalid) {
-                const F2 ek = ex2x2(fma2(raw_pair<IO>(kr(i)), L2, KM));
-                const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW)));
-                nn = fma2(nn, DK, ekv);
-                db = fma2(db, DK, ek);
-            }
+#pragma unroll kStreamUnroll
+        for (int i = 0; i < n; ++i) {
+            const F2 ek = ex2x2(fma2(raw_pair<IO>(kr(i)), L2, KM));
+            const F2 ekv = mul2(ek, raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW)));
+            nn = fma2(nn, DK, ekv);
+            db = fma2(db, DK, ek);
         }
         const float sc0 = ex2(sg.kmax[0] - qm[0]), sc1 = ex2(sg.kmax[1] - qm[1]);
         seg[0] = St{qm[0], f2lo(nn) * sc0, f2lo(db) * sc0};
@@ -141,9 +156,9 @@ __device__ __forceinline__ void stream_pass01(const unsigned char* krow, const u
             pb[j] = seg[j].p;
             m[j] = 0.f;
         }
-#pragma unroll
-        for (int i = 0; i < LS; ++i) {
-            if (FULL || i < nvalid) {
+#pragma unroll 1
+        for (int i = 0; i < n; ++i) {
+            {
                 const F2 kk = raw_pair<IO>(kr(i));
                 const F2 vv = raw_pair<IO>(*reinterpret_cast<const Raw*>(vrow + i * ROW));
 #pragma unroll
@@ -181,6 +196,7 @@ __device__ __forceinline__ void stream_pass2(const unsigned char* krow, unsigned
     constexpr int ROW = 64 * static_cast<int>(sizeof(IO));
     auto kr = [&](int i) { return *reinterpret_cast<const Raw*>(krow + i * ROW); };
     const F2 L2 = f2s(kLog2e);
+    const int cnt = FULL ? LS : nvalid;
     bool fast2 = sg.fast1;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -202,9 +218,9 @@ __device__ __forceinline__ void stream_pass2(const unsigned char* krow, unsigned
         const F2 NL = f2s(-kLog2e);
         F2 n = f2(st[0].a * ss[0], st[1].a * ss[1]);
         F2 db = f2(st[0].b * ss[0], st[1].b * ss[1]);
-#pragma unroll
-        for (int i = 0; i < LS; ++i) {
-            if (FULL || i < nvalid) {
+#pragma unroll kStreamUnroll
+        for (int i = 0; i < cnt; ++i) {
+            {
                 Raw* vp = reinterpret_cast<Raw*>(vrow + i * ROW);
                 const F2 ek = ex2x2(fma2(raw_pair<IO>(kr(i)), L2, NR));
                 const F2 ekv = mul2(ek, raw_pair<IO>(*vp));
@@ -228,9 +244,9 @@ __device__ __forceinline__ void stream_pass2(const unsigned char* krow, unsigned
             pb[j] = st[j].p;
             m[j] = 0.f;
         }
-#pragma unroll
-        for (int i = 0; i < LS; ++i) {
-            if (FULL || i < nvalid) {
+#pragma unroll 1
+        for (int i = 0; i < cnt; ++i) {
+            {
                 Raw* vp = reinterpret_cast<Raw*>(vrow + i * ROW);
                 const F2 kk = raw_pair<IO>(kr(i));
                 const F2 vv = raw_pair<IO>(*vp);
@@ -250,6 +266,43 @@ __device__ __forceinline__ void stream_pass2(const unsigned char* krow, unsigned
     }
 }
 
+// Entering state of a chained call: the words the previous call of the chain
+// published for this lane's channels, tagged with this call's position.
+// Polled by one warp with a time bound; on expiry NaN and a recorded error.
+__device__ __forceinline__ void chain_take(const ChunkArgs& A, int64_t li, bool cvalid, St* out) {
+    const uint32_t want = word_tag(A.chain_in, kKindChain);
+    const Word* src = A.chain + li;
+    const uint64_t t0 = global_ns();
+    unsigned sleep_ns = 32;
+    for (;;) {
+        Word wv[2];
+        bool mine = true;
+        if (cvalid) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                wv[j] = ld_word(src + j);
+                mine = mine && wv[j].tag == want;
+            }
+        }
+        if (__all_sync(0xffffffffu, mine)) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) out[j] = cvalid ? word_state(wv[j]) : st_identity();
+            break;
+        }
+        if (global_ns() - t0 > A.wait_limit_ns) {
+            if ((threadIdx.x & 31) == 0 && A.hdr != nullptr) record_timeout(A, -2);
+            const float nan = __int_as_float(0x7fc00000);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) out[j] = St{nan, nan, nan};
+            break;
+        }
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 256) sleep_ns <<= 1;
+    }
+    // the words were read before this CTA's later writes (state_out)
+    __threadfence();
+}
+
 template <typename IO, bool GATE, int W, int LS, int MINB>
 __global__ void __launch_bounds__(W * 32, MINB)
 stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -266,6 +319,7 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
     __shared__ St s_seg[W][V][32];                   // segment summaries of the part
     __shared__ __align__(16) float4 s_slot[V][32];   // the part's summary, read by later parts
     __shared__ St s_x[V][32];                        // summary of the chunk before this part
+    __shared__ St s_in_chain[V][32];                 // entering state of a chained call
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t q = cluster_ctarank();             // part index along T
     const int64_t last = static_cast<int64_t>(cluster_nctarank()) - 1;
@@ -275,6 +329,7 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
     const int64_t c = x0 + lane * V;
     const bool cvalid = c < A.C;                     // C is even: both channels or neither
     const bool early = A.early != 0;
+    const bool chained = A.chain != nullptr && A.chain_in != 0u;
     const float nan = __int_as_float(0x7fc00000);
 
     if (threadIdx.x == 0) {
@@ -380,15 +435,28 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
     }
 
     // -------- the entering state from here on --------
-    if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t lanes = A.B * A.C;
     St sin[V];
+    if (chained) {
+        // the previous call of the chain published it; no wait for its end
+        if (warp == 0) {
+            St x[V];
+            chain_take(A, bs * A.C + c, cvalid, x);
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-        sin[j] = st_identity();
-        if (A.s_in != nullptr && cvalid) {
-            const int64_t li = bs * A.C + c + j;
-            sin[j] = St{A.s_in[2 * lanes + li] * kLog2e, A.s_in[li], A.s_in[lanes + li]};
+            for (int j = 0; j < V; ++j) s_in_chain[j][lane] = x[j];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < V; ++j) sin[j] = s_in_chain[j][lane];
+    } else {
+        if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            sin[j] = st_identity();
+            if (A.s_in != nullptr && cvalid) {
+                const int64_t li = bs * A.C + c + j;
+                sin[j] = St{A.s_in[2 * lanes + li] * kLog2e, A.s_in[li], A.s_in[lanes + li]};
+            }
         }
     }
     // every CTA has read state_in (and its remote reads are done) once all
@@ -396,15 +464,27 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
     cluster_arrive_release();
     if (warp == W - 1 && q == last) {
         cluster_wait_acquire();
+        St so[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j)
+            so[j] = ok ? st_combine(sin[j], chunk_sum[j], static_cast<float>(A.T) * sg.w2[j]) : St{nan, nan, nan};
         if (A.s_out != nullptr && cvalid) {
 #pragma unroll
             for (int j = 0; j < V; ++j) {
-                const St so = ok ? st_combine(sin[j], chunk_sum[j], static_cast<float>(A.T) * sg.w2[j])
-                                 : St{nan, nan, nan};
                 const int64_t li = bs * A.C + c + j;
-                A.s_out[li] = so.a;
-                A.s_out[lanes + li] = so.b;
-                A.s_out[2 * lanes + li] = so.p * kLn2;
+                A.s_out[li] = so[j].a;
+                A.s_out[lanes + li] = so[j].b;
+                A.s_out[2 * lanes + li] = so[j].p * kLn2;
+            }
+        }
+        if (A.chain != nullptr) {
+            // state_out before the word: the next call writes state_out only
+            // after it has read the word
+            __threadfence();
+            if (cvalid) {
+#pragma unroll
+                for (int j = 0; j < V; ++j)
+                    st_word(A.chain + bs * A.C + c + j, so[j], word_tag(A.chain_in + 1u, kKindChain));
             }
         }
     }
@@ -442,6 +522,9 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
     // the stores must have read shared memory before the CTA exits
     if (lane == 0 && A.y != nullptr && nvalid > 0) bulk_wait_group_read0();
     if (!(warp == W - 1 && q == last)) cluster_wait_acquire();
+    // a chained call has not waited for the previous kernel: it ends after
+    // it, so the stream's kernels still finish in order
+    if (chained) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace wkv

@@ -70,6 +70,19 @@ def test_forward_rejects_bad_dtype_and_shapes(L):
     assert fwd(L, B=1 << 21, T=1 << 21, C=1 << 21) == SHAPE
 
 
+def test_forward_ex_flag_validation(L):
+    def ex(flags, **kw):
+        return L.wkv_forward_ex(2, 100, 64, F32, BASE, BASE + 4096, BASE + (1 << 30), BASE + (2 << 30), None, None,
+                                BASE + (3 << 30), None, None, 0, flags, None)
+    assert ex(8) == SHAPE                          # an unknown bit
+    assert ex(wkv.WKV_FLAG_CHAIN_BEGIN | wkv.WKV_FLAG_CHAIN_NEXT) == SHAPE
+    assert ex(0x80000000) == SHAPE
+    # a valid flag reaches the argument checks (a null k is reported, nothing launches)
+    for f in (wkv.WKV_FLAG_INPUTS_READY, wkv.WKV_FLAG_CHAIN_BEGIN, wkv.WKV_FLAG_CHAIN_NEXT):
+        assert L.wkv_forward_ex(2, 100, 64, F32, BASE, BASE + 4096, None, BASE + (2 << 30), None, None,
+                                BASE + (3 << 30), None, None, 0, f, None) == NULLPTR
+
+
 def test_forward_empty_is_a_noop(L):
     assert fwd(L, B=0) == OK
     assert fwd(L, C=0) == OK

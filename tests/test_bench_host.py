@@ -224,6 +224,12 @@ def test_defaults_follow_the_workload():
     assert b.steps == 3000 and b.warmup == 20
     c = bench.parse_args(["--gpus", "1", "--steps", "20", "--warmup", "5"])
     assert (c.steps, c.warmup, c.workload) == (20, 5, "stream_1m")
+    # the other operations default to their own single-call workloads
+    assert bench.parse_args(["--op", "backward"]).workload == "layer_1b5"
+    assert bench.parse_args(["--op", "token_shift"]).workload == "layer_14b"
+    assert bench.parse_args(["--op", "wkv5"]).workload == "v5_layer"
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--op", "backward", "--workload", "stream_1m"])
 
 
 def test_whole_stream_bytes_and_names():
