@@ -47,8 +47,8 @@
 // chain) right after writing state_out, before pass 2.  A call that
 // continues a chain (A.chain_in > 0) does not wait for the previous kernel
 // to end: one warp per CTA polls for the words tagged with its position
-// (bounded in time), and the kernel waits for the previous one only before
-// it exits, so the stream's kernels still end in order.  Its outputs then
+// (bounded in time), and one CTA waits for the previous kernel before it
+// exits, so the stream's kernels still end in order.  Its outputs then
 // overlap the previous call's outputs, and the chain's serial part is only
 // the fold of the entering state.  Programmatic launch starts a kernel only
 // once every CTA of the previous one has started, so the CTAs a call waits
@@ -299,8 +299,9 @@ __device__ __forceinline__ void chain_take(const ChunkArgs& A, int64_t li, bool 
         __nanosleep(sleep_ns);
         if (sleep_ns < 256) sleep_ns <<= 1;
     }
-    // the words were read before this CTA's later writes (state_out)
-    __threadfence();
+    // acquire: the previous call's state_out write is ordered before this
+    // call's (the word was published after it)
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 template <typename IO, bool GATE, int W, int LS, int MINB>
@@ -460,7 +461,8 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
         }
     }
     // every CTA has read state_in (and its remote reads are done) once all
-    // arrive here; the last part writes state_out after that
+    // arrive here; the last part writes state_out after that (and, in a
+    // chain, overwrites the words every part has read by then)
     cluster_arrive_release();
     if (warp == W - 1 && q == last) {
         cluster_wait_acquire();
@@ -478,9 +480,9 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
             }
         }
         if (A.chain != nullptr) {
-            // state_out before the word: the next call writes state_out only
-            // after it has read the word
-            __threadfence();
+            // release: state_out before the word (the next call writes
+            // state_out only after it has read the word)
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
             if (cvalid) {
 #pragma unroll
                 for (int j = 0; j < V; ++j)
@@ -522,9 +524,11 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
     // the stores must have read shared memory before the CTA exits
     if (lane == 0 && A.y != nullptr && nvalid > 0) bulk_wait_group_read0();
     if (!(warp == W - 1 && q == last)) cluster_wait_acquire();
-    // a chained call has not waited for the previous kernel: it ends after
-    // it, so the stream's kernels still finish in order
-    if (chained) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // a chained call has not waited for the previous kernel: one CTA waits
+    // for it before exiting, so the grid still ends after the previous one
+    // (the stream's kernels finish in order) while every other CTA frees
+    // its SM slot for the next call at once
+    if (chained && blockIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace wkv
