@@ -408,6 +408,15 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
         }
     }
     cluster_arrive_release();
+    if (chained && warp == 0) {
+        // the entering state of a chained call, taken while the cluster's
+        // other parts reach the barrier (read by every warp after the CTA
+        // barrier below)
+        St x[V];
+        chain_take(A, bs * A.C + c, cvalid, x);
+#pragma unroll
+        for (int j = 0; j < V; ++j) s_in_chain[j][lane] = x[j];
+    }
     cluster_wait_acquire();
     // the parts before this one (all full), from the chunk start
     if (warp == W - 1) {
@@ -439,14 +448,8 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
     const int64_t lanes = A.B * A.C;
     St sin[V];
     if (chained) {
-        // the previous call of the chain published it; no wait for its end
-        if (warp == 0) {
-            St x[V];
-            chain_take(A, bs * A.C + c, cvalid, x);
-#pragma unroll
-            for (int j = 0; j < V; ++j) s_in_chain[j][lane] = x[j];
-        }
-        __syncthreads();
+        // the previous call of the chain published it (taken by warp 0 at
+        // the cluster barrier above); no wait for that kernel's end
 #pragma unroll
         for (int j = 0; j < V; ++j) sin[j] = s_in_chain[j][lane];
     } else {
