@@ -96,7 +96,11 @@ typedef enum {
  *                stream, or synchronised); they race otherwise.  With it,
  *                CTAs that split one sequence exchange partial states
  *                through it (decoupled look-back, state hand-off), which is
- *                the fastest schedule for most shapes.
+ *                the fastest schedule for most shapes.  An ungated bfloat16
+ *                call longer than 2048 tokens with 48 to 147 channel blocks
+ *                of 64 (B * ceil(C/64)) runs as a chain of launches of 1024
+ *                tokens instead, handing the state from launch to launch
+ *                through the workspace (see WKV_FLAG_CHAIN_NEXT below).
  *                NULL (or too small: it is then not touched) is accepted for
  *                every shape; the call then runs a schedule that needs no
  *                scratch: the sequential kernel for T <= 16; the cluster

@@ -83,6 +83,10 @@ constexpr int kClusterMinBlocks = 4;
 // (a portable cluster) per call.
 constexpr int kStreamW = 8;
 constexpr int kStreamMax = 8;
+// A longer call with few lane blocks runs as a chain of stream launches of
+// this many parts each, the state handed on through the workspace.
+constexpr int64_t kStreamLongParts = 4;
+constexpr int64_t kStreamLongMinLB = 48;
 template <typename IO>
 constexpr int stream_ls() { return sizeof(IO) == 2 ? 32 : 16; }
 constexpr int64_t stream_pt(int dtype) { return kStreamW * (dtype == WKV_BF16 ? 32 : 16); }
@@ -172,6 +176,13 @@ std::mutex g_chain_mutex;
 ChainRec g_chain[kChainSlots];
 int g_chain_evict = 0;
 
+// Positions of a chain's published words cycle through 1 .. 2^30 - 1 (a
+// word's tag holds 30 bits of position; 0 marks a chain's first call).
+constexpr uint32_t kChainPosMax = (1u << 30) - 1u;
+uint32_t chain_advance(uint32_t p, int64_t n) {
+    return static_cast<uint32_t>((static_cast<uint64_t>(p) + static_cast<uint64_t>(n) - 1u) % kChainPosMax) + 1u;
+}
+
 // Any call that uses a workspace outside a chain ends the workspace's chain.
 void chain_forget(const void* ws) {
     if (ws == nullptr) return;
@@ -181,9 +192,10 @@ void chain_forget(const void* ws) {
 }
 
 // Position whose words hold this call's entering state (0: none, the call
-// reads state_in), and the record of this call for the next one.
+// reads state_in), and the record of this call, which publishes `count`
+// positions (one per launch), for the next one.
 uint32_t chain_enter(const void* ws, bool next, const float* state_in, const float* state_out, int64_t B, int64_t C,
-                     int dtype) {
+                     int dtype, int64_t count) {
     std::lock_guard<std::mutex> lock(g_chain_mutex);
     ChainRec* rec = nullptr;
     for (ChainRec& r : g_chain)
@@ -201,9 +213,7 @@ uint32_t chain_enter(const void* ws, bool next, const float* state_in, const flo
         rec = &g_chain[g_chain_evict];
         g_chain_evict = (g_chain_evict + 1) % kChainSlots;
     }
-    // the position counter stays clear of 0, which marks no chain
-    const uint32_t out = (in + 1u) & 0x3fffffffu;
-    *rec = ChainRec{ws, state_out, B, C, dtype, out == 0u ? 1u : out};
+    *rec = ChainRec{ws, state_out, B, C, dtype, chain_advance(in, count)};
     return in;
 }
 
@@ -510,9 +520,13 @@ int dispatch_cluster(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, si
                 : launch_cluster<IO, false>(a, dtype, ws, ws_bytes, st);
 }
 
-// Stream kernel: one cluster of ceil(T / PT) CTAs per lane block.
+// Stream kernel: one cluster of ceil(T / PT) CTAs per lane block.  With
+// tc > 0 the call runs as a chain of launches of tc tokens each (the last
+// one shorter), the state handed from launch to launch through a.chain's
+// words: launch i waits for position a.chain_in advanced i times.
 template <typename IO, bool GATE>
-int launch_stream(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+int launch_stream(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t st,
+                  int64_t tc = 0) {
     constexpr int LS = stream_ls<IO>();
     using G = wkv::StreamGeometry<IO, GATE, kStreamW, LS>;
     auto kern = wkv::stream_forward_kernel<IO, GATE, kStreamW, LS, 3>;
@@ -526,52 +540,77 @@ int launch_stream(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace
         if (rc != WKV_OK) return rc;
         ready[dev] = true;
     }
-    const ChunkGeom g = chunk_geom(a.B, a.T, a.C, 2, G::PT);
-    if (g.nchunks < 1 || g.nchunks > kStreamMax || g.units > 0x7fffffffLL) return WKV_ERR_SHAPE;
-    a.nCB = g.nCB;
-    a.nLB = g.nLB;
-    a.nchunks = g.nchunks;
-    a.units = g.units;
+    const int64_t T = a.T;
+    const int64_t per = tc > 0 ? tc : T;
+    if (per < 1 || (per + G::PT - 1) / G::PT > kStreamMax || (tc > 0 && a.chain == nullptr)) return WKV_ERR_SHAPE;
+    {
+        const ChunkGeom g = chunk_geom(a.B, per, a.C, 2, G::PT);
+        if (g.units > 0x7fffffffLL) return WKV_ERR_SHAPE;
+    }
     a.hdr = workspace != nullptr && aligned(workspace, 256) && workspace_bytes >= sizeof(wkv::WsHeader)
                 ? reinterpret_cast<wkv::WsHeader*>(workspace)
                 : nullptr;
     a.aggw = nullptr;
     a.incw = nullptr;
+    // tensor maps over the whole arrays; each launch addresses its rows by t0
     CUtensorMap tk, tv, tr, ty;
-    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
-    if (!encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
+    if (!encode_map(&tk, a.k, dtype, a.B, T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
+    if (!encode_map(&tv, a.v, dtype, a.B, T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
     if (GATE) {
-        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
+        if (!encode_map(&tr, a.r, dtype, a.B, T, a.C, G::CB, G::PT)) return WKV_ERR_CUDA;
     } else {
         tr = tv;
     }
     // outputs: one box of a warp's LS rows (no y when only the state is wanted)
     if (a.y != nullptr) {
-        if (!encode_map(&ty, a.y, dtype, a.B, a.T, a.C, G::CB, LS)) return WKV_ERR_CUDA;
+        if (!encode_map(&ty, a.y, dtype, a.B, T, a.C, G::CB, LS)) return WKV_ERR_CUDA;
     } else {
         ty = tv;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(g.units));
-    cfg.blockDim = dim3(G::THREADS);
-    cfg.dynamicSmemBytes = G::SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(g.nchunks);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tk, tv, tr, ty, a));
+    const int64_t n = (T + per - 1) / per;
+    uint32_t pos = a.chain_in;
+    for (int64_t i = 0; i < n; ++i) {
+        wkv::ChunkArgs b = a;
+        b.t0 = i * per;
+        b.T = T - b.t0 < per ? T - b.t0 : per;
+        const ChunkGeom g = chunk_geom(b.B, b.T, b.C, 2, G::PT);
+        b.nCB = g.nCB;
+        b.nLB = g.nLB;
+        b.nchunks = g.nchunks;
+        b.units = g.units;
+        b.chain_in = pos;
+        b.chain_out = chain_advance(pos, 1);
+        pos = b.chain_out;
+        if (i > 0) {
+            b.s_in = nullptr;   // the entering state comes from the previous launch's words
+            b.early = 1u;       // this call's inputs are not written by its own launches
+        }
+        if (i + 1 < n) b.s_out = nullptr;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(g.units));
+        cfg.blockDim = dim3(G::THREADS);
+        cfg.dynamicSmemBytes = G::SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(g.nchunks);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        rc = record_cuda(cudaLaunchKernelEx(&cfg, kern, tk, tv, tr, ty, b));
+        if (rc != WKV_OK) return rc;
+    }
+    return WKV_OK;
 }
 
 template <typename IO>
-int dispatch_stream(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st) {
-    return gate ? launch_stream<IO, true>(a, dtype, ws, ws_bytes, st)
-                : launch_stream<IO, false>(a, dtype, ws, ws_bytes, st);
+int dispatch_stream(bool gate, const wkv::ChunkArgs& a, int dtype, void* ws, size_t ws_bytes, cudaStream_t st,
+                    int64_t tc = 0) {
+    return gate ? launch_stream<IO, true>(a, dtype, ws, ws_bytes, st, tc)
+                : launch_stream<IO, false>(a, dtype, ws, ws_bytes, st, tc);
 }
 
 // Part buffers per CTA: as many as fit beside kPartMinBlocks CTAs per SM
@@ -831,17 +870,34 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
         // kernel of the stream ends.
         const int64_t spt = stream_pt(dtype);
         const size_t eb = elem_bytes(dtype);
-        const bool stream_ok = part_ok && (y == nullptr || aligned(y, 16)) &&
-                               (state_out == nullptr || aligned(state_out, 8)) && (T + spt - 1) / spt <= kStreamMax;
-        if (stream_ok && (force == 8 || (force == 0 && nLB < sm_count()))) {
-            // a chunk chain publishes each call's end state at the start of
-            // the workspace, right after its header
-            const size_t chain_bytes = size_t(B) * size_t(C) * sizeof(wkv::Word);
-            if ((flags & (WKV_FLAG_CHAIN_BEGIN | WKV_FLAG_CHAIN_NEXT)) && workspace != nullptr &&
-                aligned(workspace, 256) && workspace_bytes >= 256 + chain_bytes) {
+        const size_t chain_bytes = size_t(B) * size_t(C) * sizeof(wkv::Word);
+        const bool chain_ws = workspace != nullptr && aligned(workspace, 256) && workspace_bytes >= 256 + chain_bytes;
+        const bool stream_io = part_ok && (y == nullptr || aligned(y, 16)) && (state_out == nullptr || aligned(state_out, 8));
+        const bool stream_ok = stream_io && (T + spt - 1) / spt <= kStreamMax;
+        // A longer call with room for the chain's words: a chain of stream
+        // launches of kStreamLongParts parts each.  It beats the part
+        // kernel's look-back when a launch fills the GPU and its tiles are
+        // small: ungated bfloat16 with at least kStreamLongMinLB lane blocks
+        // (measured: 1959 against 2144 us at B=1, T=262144, C=4096; but 369
+        // against 159 us with 8 lane blocks, and slower for gated or float32
+        // calls, whose tiles leave fewer CTAs per SM).
+        const bool stream_long = stream_io && !stream_ok && chain_ws &&
+                                 (force == 8 || (dtype == WKV_BF16 && r == nullptr && nLB >= kStreamLongMinLB));
+        if ((stream_ok || stream_long) && (force == 8 || (force == 0 && nLB < sm_count()))) {
+            const int64_t tc = stream_long ? kStreamLongParts * spt : 0;
+            const int64_t launches = stream_long ? (T + tc - 1) / tc : 1;
+            // a chain publishes each launch's end state at the start of the
+            // workspace, right after its header
+            const bool chain_call = (flags & (WKV_FLAG_CHAIN_BEGIN | WKV_FLAG_CHAIN_NEXT)) != 0;
+            if ((chain_call && chain_ws) || stream_long) {
                 a.chain = reinterpret_cast<wkv::Word*>(static_cast<char*>(workspace) + 256);
-                a.chain_in = chain_enter(workspace, (flags & WKV_FLAG_CHAIN_NEXT) != 0, state_in, state_out, B, C,
-                                         dtype);
+                if (chain_call) {
+                    a.chain_in = chain_enter(workspace, (flags & WKV_FLAG_CHAIN_NEXT) != 0, state_in, state_out, B,
+                                             C, dtype, launches);
+                } else {
+                    chain_forget(workspace);
+                    a.chain_in = 0u;
+                }
                 if (a.chain_in == 0u) {
                     // a new chain: no word of an earlier one may look current
                     const int rc = record_cuda(cudaMemsetAsync(a.chain, 0, chain_bytes, stream));
@@ -854,9 +910,9 @@ int run_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, cons
                 chain_forget(workspace);
             }
             const int rc = dtype == WKV_F32
-                               ? dispatch_stream<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream)
+                               ? dispatch_stream<float>(r != nullptr, a, dtype, workspace, workspace_bytes, stream, tc)
                                : dispatch_stream<__nv_bfloat16>(r != nullptr, a, dtype, workspace, workspace_bytes,
-                                                                stream);
+                                                                stream, tc);
             if (rc != WKV_OK) chain_forget(workspace);
             return rc;
         }

@@ -93,10 +93,14 @@ struct ChunkArgs {
     uint64_t wait_limit_ns;
     uint32_t early;     // stream kernel: inputs may be read before the previous kernel of the stream ends
     // stream kernel, chunk chains: [B * C] words the state after the call is
-    // published to (null: none), and the position in the chain whose word
-    // holds the entering state (0: the chain's first call reads s_in)
+    // published to (null: none), the position in the chain whose word holds
+    // the entering state (0: the chain's first call reads s_in), and the
+    // position the published words carry
     Word* chain;
-    uint32_t chain_in;
+    uint32_t chain_in, chain_out;
+    // stream kernel: first token of the launch within the arrays (the
+    // arrays' own T is the tensor maps'; this launch covers T tokens)
+    int64_t t0;
 };
 
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {

@@ -34,7 +34,9 @@
 // per-token bounds tests; a part that ends inside T takes the checked copy.
 //
 // One thread block cluster of P = ceil(T / PT) CTAs per 64-channel lane block,
-// one CTA per part of PT = W * LS tokens.  With the launch flag `early` (the
+// one CTA per part of PT = W * LS tokens.  The launch covers tokens
+// [A.t0, A.t0 + T) of the arrays (A.t0 > 0 when one long call runs as a
+// chain of launches).  With the launch flag `early` (the
 // caller declares that k, v, r, w, u are not written by work still running
 // on the stream) everything above the line runs before griddepcontrol.wait,
 // so under programmatic dependent launch it overlaps the previous call.
@@ -43,8 +45,8 @@
 // path (a copy that does not land turns into NaN outputs).
 //
 // Chunk chains (A.chain set): the last part's warp W-1 publishes the state
-// after the chunk as tagged words (tag = the next call's position in the
-// chain) right after writing state_out, before pass 2.  A call that
+// after the chunk as tagged words (tag = A.chain_out, the next call's
+// position in the chain) right after writing state_out, before pass 2.  A call that
 // continues a chain (A.chain_in > 0) does not wait for the previous kernel
 // to end: one warp per CTA polls for the words tagged with its position
 // (bounded in time), and one CTA waits for the previous kernel before it
@@ -352,9 +354,10 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         const uint32_t pbytes = static_cast<uint32_t>(min(static_cast<int64_t>(CB), A.C - x0)) * 4u;
         mbar_expect_tx(&full, G::NT * G::TILE + 2u * pbytes);
-        tma_load_3d(smem, &tk, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
-        tma_load_3d(smem + G::TILE, &tv, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
-        if (GATE) tma_load_3d(smem + 2 * G::TILE, &tr, x0, static_cast<int>(t_part), static_cast<int>(bs), &full);
+        const int ty0 = static_cast<int>(A.t0 + t_part);   // row of the part in the arrays
+        tma_load_3d(smem, &tk, x0, ty0, static_cast<int>(bs), &full);
+        tma_load_3d(smem + G::TILE, &tv, x0, ty0, static_cast<int>(bs), &full);
+        if (GATE) tma_load_3d(smem + 2 * G::TILE, &tr, x0, ty0, static_cast<int>(bs), &full);
         bulk_load(prm, A.w + x0, pbytes, &full);
         bulk_load(prm + CB, A.u + x0, pbytes, &full);
     }
@@ -489,7 +492,7 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
             if (cvalid) {
 #pragma unroll
                 for (int j = 0; j < V; ++j)
-                    st_word(A.chain + bs * A.C + c + j, so[j], word_tag(A.chain_in + 1u, kKindChain));
+                    st_word(A.chain + bs * A.C + c + j, so[j], word_tag(A.chain_out, kKindChain));
             }
         }
     }
@@ -515,7 +518,8 @@ stream_forward_kernel(const __grid_constant__ CUtensorMap tk, const __grid_const
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) {
-            tma_store_3d(&ty, smem + G::TILE + warp * LS * ROW, x0, static_cast<int>(t_seg), static_cast<int>(bs));
+            tma_store_3d(&ty, smem + G::TILE + warp * LS * ROW, x0, static_cast<int>(A.t0 + t_seg),
+                         static_cast<int>(bs));
             bulk_commit_group();
         }
     }

@@ -217,3 +217,49 @@ def test_missing_word_times_out():
     assert out["STATUS"] == "-7"           # WKV_ERR_TIMEOUT
     assert out["NAN"] == "True" and out["STATE_NAN"] == "True"
     assert out["AFTER_RESET"] == "0"
+
+
+# Calls longer than one stream launch (8 parts) with few lane blocks and a
+# workspace: ungated bfloat16 calls with at least 48 lane blocks run as a
+# chain of 4-part launches (forced with WKV_FORWARD_KERNEL=stream for the
+# others in test_forced_kernels_gpu.py).
+LONG = [
+    # B, T, C, dtype, gate, state
+    (1, 5000, 4096, torch.bfloat16, False, True),     # 5 launches, the last one ragged
+    (1, 2049, 4096, torch.bfloat16, False, False),    # one token past a single launch
+    (2, 3000, 2048, torch.bfloat16, False, True),
+    (1, 9000, 3100, torch.bfloat16, False, True),     # ragged channel block (49 lane blocks)
+]
+
+
+@pytest.mark.parametrize("B,T,C,dtype,gate,state", LONG)
+def test_long_call_equals_oracle(B, T, C, dtype, gate, state):
+    d = gen_case(B, T, C, dtype, gate, state, seed=T + C)
+    d["k"][:, ::991] = 50.0
+    ws = wkv.Workspace()
+    y, s = wkv.wkv_forward(d["w"], d["u"], d["k"], d["v"], d["r"], d["state"], workspace=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    check_forward(d, y, s)
+    # the state alone (no outputs) takes the same launches
+    s2 = wkv.wkv_state(d["w"], d["k"], d["v"], d["state"], workspace=ws)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(s2, s, rtol=1e-5, atol=1e-6)
+
+
+def test_long_calls_in_a_chain():
+    """A chain whose calls are themselves several launches long: positions
+    continue across the calls."""
+    T1, T2, T3, C = 5000, 3001, 4096, 4096
+    d = gen_case(1, T1 + T2 + T3, C, torch.bfloat16, False, True, seed=77)
+    ws = wkv.Workspace()
+    state = d["state"].clone()
+    ys = []
+    for i, (a, b) in enumerate(((0, T1), (T1, T1 + T2), (T1 + T2, T1 + T2 + T3))):
+        k, v = d["k"][:, a:b].contiguous(), d["v"][:, a:b].contiguous()
+        y, _ = wkv.wkv_forward(d["w"], d["u"], k, v, None, state, state_out=state, workspace=ws,
+                               chain="begin" if i == 0 else "next")
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    check_forward(d, torch.cat(ys, dim=1), state)

@@ -8,7 +8,9 @@ with the oracle on the same seeded inputs.
 - cluster: few lane blocks (where the stream kernel runs) and many (more
   clusters than fit the GPU at once), which with a workspace take the
   lane-resident kernel;
-- stream: many lane blocks, which take the lane-resident kernel.
+- stream: many lane blocks, which take the lane-resident kernel; and calls
+  longer than one launch that are gated, float32 or have few lane blocks,
+  which take the part kernel (forced, they run as a chain of launches).
 """
 import os
 import subprocess
@@ -64,6 +66,9 @@ FORCED = {
         (5, 1000, 3840, "float32", True, True),      # 300 clusters of 8 CTAs
         (7, 130, 2728, "bfloat16", True, True),      # ragged channel block
         (3, 2048, 4096, "bfloat16", False, True),    # 8 parts of 256 tokens, 192 lane blocks
+        (2, 3000, 128, "float32", True, True),       # a chain of six 512-token launches
+        (1, 5000, 256, "bfloat16", True, False),     # five 1024-token launches, the last ragged
+        (3, 2500, 72, "bfloat16", False, True),      # ragged channel block
     ],
 }
 
