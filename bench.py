@@ -1011,18 +1011,31 @@ def run_ours(args):
         "clocks": clocks.summary(t0, t1),
     }
     if isinstance(case, Wkv5Case):
-        # the recurrence is bound by FP32 arithmetic: the roofline is the FP32
-        # pipe; the memory fraction stays beside it
+        # the recurrence on the CUDA cores is bound by FP32 arithmetic: its
+        # roofline is the FP32 pipe; the tensor-core blocks move that work onto
+        # the tensor cores, and their bound is the memory traffic
         tflops = case.flops / per_launch / 1e12
+        tc_kernel = (os.environ.get("WKV5_KERNEL") != "recurrent" and case.wl.dtype == "bf16"
+                     and case.C // case.H == 64)
         out["metric"] = METRIC_WKV5
         out["config"].update({"H": case.H, "head_size": case.C // case.H, "decay": (
-            "per token and channel (v6)" if case.wl.per_token_decay else "per channel (v5)"), "gate": False})
-        out["roofline"] = {"bound": "alu", "achieved": tflops, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                           "frac": tflops / FP32_PEAK_TFLOPS,
-                           "peak_kind": "derived: 148 SMs x 128 FP32 FMA/clock x 2 x 1965 MHz",
-                           "flops_per_launch": case.flops, "algorithmic_bytes_per_launch": case.bytes,
-                           "hbm_frac_of_measured": achieved / peak, "scope": "the step's one kernel",
-                           "traffic": load_traffic(args.workload + "_wkv5")}
+            "per token and channel (v6)" if case.wl.per_token_decay else "per channel (v5)"), "gate": False,
+            "kernel": ("recurrence on the CUDA cores (WKV5_KERNEL=recurrent)"
+                       if os.environ.get("WKV5_KERNEL") == "recurrent" or case.wl.dtype != "bf16" or case.C // case.H != 64
+                       else "blocks of 64 tokens on the tensor cores (tcgen05, tf32)")})
+        if tc_kernel:
+            out["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                               "frac": achieved / peak, "peak_kind": peak_kind,
+                               "algorithmic_bytes_per_launch": case.bytes, "scope": "the step's one kernel",
+                               "recurrence_tflops": tflops, "recurrence_flops_per_launch": case.flops,
+                               "traffic": load_traffic(args.workload + "_wkv5")}
+        else:
+            out["roofline"] = {"bound": "alu", "achieved": tflops, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                               "frac": tflops / FP32_PEAK_TFLOPS,
+                               "peak_kind": "derived: 148 SMs x 128 FP32 FMA/clock x 2 x 1965 MHz",
+                               "flops_per_launch": case.flops, "algorithmic_bytes_per_launch": case.bytes,
+                               "hbm_frac_of_measured": achieved / peak, "scope": "the step's one kernel",
+                               "traffic": load_traffic(args.workload + "_wkv5")}
     if not args.no_e2e:
         e2e_steps = min(args.steps, 2 if isinstance(case, StreamCase) else args.e2e_steps)
         e = e2e_measure(case, wkv, ws, e2e_steps, 1 if isinstance(case, StreamCase) else 2, stream)

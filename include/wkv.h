@@ -435,8 +435,14 @@ int wkv_abi_version(void);
  *                overlap anything else.  Feeding it back as the next call's
  *                state_in chains chunks exactly like one pass.
  * Errors as wkv_forward (WKV_ERR_SHAPE for a head size other than 32 or 64).
- * The recurrence runs in float32 on the CUDA cores: 2 N multiply-adds per
- * element.  Asynchronous on `stream`; no workspace.
+ * bfloat16 heads of 64 (with y, r, k, v, w and the states 16-byte aligned)
+ * run in blocks of up to 64 tokens on the tensor cores: the same sums
+ * regrouped into 64 x 64 products, with tf32 operands for the outputs
+ * (errors of order 1e-3 of the output's magnitude, below bf16's own
+ * rounding) and float32 accuracy kept for the state.  Every other call runs
+ * the recurrence in float32 on the CUDA cores (2 N multiply-adds per
+ * element); the environment variable WKV5_KERNEL=recurrent, read once per
+ * process, keeps every call on it.  Asynchronous on `stream`; no workspace.
  */
 int wkv5_forward(int64_t B, int64_t T, int64_t C, int64_t H, int dtype,
                  const float* w, int w_per_token, const float* u,

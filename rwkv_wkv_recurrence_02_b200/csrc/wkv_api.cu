@@ -23,6 +23,7 @@
 #include "wkv_step.cuh"
 #include "wkv_shift.cuh"
 #include "wkv5.cuh"
+#include "wkv5_tc.cuh"
 
 namespace {
 
@@ -1470,6 +1471,55 @@ int launch_wkv5(const wkv::Wkv5Args& a, cudaStream_t st) {
     return record_cuda(cudaLaunchKernelEx(&cfg, kern, a));
 }
 
+// Matrix-state WKV in blocks of tokens on the tensor cores: one CTA of 128
+// threads per (sequence, head).
+template <bool PERTOK>
+int launch_wkv5_tc(const wkv::Wkv5Args& a, cudaStream_t st) {
+    using SG = wkv::TcStage<PERTOK>;
+    auto kern = wkv::wkv5_tc_kernel<PERTOK>;
+    static bool ready[kMaxDevices] = {false};
+    int dev = 0;
+    int rc = record_cuda(cudaGetDevice(&dev));
+    if (rc != WKV_OK) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return WKV_ERR_CUDA;
+    if (!ready[dev]) {
+        rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM));
+        if (rc != WKV_OK) return rc;
+        ready[dev] = true;
+    }
+    // windows of 64 tokens x one head's 64 channels
+    CUtensorMap tr, tk, tv, tw;
+    if (!encode_map(&tr, a.r, WKV_BF16, a.B, a.T, a.C, 64, 64) || !encode_map(&tk, a.k, WKV_BF16, a.B, a.T, a.C, 64, 64) ||
+        !encode_map(&tv, a.v, WKV_BF16, a.B, a.T, a.C, 64, 64))
+        return WKV_ERR_CUDA;
+    if (PERTOK) {
+        if (!encode_map(&tw, a.w, WKV_F32, a.B, a.T, a.C, 64, 64)) return WKV_ERR_CUDA;
+    } else {
+        tw = tk;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.H));
+    cfg.blockDim = dim3(wkv::kTcThreads);
+    cfg.dynamicSmemBytes = SG::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return record_cuda(cudaLaunchKernelEx(&cfg, kern, tr, tk, tv, tw, a));
+}
+
+// WKV5_KERNEL=recurrent keeps every shape on the CUDA-core recurrence; read
+// once.
+bool wkv5_recurrent_forced() {
+    static const bool v = []() {
+        const char* e = std::getenv("WKV5_KERNEL");
+        return e != nullptr && std::strcmp(e, "recurrent") == 0;
+    }();
+    return v;
+}
+
 template <typename IO, int N>
 int dispatch_wkv5(bool pertok, const wkv::Wkv5Args& a, cudaStream_t st) {
     return pertok ? launch_wkv5<IO, N, true>(a, st) : launch_wkv5<IO, N, false>(a, st);
@@ -1528,7 +1578,17 @@ int wkv5_forward(int64_t B, int64_t T, int64_t C, int64_t H, int dtype, const fl
     a.H = H;
     const bool pt = w_per_token != 0;
     int rc;
-    if (dtype == WKV_F32)
+    // bf16 heads of 64 take the tensor-core blocks (their outputs carry tf32
+    // products, within bf16's own rounding; the state keeps fp32 accuracy);
+    // they read r, k, v, w by TMA and store y and the states 16 bytes at a
+    // time.  float32 keeps the exact-fp32 recurrence.
+    const bool tc = dtype == WKV_BF16 && N == 64 && aligned(y, 16) && (!state_in || aligned(state_in, 16)) &&
+                    (!state_out || aligned(state_out, 16)) && aligned(r, 16) && aligned(k, 16) && aligned(v, 16) &&
+                    (!pt || aligned(w, 16)) && T < (int64_t(1) << 31) && B < (int64_t(1) << 31) &&
+                    encode_fn() != nullptr && !wkv5_recurrent_forced();
+    if (tc)
+        rc = pt ? launch_wkv5_tc<true>(a, stream) : launch_wkv5_tc<false>(a, stream);
+    else if (dtype == WKV_F32)
         rc = N == 64 ? dispatch_wkv5<float, 64>(pt, a, stream) : dispatch_wkv5<float, 32>(pt, a, stream);
     else
         rc = N == 64 ? dispatch_wkv5<__nv_bfloat16, 64>(pt, a, stream) : dispatch_wkv5<__nv_bfloat16, 32>(pt, a, stream);
