@@ -29,22 +29,30 @@
 // in 8 steps of 8, operands fp32 in shared memory read as tf32, K-major,
 // no swizzle:
 //   batch 1:  D_A  = R~ K~^T          (scores before masking)
-//             D_Y  = R^ S0            (inter outputs)
+//             D_Y  = R~ S0'           (inter outputs)
 //             D_S  = hi(K^)^T V       (state increment)
 //   batch 2:  D_Y += mask(D_A) V      (intra outputs and the bonus diagonal)
 //             D_S += lo(K^)^T V
+// R~ = r e^{-(Lam_t - Lam_m)} already carries the inter factor but for a
+// per-channel e^{-Lam_m}, which goes into the state instead: S0' =
+// diag(e^{-Lam_m}) S0, so R~ S0' = sum_i r_t[i] e^{-Lam_t[i]} S0[i][:].
 // K^ = k e^{-(Lam_L - Lam_{s+1})} is split into hi + lo (hi: the 19 bits tf32
 // keeps, lo: the rest), so the state increment keeps fp32 accuracy (v is
 // bf16, exact in tf32); the outputs take the tf32 products (errors of order
 // 1e-3 of the output scale, below the bf16 output's own rounding).  The state
 // S stays fp32 in registers: the M = 64 accumulator layout puts row 16q + l
 // in lane l of tensor-memory lane quarter q; warps q and q + 4 read that
-// quarter, the first columns [0, 32), the second [32, 64), and thread l < 16
-// owns that half row of S.
+// quarter, the first columns [0, 32), the second [32, 64), with the
+// 16-lane x 256-bit load shape, in which thread l holds rows l / 4 and
+// l / 4 + 8 of the 16 and, of every 8 columns, columns 2 (l % 4) and
+// 2 (l % 4) + 1: 16 entries of S per thread.
 // One thread issues the MMAs; tcgen05.commit arrives on an mbarrier that the
 // others wait on (bounded).  A window's r, k, v (and per-token w) come by TMA
-// into a two-stage ring one window ahead.  Tensor memory: 3 accumulators of
-// 64 columns, 256 columns allocated; one CTA per SM (shared memory).
+// into a ring: for per-channel decays one stage, refilled once the window's
+// last block has read it, so that two CTAs fit per SM (113.7 KB of shared
+// memory, at most 128 registers); for per-token decays (16 KB more per stage)
+// two stages, one window ahead, and one CTA per SM.  Tensor memory: 3
+// accumulators of 64 columns, 256 columns allocated per CTA.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -63,7 +71,7 @@ namespace wkv {
 // groups, so the staging stores do not conflict.
 constexpr uint32_t kTcLbo = 9, kTcSbo = 17, kTcKs = 138;
 constexpr uint32_t kTcTile = (7 * kTcKs + 8 * kTcSbo) * 16;   // one fp32 operand tile (17632 bytes)
-constexpr uint32_t kTcTiles = 6 * kTcTile;          // R~, K~, R^, hi(K^)^T, V^T, S0^T
+constexpr uint32_t kTcTiles = 5 * kTcTile;          // R~, K~, hi(K^)^T, V^T, S0'^T
 // Staging ring: a window's r, k, v (bf16) and, with per-token decays, w (fp32)
 // as 64 tokens x 64 channels, brought by TMA one window ahead.
 template <bool PERTOK>
@@ -71,8 +79,10 @@ struct TcStage {
     static constexpr uint32_t IO = 64 * 64 * 2;                   // one bf16 array
     static constexpr uint32_t W = PERTOK ? 64 * 64 * 4 : 0;       // the decays
     static constexpr uint32_t BYTES = 3 * IO + W;
+    static constexpr uint32_t NST = PERTOK ? 2 : 1;               // ring stages
+    static constexpr int MINB = PERTOK ? 1 : 2;                   // CTAs per SM
     static constexpr uint32_t BASE = (kTcTiles + 1023u) & ~1023u; // stages start 1024-byte aligned
-    static constexpr uint32_t SMEM = BASE + 2 * BYTES;            // tiles, then two stages
+    static constexpr uint32_t SMEM = BASE + NST * BYTES;          // tiles, then the stages
 };
 constexpr uint32_t kTcCols = 256;                   // tensor memory columns allocated
 constexpr float kTcSpan = 60.f;                     // bound of |Lam_t - Lam_m| (natural units)
@@ -119,25 +129,28 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 accumulator columns of this thread's tensor-memory lane (warp-wide).
-__device__ __forceinline__ void tc_ld_row32(uint32_t taddr, float* x) {
+// 16 accumulator rows (lanes 0..15 of the warp's lane quarter) x 32 columns
+// from taddr's column (warp-wide, 16-lane x 256-bit shape, 4 repeats):
+// x[4 g + 2 h + e] = row l / 4 + 8 h, column 8 g + 2 (l % 4) + e.
+__device__ __forceinline__ void tc_ld16x32(uint32_t taddr, float* x) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int c = 0; c < 32; c += 16) {
-        uint32_t r[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-            : "r"(taddr + static_cast<uint32_t>(c))
-            : "memory");
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-        for (int q = 0; q < 16; ++q) x[c + q] = __uint_as_float(r[q]);
-    }
+    for (int q = 0; q < 16; ++q) x[q] = __uint_as_float(r[q]);
 }
 
 __device__ __forceinline__ void tc_st(unsigned char* tile, int row, int k, float x) {
     *reinterpret_cast<float*>(tile + tc_off(row, k)) = x;
+}
+// two consecutive k (k even) of one row: half a slot
+__device__ __forceinline__ void tc_st2(unsigned char* tile, int row, int k, float a, float b) {
+    *reinterpret_cast<float2*>(tile + tc_off(row, k)) = make_float2(a, b);
 }
 // four consecutive k (k % 4 == 0) of one row: one slot
 __device__ __forceinline__ void tc_st4(unsigned char* tile, int row, int k, float a, float b, float c, float d) {
@@ -170,31 +183,29 @@ __device__ __forceinline__ int tc_block_len(int n, Rate rate) {
 }
 
 template <bool PERTOK>
-__global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_constant__ CUtensorMap tr,
-                                                                const __grid_constant__ CUtensorMap tk,
-                                                                const __grid_constant__ CUtensorMap tv,
-                                                                const __grid_constant__ CUtensorMap tw,
-                                                                const Wkv5Args A) {
+__global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
+    wkv5_tc_kernel(const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
+                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw, const Wkv5Args A) {
     using SG = TcStage<PERTOK>;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char* RT = smem;                  // R~ [t][i]; after batch 1: lo(K^)^T [i][s]
     unsigned char* KT = smem + kTcTile;        // K~ [s][i]; after batch 1: the masked scores [t][s]
-    unsigned char* RH = smem + 2 * kTcTile;    // R^ [t][i] = r e^{-Lam_t}
-    unsigned char* KH = smem + 3 * kTcTile;    // hi(K^)^T [i][s]
-    unsigned char* VT = smem + 4 * kTcTile;    // V^T [j][s]
-    unsigned char* ST = smem + 5 * kTcTile;    // S0^T [j][i]
+    unsigned char* KH = smem + 2 * kTcTile;    // hi(K^)^T [i][s]
+    unsigned char* VT = smem + 3 * kTcTile;    // V^T [j][s]
+    unsigned char* ST = smem + 4 * kTcTile;    // S0'^T [j][i] = e^{-Lam_m[i]} S0[i][j]
     __shared__ __align__(8) uint64_t bar[2], full[2];
     __shared__ uint32_t tslot;
-    __shared__ float s_u[64], s_eend[64];
+    __shared__ float s_u[64], s_eend[64], s_emid[64];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // staging: channel ci, tokens [16 qq, 16 qq + 16) of a block
     const int ci = tid & 63, qq = tid >> 6;
-    // accumulators: warp w reads lane quarter w % 4 (rows 16 (w % 4) + lane,
-    // lanes < 16 of the M = 64 layout) and columns [32 (w / 4), +32)
-    const int rr = 16 * (warp & 3) + lane;
+    // accumulators: warp w reads lane quarter w % 4 (rows 16 (w % 4) .. + 15)
+    // and columns [c0, c0 + 32); this thread holds rows R0 + 8 h and, of
+    // every 8 columns from c0, columns 2 (lane % 4) + e
+    const int R0 = 16 * (warp & 3) + (lane >> 2);
     const int c0 = 32 * (warp >> 2);
-    const bool has_row = lane < 16;
+    const int cl = 2 * (lane & 3);
     const int64_t bh = blockIdx.x, b = bh / A.H, h = bh % A.H;
     const int64_t T = A.T, C = A.C;
     const int64_t ch0 = h * 64;
@@ -204,10 +215,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // TMA of window wi's r, k, v (and w) into stage wi & 1
+    // TMA of window wi's r, k, v (and w) into its stage
     auto fetch = [&](int64_t wi) {
-        unsigned char* st = smem + SG::BASE + static_cast<uint32_t>(wi & 1) * SG::BYTES;
-        uint64_t* fb = &full[wi & 1];
+        const uint32_t sidx = SG::NST == 2 ? static_cast<uint32_t>(wi & 1) : 0u;
+        unsigned char* st = smem + SG::BASE + sidx * SG::BYTES;
+        uint64_t* fb = &full[sidx];
         mbar_expect_tx(fb, SG::BYTES);
         const int x = static_cast<int>(ch0), y = static_cast<int>(wi * 64), z = static_cast<int>(b);
         tma_load_3d(st, &tr, x, y, z, fb);
@@ -234,19 +246,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid < 64) s_u[tid] = A.u[ch0 + tid];
-    // the state this thread owns: row rr, columns [c0, c0 + 32)
-    float S[32];
+    // the state this thread owns: S[4 g + 2 hh + e] = S[R0 + 8 hh][c0 + 8 g + cl + e]
+    float S[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) S[j] = 0.f;
-    if (has_row && A.s_in != nullptr) {
-        const float4* src = reinterpret_cast<const float4*>(A.s_in + (bh * 64 + rr) * 64 + c0);
+    for (int j = 0; j < 16; ++j) S[j] = 0.f;
+    if (A.s_in != nullptr) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 x = src[q];
-            S[4 * q] = x.x;
-            S[4 * q + 1] = x.y;
-            S[4 * q + 2] = x.z;
-            S[4 * q + 3] = x.w;
+        for (int hh = 0; hh < 2; ++hh) {
+            const float* src = A.s_in + (bh * 64 + R0 + 8 * hh) * 64 + c0 + cl;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const float2 x = *reinterpret_cast<const float2*>(src + 8 * g);
+                S[4 * g + 2 * hh] = x.x;
+                S[4 * g + 2 * hh + 1] = x.y;
+            }
         }
     }
     tc_fence_before();
@@ -257,27 +270,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
     // loads add this warp's lane quarter and column half
     const uint32_t tA = tbase, tY = tbase + 64, tS = tbase + 128;
     const uint32_t lane_off = (static_cast<uint32_t>(32 * (warp & 3)) << 16) + static_cast<uint32_t>(c0);
-    const uint32_t aRT = smem_u32(RT), aKT = smem_u32(KT), aRH = smem_u32(RH), aKH = smem_u32(KH),
-                   aVT = smem_u32(VT), aST = smem_u32(ST);
+    const uint32_t aRT = smem_u32(RT), aKT = smem_u32(KT), aKH = smem_u32(KH), aVT = smem_u32(VT),
+                   aST = smem_u32(ST);
     uint32_t phase = 0;
     bool ok = true;
+    int64_t issued = 1, consumed = 0;   // windows whose copy was started / waited for
 
     const float wc = PERTOK ? 0.f : A.w[ch0 + ci];
+    // per-channel decays: the factors of consecutive tokens differ by e^{-+w}
+    const float dec1 = PERTOK ? 1.f : ex2(-wc * kLog2e), inc1 = PERTOK ? 1.f : ex2(wc * kLog2e);
     for (int64_t w0 = 0; w0 < T && ok; w0 += 64) {
         const int wn = static_cast<int>(T - w0 < 64 ? T - w0 : 64);
         const int64_t wi = w0 / 64;
-        // this window's inputs; the next window's copy starts now (the stage
-        // it overwrites was last read two windows ago)
-        if (tid == 0 && w0 + 64 < T) fetch(wi + 1);
-        ok = __syncthreads_and(mbar_wait(&full[wi & 1], static_cast<uint32_t>((wi >> 1) & 1), kCopyWaitNs));
-        if (!ok) {
-            // a copy that did not land: let the next window's copy land before
-            // this CTA's shared memory is released
-            if (tid == 0 && w0 + 64 < T)
-                mbar_wait(&full[(wi + 1) & 1], static_cast<uint32_t>(((wi + 1) >> 1) & 1), kCopyWaitNs);
-            break;
+        const uint32_t sidx = SG::NST == 2 ? static_cast<uint32_t>(wi & 1) : 0u;
+        const uint32_t spar = SG::NST == 2 ? static_cast<uint32_t>((wi >> 1) & 1) : static_cast<uint32_t>(wi & 1);
+        // two stages: the next window's copy starts now (the stage it
+        // overwrites was last read two windows ago)
+        if (SG::NST == 2 && w0 + 64 < T) {
+            if (tid == 0) fetch(wi + 1);
+            issued = wi + 2;
         }
-        const unsigned char* st = smem + SG::BASE + static_cast<uint32_t>(wi & 1) * SG::BYTES;
+        ok = __syncthreads_and(mbar_wait(&full[sidx], spar, kCopyWaitNs));
+        if (!ok) break;
+        consumed = wi + 1;
+        const unsigned char* st = smem + SG::BASE + sidx * SG::BYTES;
         const __nv_bfloat16* sr = reinterpret_cast<const __nv_bfloat16*>(st);
         const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(st + SG::IO);
         const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(st + 2 * SG::IO);
@@ -295,11 +311,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
         }
         const int L = !__syncthreads_or(lm < 64) ? 64 : !__syncthreads_or(lm < 16) ? 16
                     : !__syncthreads_or(lm < 4)  ? 4  : 1;
+        // In a block of more than one token no factor is clamped, so the
+        // state-increment factor follows from the intra one:
+        // e^{-(Lam_L - Lam_{t+1})} = e^{Lam_{t+1} - Lam_m} e^{-(Lam_L - Lam_m)}.
+        // (The inter factor e^{-Lam_t} = e^{Lam_m - Lam_t} e^{-Lam_m} holds in
+        // every block: in a block of one token both sides are 1.)
+        const bool tame = L > 1;
 
         for (int b0 = 0; b0 < wn && ok; b0 += L) {
             const int bl = wn - b0 < L ? wn - b0 : L;   // tokens of this block
             const int mid = bl / 2;                     // the reference token
             const int64_t t0 = w0 + b0;
+            const bool last_block = b0 + L >= wn;
             // ---- stage 1: decays and the operand tiles ----
             // Lam at the middle and at the end of the block, and at this
             // thread's first row, for channel ci
@@ -316,57 +339,84 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
                 lam_end = static_cast<float>(bl) * wc;
                 lam_row = static_cast<float>(min(16 * qq, bl)) * wc;
             }
-            if (qq == 0) s_eend[ci] = ex2(-lam_end * kLog2e);
-            // In a block of more than one token no factor is clamped, so the
-            // inter factors follow from the intra ones: e^{-Lam_t} =
-            // e^{Lam_m - Lam_t} e^{-Lam_m}, and the state-increment factor
-            // e^{-(Lam_L - Lam_{t+1})} = e^{Lam_{t+1} - Lam_m} e^{-(Lam_L - Lam_m)}.
-            const bool tame = L > 1;
             const float emid = ex2(-lam_mid * kLog2e), erest = ex2(-(lam_end - lam_mid) * kLog2e);
-            float klo[16], khq[4], vq[4];
-            float lam = lam_row;
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int t = 16 * qq + q;
-                float r = 0.f, k = 0.f, v = 0.f, er = 0.f, ek = 0.f, eh = 0.f, eg = 0.f;
-                if (t < bl) {
-                    const int e = (b0 + t) * 64 + ci;   // window row b0 + t, channel ci
-                    r = __bfloat162float(sr[e]);
-                    k = __bfloat162float(sk[e]);
-                    v = __bfloat162float(sv[e]);
-                    float lt, lt1;
-                    if (PERTOK) {
-                        lt = lam;
-                        lam += rate(b0 + t);
-                        lt1 = lam;
-                    } else {
-                        lt = static_cast<float>(t) * wc;
-                        lt1 = static_cast<float>(t + 1) * wc;
-                    }
-                    er = ex2(fminf(lam_mid - lt, kTcSpan) * kLog2e);
-                    ek = ex2(fminf(lt1 - lam_mid, kTcSpan) * kLog2e);
-                    eh = tame ? er * emid : ex2(-lt * kLog2e);
-                    eg = tame ? ek * erest : ex2(-(lam_end - lt1) * kLog2e);
+            if (qq == 0) {
+                s_eend[ci] = ex2(-lam_end * kLog2e);
+                s_emid[ci] = emid;
+            }
+            // per-token decays (one CTA per SM, registers to spare): lo(K^)
+            // is kept from here to stage 3; per-channel decays form it again
+            float klo[PERTOK ? 16 : 1];
+            {
+                float khq[4], vq[4];
+                float lam = lam_row;
+                // per-channel decays in a block of more than one token: the
+                // factors of the thread's first token, then products
+                float er = 1.f, ek = 1.f;
+                if (!PERTOK && tame) {
+                    const float t1 = static_cast<float>(16 * qq);
+                    er = ex2((lam_mid - t1 * wc) * kLog2e);
+                    ek = ex2(((t1 + 1.f) * wc - lam_mid) * kLog2e);
                 }
-                // row t across 32 channels: one word per lane, no bank conflict
-                tc_st(RT, t, ci, r * er);
-                tc_st(KT, t, ci, k * ek);
-                tc_st(RH, t, ci, r * eh);
-                const float kh_full = k * eg;
-                const float kh = __uint_as_float(__float_as_uint(kh_full) & 0xFFFFE000u);   // the bits tf32 keeps
-                klo[q] = kh_full - kh;
-                khq[q & 3] = kh;
-                vq[q & 3] = v;
-                if ((q & 3) == 3) {
-                    // channel ci's row, four tokens: one slot per lane
-                    tc_st4(KH, ci, t - 3, khq[0], khq[1], khq[2], khq[3]);
-                    tc_st4(VT, ci, t - 3, vq[0], vq[1], vq[2], vq[3]);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int t = 16 * qq + q;
+                    float rt = 0.f, kt = 0.f, kh_full = 0.f, v = 0.f;
+                    if (t < bl) {
+                        const int e = (b0 + t) * 64 + ci;   // window row b0 + t, channel ci
+                        const float r = __bfloat162float(sr[e]);
+                        const float k = __bfloat162float(sk[e]);
+                        v = __bfloat162float(sv[e]);
+                        float fr, fk, fg;
+                        if (!PERTOK && tame) {
+                            fr = er;
+                            fk = ek;
+                            fg = ek * erest;
+                            er *= dec1;
+                            ek *= inc1;
+                        } else {
+                            float lt, lt1;
+                            if (PERTOK) {
+                                lt = lam;
+                                lam += rate(b0 + t);
+                                lt1 = lam;
+                            } else {
+                                lt = static_cast<float>(t) * wc;
+                                lt1 = static_cast<float>(t + 1) * wc;
+                            }
+                            fr = ex2(fminf(lam_mid - lt, kTcSpan) * kLog2e);
+                            fk = ex2(fminf(lt1 - lam_mid, kTcSpan) * kLog2e);
+                            fg = tame ? fk * erest : ex2(-(lam_end - lt1) * kLog2e);
+                        }
+                        rt = r * fr;
+                        kt = k * fk;
+                        kh_full = k * fg;
+                    }
+                    // row t across 32 channels: one word per lane, no bank conflict
+                    tc_st(RT, t, ci, rt);
+                    tc_st(KT, t, ci, kt);
+                    khq[q & 3] = __uint_as_float(__float_as_uint(kh_full) & 0xFFFFE000u);   // the bits tf32 keeps
+                    if constexpr (PERTOK) klo[q] = kh_full - khq[q & 3];
+                    vq[q & 3] = v;
+                    if ((q & 3) == 3) {
+                        // channel ci's row, four tokens: one slot per lane
+                        tc_st4(KH, ci, t - 3, khq[0], khq[1], khq[2], khq[3]);
+                        tc_st4(VT, ci, t - 3, vq[0], vq[1], vq[2], vq[3]);
+                    }
                 }
             }
-            // S0^T for the inter product: this thread's half row of S
-            if (has_row) {
+            // S0'^T for the inter product: this thread's entries of S, times
+            // e^{-Lam_m} of their row's channel
+            __syncthreads();   // s_emid
+            {
+                const float em[2] = {s_emid[R0], s_emid[R0 + 8]};
 #pragma unroll
-                for (int j = 0; j < 32; ++j) tc_st(ST, c0 + j, rr, S[j]);
+                for (int g = 0; g < 4; ++g)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e)
+                            tc_st(ST, c0 + 8 * g + cl + e, R0 + 8 * hh, S[4 * g + 2 * hh + e] * em[hh]);
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
@@ -375,7 +425,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
             // ---- batch 1 ----
             if (tid == 0) {
                 tc_gemm(tA, aRT, aKT, false);
-                tc_gemm(tY, aRH, aST, false);
+                tc_gemm(tY, aRT, aST, false);
                 tc_gemm(tS, aKH, aVT, false);
                 tc_commit(&bar[0]);
             }
@@ -383,50 +433,104 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
             tc_fence_after();
             // ---- stage 3: masked scores, lo(K^)^T ----
             {
-                float a[32];
-                tc_ld_row32(lane_off + tA, a);
-                if (has_row) {
-                    // the bonus diagonal of row rr (in this warp's column
-                    // half): sum over the head's channels of r u k, from the
-                    // staged inputs of the token
-                    float dg = 0.f;
-                    if (rr < bl && rr >= c0 && rr < c0 + 32) {
-                        const uint4* r8 = reinterpret_cast<const uint4*>(sr + (b0 + rr) * 64);
-                        const uint4* k8 = reinterpret_cast<const uint4*>(sk + (b0 + rr) * 64);
+                // the bonus diagonal of rows R0 and R0 + 8 where this warp's
+                // column half holds them: sum over the head's channels of
+                // r u k, from the staged inputs of the token, split over the
+                // four threads of a row (16 channels each, the quarters
+                // rotated by row so that the 8 rows of a load do not share
+                // banks) and summed by two shuffles
+                float dg[2] = {0.f, 0.f};
+                if ((warp & 3) / 2 == warp / 4) {
+                    const int part = ((lane & 3) + (lane >> 2)) & 3;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            // lanes start at different 16-byte chunks of their
-                            // rows (rows are 128 bytes apart): no bank conflict
-                            const int c8 = (c + lane) & 7;
-                            const uint4 rv = r8[c8], kv = k8[c8];
-                            const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w}, kw[4] = {kv.x, kv.y, kv.z, kv.w};
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int row = R0 + 8 * hh;
+                        if (row < bl) {
+                            const uint4* r8 = reinterpret_cast<const uint4*>(sr + (b0 + row) * 64 + 16 * part);
+                            const uint4* k8 = reinterpret_cast<const uint4*>(sk + (b0 + row) * 64 + 16 * part);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float r0 = __uint_as_float(rw[e] << 16), r1 = __uint_as_float(rw[e] & 0xffff0000u);
-                                const float k0 = __uint_as_float(kw[e] << 16), k1 = __uint_as_float(kw[e] & 0xffff0000u);
-                                dg = fmaf(r0 * s_u[8 * c8 + 2 * e], k0, dg);
-                                dg = fmaf(r1 * s_u[8 * c8 + 2 * e + 1], k1, dg);
+                            for (int c = 0; c < 2; ++c) {
+                                const uint4 rv = r8[c], kv = k8[c];
+                                const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w}, kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int ch = 16 * part + 8 * c + 2 * e;
+                                    const float r0 = __uint_as_float(rw[e] << 16), r1 = __uint_as_float(rw[e] & 0xffff0000u);
+                                    const float k0 = __uint_as_float(kw[e] << 16), k1 = __uint_as_float(kw[e] & 0xffff0000u);
+                                    dg[hh] = fmaf(r0 * s_u[ch], k0, dg[hh]);
+                                    dg[hh] = fmaf(r1 * s_u[ch + 1], k1, dg[hh]);
+                                }
                             }
                         }
+                        dg[hh] += __shfl_xor_sync(0xffffffffu, dg[hh], 1);
+                        dg[hh] += __shfl_xor_sync(0xffffffffu, dg[hh], 2);
                     }
+                }
+                float a[16];
+                tc_ld16x32(lane_off + tA, a);
 #pragma unroll
-                    for (int s = 0; s < 32; s += 4) {
-                        float m[4];
+                for (int g = 0; g < 4; ++g) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int sc = c0 + s + e;
-                            m[e] = sc < rr ? a[s + e] : (sc == rr ? dg : 0.f);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int row = R0 + 8 * hh;
+                        float m[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int sc = c0 + 8 * g + cl + e;
+                            m[e] = sc < row ? a[4 * g + 2 * hh + e] : (sc == row ? dg[hh] : 0.f);
                         }
-                        tc_st4(KT, rr, c0 + s, m[0], m[1], m[2], m[3]);
+                        tc_st2(KT, row, c0 + 8 * g + cl, m[0], m[1]);
                     }
                 }
             }
+            if constexpr (PERTOK) {
 #pragma unroll
-            for (int q = 0; q < 16; q += 4) tc_st4(RT, ci, 16 * qq + q, klo[q], klo[q + 1], klo[q + 2], klo[q + 3]);
+                for (int q = 0; q < 16; q += 4) tc_st4(RT, ci, 16 * qq + q, klo[q], klo[q + 1], klo[q + 2], klo[q + 3]);
+            } else {
+                // lo(K^) of this thread's channel and tokens, formed again
+                // exactly as in stage 1, into R~'s tile (free after batch 1)
+                float lo[16];
+                float lam = lam_row;
+                float ek = 1.f;
+                if (!PERTOK && tame) ek = ex2(((static_cast<float>(16 * qq) + 1.f) * wc - lam_mid) * kLog2e);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int t = 16 * qq + q;
+                    lo[q] = 0.f;
+                    if (t < bl) {
+                        const float k = __bfloat162float(sk[(b0 + t) * 64 + ci]);
+                        float fg;
+                        if (!PERTOK && tame) {
+                            fg = ek * erest;
+                            ek *= inc1;
+                        } else {
+                            float lt1;
+                            if (PERTOK) {
+                                lam += rate(b0 + t);
+                                lt1 = lam;
+                            } else {
+                                lt1 = static_cast<float>(t + 1) * wc;
+                            }
+                            fg = tame ? ex2(fminf(lt1 - lam_mid, kTcSpan) * kLog2e) * erest
+                                      : ex2(-(lam_end - lt1) * kLog2e);
+                        }
+                        const float kh_full = k * fg;
+                        lo[q] = kh_full - __uint_as_float(__float_as_uint(kh_full) & 0xFFFFE000u);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 16; q += 4) tc_st4(RT, ci, 16 * qq + q, lo[q], lo[q + 1], lo[q + 2], lo[q + 3]);
+            }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
+            // one stage: the window's inputs are read (stage 1 and the lines
+            // above of its last block); the next window's copy starts now
+            if (SG::NST == 1 && last_block && w0 + 64 < T) {
+                if (tid == 0) fetch(wi + 1);
+                issued = wi + 2;
+            }
             // ---- batch 2 ----
             if (tid == 0 && ok) {
                 tc_gemm(tY, aKT, aVT, true);
@@ -437,28 +541,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
             tc_fence_after();
             // ---- stage 5: outputs, state ----
             {
-                float x[32];
-                tc_ld_row32(lane_off + tY, x);
-                if (has_row && rr < bl) {
-                    uint4* dst = reinterpret_cast<uint4*>(yg + (b * T + t0 + rr) * C + ch0 + c0);
+                float x[16];
+                tc_ld16x32(lane_off + tY, x);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t w4[4];
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int row = R0 + 8 * hh;
+                    if (row < bl) {
+                        __nv_bfloat16* dst = yg + (b * T + t0 + row) * C + ch0 + c0 + cl;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 p = __floats2bfloat162_rn(ok ? x[8 * q + 2 * e] : nan,
-                                                                     ok ? x[8 * q + 2 * e + 1] : nan);
-                            w4[e] = *reinterpret_cast<uint32_t*>(&p);
+                        for (int g = 0; g < 4; ++g) {
+                            const __nv_bfloat162 p = __floats2bfloat162_rn(ok ? x[4 * g + 2 * hh] : nan,
+                                                                           ok ? x[4 * g + 2 * hh + 1] : nan);
+                            *reinterpret_cast<__nv_bfloat162*>(dst + 8 * g) = p;
                         }
-                        dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
                 }
-                tc_ld_row32(lane_off + tS, x);
-                if (has_row) {
-                    const float dec = s_eend[rr];
+                tc_ld16x32(lane_off + tS, x);
+                const float dec[2] = {s_eend[R0], s_eend[R0 + 8]};
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) S[j] = ok ? fmaf(dec, S[j], x[j]) : nan;
-                }
+                for (int g = 0; g < 4; ++g)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 4 * g + 2 * hh + e;
+                            S[j] = ok ? fmaf(dec[hh], S[j], x[j]) : nan;
+                        }
             }
             tc_fence_before();
             __syncthreads();
@@ -466,12 +574,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) wkv5_tc_kernel(const __grid_con
             phase ^= 1u;
         }
     }
-    if (has_row && A.s_out != nullptr) {
-        float4* dst = reinterpret_cast<float4*>(A.s_out + (bh * 64 + rr) * 64 + c0);
+    // a wait that failed leaves copies started but not waited for: they
+    // must land before this CTA's shared memory is released
+    if (tid == 0) {
+        for (int64_t w = consumed; w < issued; ++w) {
+            const uint32_t si = SG::NST == 2 ? static_cast<uint32_t>(w & 1) : 0u;
+            const uint32_t sp = SG::NST == 2 ? static_cast<uint32_t>((w >> 1) & 1) : static_cast<uint32_t>(w & 1);
+            mbar_wait(&full[si], sp, kCopyWaitNs);
+        }
+    }
+    if (A.s_out != nullptr) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            dst[q] = ok ? make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3])
-                        : make_float4(nan, nan, nan, nan);
+        for (int hh = 0; hh < 2; ++hh) {
+            float* dst = A.s_out + (bh * 64 + R0 + 8 * hh) * 64 + c0 + cl;
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                *reinterpret_cast<float2*>(dst + 8 * g) =
+                    ok ? make_float2(S[4 * g + 2 * hh], S[4 * g + 2 * hh + 1]) : make_float2(nan, nan);
+        }
     }
     tc_fence_before();
     __syncthreads();

@@ -1485,6 +1485,11 @@ int launch_wkv5_tc(const wkv::Wkv5Args& a, cudaStream_t st) {
     if (!ready[dev]) {
         rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM));
         if (rc != WKV_OK) return rc;
+        // all of the unified L1 / shared memory as shared memory, so that the
+        // per-channel-decay kernel's two CTAs fit on one SM
+        rc = record_cuda(
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared));
+        if (rc != WKV_OK) return rc;
         ready[dev] = true;
     }
     // windows of 64 tokens x one head's 64 channels
