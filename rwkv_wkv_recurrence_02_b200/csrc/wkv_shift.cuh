@@ -19,6 +19,8 @@
 namespace wkv {
 
 constexpr int kShiftMaxMix = 8;
+// mixes whose mu a whole unit keeps in registers (more take the per-token loop)
+constexpr int kShiftRegMix = 4;
 
 template <typename IO, int V>
 struct ShiftVec;
@@ -120,24 +122,30 @@ token_shift_kernel(int64_t B, int64_t T, int64_t C, int nmix, const IO* __restri
         for (int j = 0; j < V; ++j) prev[j] = 0.f;
     }
     const int64_t plane = B * T * C;
-    if (t1 - t0 == TS) {
-        // a whole unit: all TS rows in flight before the first is used
+    if (t1 - t0 == TS && nmix <= kShiftRegMix) {
+        // a whole unit: all TS rows in flight before the first is used, and
+        // the mixes' mu of the unit's channels held in registers
         typename ShiftVec<IO, V>::Raw raw[TS];
 #pragma unroll
         for (int i = 0; i < TS; ++i) raw[i] = ShiftVec<IO, V>::load_raw(x + (b * T + t0 + i) * C + c);
+        float mm[kShiftRegMix][V];
+#pragma unroll
+        for (int m = 0; m < kShiftRegMix; ++m) {
+            if (m < nmix) {
+                ShiftVec<float, V == 8 ? 4 : V>::load(mu + m * C + c, mm[m]);
+                if constexpr (V == 8) ShiftVec<float, 4>::load(mu + m * C + c + 4, mm[m] + 4);
+            }
+        }
 #pragma unroll
         for (int i = 0; i < TS; ++i) {
             float cur[V];
             ShiftVec<IO, V>::widen_raw(raw[i], cur);
 #pragma unroll
-            for (int m = 0; m < kShiftMaxMix; ++m) {
+            for (int m = 0; m < kShiftRegMix; ++m) {
                 if (m < nmix) {
-                    // mu of the unit's channels (L1-resident after the first token)
-                    float mm[V], o[V];
-                    ShiftVec<float, V == 8 ? 4 : V>::load(mu + m * C + c, mm);
-                    if constexpr (V == 8) ShiftVec<float, 4>::load(mu + m * C + c + 4, mm + 4);
+                    float o[V];
 #pragma unroll
-                    for (int j = 0; j < V; ++j) o[j] = fmaf(mm[j], cur[j], (1.f - mm[j]) * prev[j]);
+                    for (int j = 0; j < V; ++j) o[j] = fmaf(mm[m][j], cur[j], (1.f - mm[m][j]) * prev[j]);
                     ShiftVec<IO, V>::store(out + m * plane + (b * T + t0 + i) * C + c, o);
                 }
             }
