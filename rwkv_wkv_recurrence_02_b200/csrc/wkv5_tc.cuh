@@ -47,11 +47,13 @@
 // l / 4 + 8 of the 16 and, of every 8 columns, columns 2 (l % 4) and
 // 2 (l % 4) + 1: 16 entries of S per thread.
 // One thread issues the MMAs; tcgen05.commit arrives on an mbarrier that the
-// others wait on (bounded).  A window's r, k, v (and per-token w) come by TMA
-// into a ring: for per-channel decays one stage, refilled once the window's
-// last block has read it, so that two CTAs fit per SM (113.7 KB of shared
-// memory, at most 128 registers); for per-token decays (16 KB more per stage)
-// two stages, one window ahead, and one CTA per SM.  Tensor memory: 3
+// others wait on (bounded).  A window's r, k, v come by TMA into one stage,
+// refilled once the window's last block has read it; per-token decays come
+// by TMA into the staged state's tile, which is free from the last block's
+// first batch of products until the next window's stage 1 writes it (the
+// decays are read before that; a window cut into blocks shorter than 64
+// tokens reads them from global memory instead).  So two CTAs fit per SM
+// (112.8 KB of shared memory, at most 128 registers).  Tensor memory: 3
 // accumulators of 64 columns, 256 columns allocated per CTA.
 #pragma once
 
@@ -74,15 +76,13 @@ constexpr uint32_t kTcTile = (7 * kTcKs + 8 * kTcSbo) * 16;   // one fp32 operan
 constexpr uint32_t kTcTiles = 5 * kTcTile;          // R~, K~, hi(K^)^T, V^T, S0'^T
 // Staging ring: a window's r, k, v (bf16) and, with per-token decays, w (fp32)
 // as 64 tokens x 64 channels, brought by TMA one window ahead.
-template <bool PERTOK>
 struct TcStage {
     static constexpr uint32_t IO = 64 * 64 * 2;                   // one bf16 array
-    static constexpr uint32_t W = PERTOK ? 64 * 64 * 4 : 0;       // the decays
-    static constexpr uint32_t BYTES = 3 * IO + W;
-    static constexpr uint32_t NST = PERTOK ? 2 : 1;               // ring stages
-    static constexpr int MINB = PERTOK ? 1 : 2;                   // CTAs per SM
-    static constexpr uint32_t BASE = (kTcTiles + 1023u) & ~1023u; // stages start 1024-byte aligned
-    static constexpr uint32_t SMEM = BASE + NST * BYTES;          // tiles, then the stages
+    static constexpr uint32_t BYTES = 3 * IO;                     // r, k, v of a window
+    static constexpr int MINB = 2;                                // CTAs per SM
+    static constexpr uint32_t BASE = (kTcTiles + 127u) & ~127u;   // the stage, 128-byte aligned
+    static constexpr uint32_t SMEM = BASE + BYTES;                // tiles, then the stage
+    static_assert(64 * 64 * 4 <= kTcTile, "a window's decays fit the state's tile");
 };
 constexpr uint32_t kTcCols = 256;                   // tensor memory columns allocated
 constexpr float kTcSpan = 60.f;                     // bound of |Lam_t - Lam_m| (natural units)
@@ -183,19 +183,20 @@ __device__ __forceinline__ int tc_block_len(int n, Rate rate) {
 }
 
 template <bool PERTOK>
-__global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
+__global__ void __launch_bounds__(kTcThreads, TcStage::MINB)
     wkv5_tc_kernel(const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
                    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw, const Wkv5Args A) {
-    using SG = TcStage<PERTOK>;
+    using SG = TcStage;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char* RT = smem;                  // R~ [t][i]; after batch 1: lo(K^)^T [i][s]
     unsigned char* KT = smem + kTcTile;        // K~ [s][i]; after batch 1: the masked scores [t][s]
     unsigned char* KH = smem + 2 * kTcTile;    // hi(K^)^T [i][s]
     unsigned char* VT = smem + 3 * kTcTile;    // V^T [j][s]
-    unsigned char* ST = smem + 4 * kTcTile;    // S0'^T [j][i] = e^{-Lam_m[i]} S0[i][j]
-    __shared__ __align__(8) uint64_t bar[2], full[2];
+    unsigned char* ST = smem + 4 * kTcTile;    // S0'^T [j][i] = e^{-Lam_m[i]} S0[i][j]; per-token decays [t][i]
+    __shared__ __align__(8) uint64_t bar[2], full[2];   // full[0]: r, k, v; full[1]: the decays
     __shared__ uint32_t tslot;
     __shared__ float s_u[64], s_eend[64], s_emid[64];
+    __shared__ float s_wq[PERTOK ? 4 : 1][64];   // per-token decays: sums over the window's quarters
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // staging: channel ci, tokens [16 qq, 16 qq + 16) of a block
@@ -215,17 +216,19 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // TMA of window wi's r, k, v (and w) into its stage
+    // TMA of window wi's r, k, v into the stage, and of its decays into the
+    // state's tile
     auto fetch = [&](int64_t wi) {
-        const uint32_t sidx = SG::NST == 2 ? static_cast<uint32_t>(wi & 1) : 0u;
-        unsigned char* st = smem + SG::BASE + sidx * SG::BYTES;
-        uint64_t* fb = &full[sidx];
-        mbar_expect_tx(fb, SG::BYTES);
+        unsigned char* st = smem + SG::BASE;
+        mbar_expect_tx(&full[0], SG::BYTES);
         const int x = static_cast<int>(ch0), y = static_cast<int>(wi * 64), z = static_cast<int>(b);
-        tma_load_3d(st, &tr, x, y, z, fb);
-        tma_load_3d(st + SG::IO, &tk, x, y, z, fb);
-        tma_load_3d(st + 2 * SG::IO, &tv, x, y, z, fb);
-        if (PERTOK) tma_load_3d(st + 3 * SG::IO, &tw, x, y, z, fb);
+        tma_load_3d(st, &tr, x, y, z, &full[0]);
+        tma_load_3d(st + SG::IO, &tk, x, y, z, &full[0]);
+        tma_load_3d(st + 2 * SG::IO, &tv, x, y, z, &full[0]);
+    };
+    auto fetch_w = [&](int64_t wi) {
+        mbar_expect_tx(&full[1], 64u * 64u * 4u);
+        tma_load_3d(ST, &tw, static_cast<int>(ch0), static_cast<int>(wi * 64), static_cast<int>(b), &full[1]);
     };
     if (tid == 0) {
         prefetch_tensormap(&tr);
@@ -238,6 +241,7 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
         mbar_init(&full[1], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fetch(0);
+        if (PERTOK) fetch_w(0);
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tslot)),
@@ -274,7 +278,8 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
                    aST = smem_u32(ST);
     uint32_t phase = 0;
     bool ok = true;
-    int64_t issued = 1, consumed = 0;   // windows whose copy was started / waited for
+    // windows whose copies were started / waited for (r, k, v; the decays)
+    int64_t issued = 1, consumed = 0, issued_w = PERTOK ? 1 : 0, consumed_w = 0;
 
     const float wc = PERTOK ? 0.f : A.w[ch0 + ci];
     // per-channel decays: the factors of consecutive tokens differ by e^{-+w}
@@ -282,27 +287,42 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
     for (int64_t w0 = 0; w0 < T && ok; w0 += 64) {
         const int wn = static_cast<int>(T - w0 < 64 ? T - w0 : 64);
         const int64_t wi = w0 / 64;
-        const uint32_t sidx = SG::NST == 2 ? static_cast<uint32_t>(wi & 1) : 0u;
-        const uint32_t spar = SG::NST == 2 ? static_cast<uint32_t>((wi >> 1) & 1) : static_cast<uint32_t>(wi & 1);
-        // two stages: the next window's copy starts now (the stage it
-        // overwrites was last read two windows ago)
-        if (SG::NST == 2 && w0 + 64 < T) {
-            if (tid == 0) fetch(wi + 1);
-            issued = wi + 2;
+        const uint32_t spar = static_cast<uint32_t>(wi & 1);
+        {
+            bool got = mbar_wait(&full[0], spar, kCopyWaitNs);
+            if (PERTOK) got = mbar_wait(&full[1], spar, kCopyWaitNs) && got;
+            ok = __syncthreads_and(got);
         }
-        ok = __syncthreads_and(mbar_wait(&full[sidx], spar, kCopyWaitNs));
         if (!ok) break;
         consumed = wi + 1;
-        const unsigned char* st = smem + SG::BASE + sidx * SG::BYTES;
+        consumed_w = PERTOK ? wi + 1 : 0;
+        const unsigned char* st = smem + SG::BASE;
         const __nv_bfloat16* sr = reinterpret_cast<const __nv_bfloat16*>(st);
         const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(st + SG::IO);
         const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(st + 2 * SG::IO);
-        const float* sw = reinterpret_cast<const float*>(st + 3 * SG::IO);
+        const float* sw = reinterpret_cast<const float*>(ST);
+        const float* gw = PERTOK ? A.w + (b * T + w0) * C + ch0 + ci : nullptr;
         // ---- block length for this window (the shortest any channel needs) ----
-        auto rate = [&](int t) -> float { return PERTOK ? sw[t * 64 + ci] : wc; };
+        auto rate_s = [&](int t) -> float { return PERTOK ? sw[t * 64 + ci] : wc; };
         int lm;
+        // a full window with per-token decays: each of a channel's four
+        // threads sums its quarter of the window once; blocks of 64 tokens
+        // need only the sums of the two halves, and the block's cumulative
+        // decays follow from the quarters
+        bool quarters = false;
+        float wq[4] = {0.f, 0.f, 0.f, 0.f};
+        if (PERTOK && wn == 64) {
+            float part = 0.f;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) part += sw[(16 * qq + q) * 64 + ci];
+            s_wq[PERTOK ? qq : 0][ci] = part;
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) wq[q] = s_wq[PERTOK ? q : 0][ci];
+            quarters = wq[0] + wq[1] <= kTcSpan && wq[2] + wq[3] <= kTcSpan;
+        }
         if (PERTOK) {
-            lm = tc_block_len(wn, rate);
+            lm = quarters ? 64 : tc_block_len(wn, rate_s);
         } else {
             // a constant rate: the longest half of a block (of bl tokens, the
             // last one possibly shorter) is ceil(bl / 2) tokens
@@ -317,6 +337,13 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
         // (The inter factor e^{-Lam_t} = e^{Lam_m - Lam_t} e^{-Lam_m} holds in
         // every block: in a block of one token both sides are 1.)
         const bool tame = L > 1;
+        // the decays: from the state's tile while it still holds them (a
+        // window of one block: its stage 1 reads them before it writes the
+        // state), else from global memory
+        const bool rate_smem = L == 64;
+        auto rate = [&](int t) -> float {
+            return PERTOK ? (rate_smem ? sw[t * 64 + ci] : __ldg(gw + static_cast<int64_t>(t) * C)) : wc;
+        };
 
         for (int b0 = 0; b0 < wn && ok; b0 += L) {
             const int bl = wn - b0 < L ? wn - b0 : L;   // tokens of this block
@@ -327,7 +354,12 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
             // Lam at the middle and at the end of the block, and at this
             // thread's first row, for channel ci
             float lam_mid = 0.f, lam_end = 0.f, lam_row = 0.f;
-            if (PERTOK) {
+            if (PERTOK && quarters && L == 64) {
+                lam_mid = wq[0] + wq[1];
+                lam_end = lam_mid + (wq[2] + wq[3]);
+                for (int q = 0; q < 4; ++q)
+                    if (q < qq) lam_row += wq[q];
+            } else if (PERTOK) {
                 for (int t = 0; t < bl; ++t) {
                     if (t == mid) lam_mid = lam_end;
                     if (t == 16 * qq) lam_row = lam_end;
@@ -431,6 +463,12 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
             }
             ok = __syncthreads_and(mbar_wait(&bar[0], phase, kCopyWaitNs));
             tc_fence_after();
+            // the products have read the state's tile: the next window's
+            // decays go there now
+            if (PERTOK && last_block && ok && w0 + 64 < T) {
+                if (tid == 0) fetch_w(wi + 1);
+                issued_w = wi + 2;
+            }
             // ---- stage 3: masked scores, lo(K^)^T ----
             {
                 // the bonus diagonal of rows R0 and R0 + 8 where this warp's
@@ -527,7 +565,7 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
             tc_fence_after();
             // one stage: the window's inputs are read (stage 1 and the lines
             // above of its last block); the next window's copy starts now
-            if (SG::NST == 1 && last_block && w0 + 64 < T) {
+            if (last_block && w0 + 64 < T) {
                 if (tid == 0) fetch(wi + 1);
                 issued = wi + 2;
             }
@@ -577,11 +615,8 @@ __global__ void __launch_bounds__(kTcThreads, TcStage<PERTOK>::MINB)
     // a wait that failed leaves copies started but not waited for: they
     // must land before this CTA's shared memory is released
     if (tid == 0) {
-        for (int64_t w = consumed; w < issued; ++w) {
-            const uint32_t si = SG::NST == 2 ? static_cast<uint32_t>(w & 1) : 0u;
-            const uint32_t sp = SG::NST == 2 ? static_cast<uint32_t>((w >> 1) & 1) : static_cast<uint32_t>(w & 1);
-            mbar_wait(&full[si], sp, kCopyWaitNs);
-        }
+        for (int64_t w = consumed; w < issued; ++w) mbar_wait(&full[0], static_cast<uint32_t>(w & 1), kCopyWaitNs);
+        for (int64_t w = consumed_w; w < issued_w; ++w) mbar_wait(&full[1], static_cast<uint32_t>(w & 1), kCopyWaitNs);
     }
     if (A.s_out != nullptr) {
 #pragma unroll

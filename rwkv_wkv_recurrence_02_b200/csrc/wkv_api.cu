@@ -1475,7 +1475,7 @@ int launch_wkv5(const wkv::Wkv5Args& a, cudaStream_t st) {
 // threads per (sequence, head).
 template <bool PERTOK>
 int launch_wkv5_tc(const wkv::Wkv5Args& a, cudaStream_t st) {
-    using SG = wkv::TcStage<PERTOK>;
+    using SG = wkv::TcStage;
     auto kern = wkv::wkv5_tc_kernel<PERTOK>;
     static bool ready[kMaxDevices] = {false};
     int dev = 0;
@@ -1485,8 +1485,8 @@ int launch_wkv5_tc(const wkv::Wkv5Args& a, cudaStream_t st) {
     if (!ready[dev]) {
         rc = record_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SG::SMEM));
         if (rc != WKV_OK) return rc;
-        // all of the unified L1 / shared memory as shared memory, so that the
-        // per-channel-decay kernel's two CTAs fit on one SM
+        // all of the unified L1 / shared memory as shared memory, so that two
+        // CTAs fit on one SM
         rc = record_cuda(
             cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared));
         if (rc != WKV_OK) return rc;
