@@ -6,7 +6,9 @@ for the bf16 outputs, 2e-5 of the head's largest |S| for the state.
 
 Decays large enough that a 64-token block would leave the range of its
 factors make the kernel cut windows into blocks of 16, 4 or 1 token; those
-cases are pinned here too, as are ragged windows, the carried state and the
+cases are pinned here too, as are windows of one sequence that alternate
+between the two (per-token decays staged in the state's tile, or read from
+global memory), ragged windows, the carried state and the
 fallback to the recurrent kernel for outputs it cannot store 16 bytes at a
 time, and the full layer workloads.  The cases run in a child process, and
 the same cases with WKV5_KERNEL=recurrent keep the CUDA-core recurrence
@@ -59,6 +61,19 @@ for wmax, v6 in [(5.0, False), (20.0, False), (200.0, False), (12.0, True), (300
     y, s = run(d, H)
     res.append(("decay", check(d, H, y, s, TOL[BF])))
 
+# per-token decays large in some windows only: a sequence's windows alternate between blocks of 64 tokens (the
+# decays staged in the state's tile, the quarter sums) and shorter blocks (the decays read from global memory),
+# while the other sequence keeps 64-token blocks throughout; the last window is ragged
+B, T, C, H = 2, 5 * 64 + 17, 128, 2
+d = case(B, T, C, H, BF, True, True, seed=71)
+w = d["w"].clone()
+w[1, 64:128] = 40.0          # sequence 1, window 1: blocks of one token
+w[1, 192:256, :64] = 3.0     # window 3, head 0: blocks of 16
+w[1, 320:, 64:] = 2.5        # the ragged last window, head 1
+d["w"] = w.contiguous()
+y, s = run(d, H)
+res.append(("mixed", check(d, H, y, s, TOL[BF])))
+
 # calls of 1, 63, 64, 65 and 307 tokens chained in place, and one call
 B, T, C, H = 2, 500, 128, 2
 d = case(B, T, C, H, BF, True, True, seed=61)
@@ -108,4 +123,4 @@ def test_matrix_state_kernels_match_the_oracle(kernel):
     r = subprocess.run([sys.executable, "-c", CHILD.replace("@ROOT@", repr(ROOT))], env=env, capture_output=True,
                        text=True, timeout=900, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-3000:]
-    assert r.stdout.count("OK ") == 6 + 5 + 1 + 1 + 8, r.stdout
+    assert r.stdout.count("OK ") == 6 + 5 + 1 + 1 + 1 + 8, r.stdout
