@@ -280,7 +280,9 @@ EncodeTiledFn encode_fn() {
 
 // 3-D map over a (B, T, C) array: box = CB channels x TT tokens x 1 sequence.
 // Coordinates past T or C read as zeros.
-bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t T, int64_t C, int CB, int TT) {
+// promo: the L2 sector promotion of the copies (256 bytes unless given).
+bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t T, int64_t C, int CB, int TT,
+                CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     const cuuint64_t eb = elem_bytes(dtype);
@@ -290,8 +292,7 @@ bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t T
     const cuuint32_t es[3] = {1, 1, 1};
     return fn(m, dtype == WKV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
               const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_SWIZZLE_NONE, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // TMA needs 16-byte aligned bases and row strides, and coordinates in int32.
@@ -380,11 +381,16 @@ int launch_lane(wkv::ChunkArgs a, int dtype, void* workspace, size_t workspace_b
         capacity[dev] = per_sm * sm_count();
     }
     CUtensorMap tk, tv, tr;
-    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
-        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT))
+    // CTAs that split lane blocks read neighbouring lane blocks' rows at
+    // different times: L2 fetches of a row's width (128 bytes for bfloat16)
+    // waste no DRAM bandwidth on bytes evicted before their CTA reads them
+    const CUtensorMapL2promotion promo =
+        G::ROW >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT, promo) ||
+        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT, promo))
         return WKV_ERR_CUDA;
     if (GATE) {
-        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT)) return WKV_ERR_CUDA;
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT, promo)) return WKV_ERR_CUDA;
     } else {
         tr = tv;
     }
@@ -1282,13 +1288,19 @@ int launch_backward(wkv::BwdArgs a, int dtype, void* workspace, cudaStream_t st)
         a.hdr = nullptr;
         a.incw = nullptr;
     }
+    // The walk visits neighbouring lane blocks at different times when CTAs
+    // split them, so an L2 fetch wider than a tile row brings in bytes no CTA
+    // reads before they are evicted: promote to the row's width (128 bytes
+    // for bfloat16), not 256 bytes.
+    const CUtensorMapL2promotion promo =
+        G::ROW >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
     CUtensorMap tk, tv, tdy, tr;
-    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
-        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT) ||
-        !encode_map(&tdy, a.dy, dtype, a.B, a.T, a.C, G::CB, G::TT))
+    if (!encode_map(&tk, a.k, dtype, a.B, a.T, a.C, G::CB, G::TT, promo) ||
+        !encode_map(&tv, a.v, dtype, a.B, a.T, a.C, G::CB, G::TT, promo) ||
+        !encode_map(&tdy, a.dy, dtype, a.B, a.T, a.C, G::CB, G::TT, promo))
         return WKV_ERR_CUDA;
     if (GATE) {
-        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT)) return WKV_ERR_CUDA;
+        if (!encode_map(&tr, a.r, dtype, a.B, a.T, a.C, G::CB, G::TT, promo)) return WKV_ERR_CUDA;
     } else {
         tr = tk;
     }
