@@ -39,7 +39,8 @@ def run(d, H, **kw):
     return y, s
 
 # shapes: one token, one window, ragged windows, carried states, 64 windows
-for (B, T, C, H, v6, st) in [(1, 1, 64, 1, False, False), (1, 64, 64, 1, True, True), (2, 63, 128, 2, False, True),
+for (B, T, C, H, v6, st) in [(1, 1, 64, 1, False, False), (1, 1, 64, 1, True, True), (1, 64, 64, 1, True, True),
+                            (2, 63, 128, 2, False, True),
                             (3, 200, 256, 4, True, True), (2, 1000, 512, 8, False, False),
                             (1, 4096, 128, 2, True, True)]:
     d = case(B, T, C, H, BF, v6, st, seed=B * 5 + T + C)
@@ -123,4 +124,4 @@ def test_matrix_state_kernels_match_the_oracle(kernel):
     r = subprocess.run([sys.executable, "-c", CHILD.replace("@ROOT@", repr(ROOT))], env=env, capture_output=True,
                        text=True, timeout=900, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-3000:]
-    assert r.stdout.count("OK ") == 6 + 5 + 1 + 1 + 1 + 8, r.stdout
+    assert r.stdout.count("OK ") == 7 + 5 + 1 + 1 + 1 + 8, r.stdout
